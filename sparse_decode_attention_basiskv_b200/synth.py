@@ -1,0 +1,304 @@
+"""Seeded synthetic workloads for the BasisKV decode-attention block.
+
+This module only draws random numbers and lays data out; it contains none of
+the method's own arithmetic (no append projection, no routing, no selection,
+no attention, no out-projection).  Both the CUDA path (through the C-ABI) and
+the CPU oracle receive the tensors produced here.
+
+Input recipe (BasisKV, "Value Latents for Communication and Key Routing":
+per-token state of Table 4; model shapes of Figure 3's caption):
+
+* Factors, per KV head g, drawn on the CPU from ``torch.Generator(seed)`` in
+  this order: A_V [d][r_v] ~ N(0, 1/d); P_K [r_v][d] ~ N(0, 1/r_v);
+  U_K [d][r_k] = Q of a QR of an N(0,1) matrix (columns orthonormal, the sign
+  of each column fixed so diag(R) > 0); B_V [r_v][d] ~ N(0, 1/r_v);
+  W_O [Hq*d][hidden] ~ N(0, 1/(Hq*d)).  Every factor is rounded to bf16 once.
+* Cache contents for tokens t < T of every (sequence b, KV head g), drawn
+  with ``torch.Generator(device).manual_seed(seed*1000 + 1)``: z ~ N(0,1),
+  e ~ N(0,1) (both bf16), and the exact key
+  K = z.P_K + e.U_K^T + N(0, 0.1^2), rounded to bf16.  This makes part of
+  each key predictable from the Value latent, the structure BasisKV's router
+  relies on.  Slots at t >= T hold a large finite filler so that a kernel
+  that forgets the length mask is caught.
+* Planted pages and queries (CPU generator seed*1000 + 2 for the choices):
+  per (b, g) ``n_planted`` distinct pages from 1..P-2; each query head h of
+  group g sums the keys of one uniform token in each of 2 distinct planted
+  pages of its group, plus N(0, 0.1^2) noise.  Retrieval-style attention:
+  the planted pages should win the routing.
+* New tokens for decode step ``s`` (generator seed*1000 + 3 + s on the
+  device): v ~ N(0,1); k = (v.A_V).P_K + e'.U_K^T + N(0, 0.1^2) with
+  e' ~ N(0,1); both bf16.  The same recipe draws a prefill chunk.
+* Paging: physical pages are a random permutation (CPU generator
+  seed*1000 + 4) of ``B * pages_capacity`` slots, so every logical page is
+  fetched through the block table from a scattered location.
+
+The public benchmarks of the pages (RULER, LongBench, ...) need datasets and
+trained checkpoints; these synthetic inputs stand in for them at the pages'
+model shapes (Llama-3.1-8B and Qwen3-32B attention layers).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field, replace
+
+import torch
+
+FILLER = 64.0  # value stored in cache slots beyond a sequence's length
+
+
+@dataclass(frozen=True)
+class Workload:
+    """Shape and seed of one synthetic decode-attention workload."""
+
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    hidden: int
+    T: int
+    page_size: int
+    r_v: int
+    r_k: int
+    top_k: int
+    n_planted: int
+    seed: int
+    append_tokens: int = 0  # decode tokens appended per sequence per step
+    prefill_tokens: int = 0  # tokens of one prefill chunk (sequence 0)
+    layers: int = 1
+    steps: int = 1
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def pages(self) -> int:
+        return -(-self.T // self.page_size)
+
+    def capacity_tokens(self) -> int:
+        """Token slots per sequence: context plus every token appended."""
+        return self.T + self.append_tokens * self.steps + self.prefill_tokens
+
+    def pages_capacity(self) -> int:
+        return -(-self.capacity_tokens() // self.page_size)
+
+    def describe(self) -> dict:
+        return {k: getattr(self, k) for k in (
+            "name", "B", "Hq", "Hkv", "d", "hidden", "T", "page_size", "r_v",
+            "r_k", "top_k", "append_tokens", "prefill_tokens", "layers",
+            "steps")}
+
+
+# The five workloads.  Names say what they are; sizes follow the pages' model
+# shapes (Llama-3.1-8B: 32 query / 8 KV heads, d 128, hidden 4096; Qwen3-32B:
+# 64 query / 8 KV heads, hidden 5120) and Value widths V96 / V64.
+TINY = Workload("tiny_b1_t512", B=1, Hq=4, Hkv=1, d=64, hidden=256, T=512,
+                page_size=16, r_v=32, r_k=16, top_k=8, n_planted=2, seed=0)
+LLAMA8B_T4K = Workload("llama8b_layer_b1_t4k_v96", B=1, Hq=32, Hkv=8, d=128,
+                       hidden=4096, T=4096, page_size=16, r_v=96, r_k=32,
+                       top_k=64, n_planted=8, seed=1)
+LLAMA8B_T32K_B16 = Workload("llama8b_layer_b16_t32k_v64_append1", B=16, Hq=32,
+                            Hkv=8, d=128, hidden=4096, T=32768, page_size=16,
+                            r_v=64, r_k=32, top_k=128, n_planted=8, seed=2,
+                            append_tokens=1)
+QWEN32B_T64K_B8 = Workload("qwen32b_layer_b8_t64k_v96_prefill4k", B=8, Hq=64,
+                           Hkv=8, d=128, hidden=5120, T=65536, page_size=32,
+                           r_v=96, r_k=32, top_k=64, n_planted=8, seed=3,
+                           prefill_tokens=4096)
+
+
+def sweep_point(B: int, T: int, r_v: int, layers: int = 32,
+                steps: int = 128) -> Workload:
+    """One point of the 32-layer decode sweep at the Llama-3.1-8B layer shape:
+    top-k = T/64 pages of 16 tokens (a quarter of the context), one token
+    appended per sequence per step."""
+    return Workload(f"llama8b_sweep_b{B}_t{T // 1024}k_v{r_v}", B=B, Hq=32,
+                    Hkv=8, d=128, hidden=4096, T=T, page_size=16, r_v=r_v,
+                    r_k=32, top_k=T // 64, n_planted=8, seed=4,
+                    append_tokens=1, layers=layers, steps=steps)
+
+
+SWEEP = [sweep_point(B, T, r_v) for B in (1, 8, 32, 64)
+         for T in (4096, 32768, 131072) for r_v in (96, 64)]
+
+WORKLOADS = {w.name: w for w in (TINY, LLAMA8B_T4K, LLAMA8B_T32K_B16,
+                                  QWEN32B_T64K_B8)}
+
+
+def _bf16(x: torch.Tensor) -> torch.Tensor:
+    return x.to(torch.bfloat16)
+
+
+def make_factors(wl: Workload, layer: int = 0) -> dict:
+    """Per-KV-head factors and W_O, drawn on the CPU (device independent)."""
+    g = torch.Generator().manual_seed(wl.seed * 7919 + layer)
+    Hkv, d, r_v, r_k = wl.Hkv, wl.d, wl.r_v, wl.r_k
+    A_V = torch.randn(Hkv, d, r_v, generator=g, dtype=torch.float64) / math.sqrt(d)
+    P_K = torch.randn(Hkv, r_v, d, generator=g, dtype=torch.float64) / math.sqrt(r_v)
+    raw = torch.randn(Hkv, d, r_k, generator=g, dtype=torch.float64)
+    U_K = torch.empty_like(raw)
+    for h in range(Hkv):
+        qm, rm = torch.linalg.qr(raw[h])
+        U_K[h] = qm * torch.sign(torch.diagonal(rm)).unsqueeze(0)
+    B_V = torch.randn(Hkv, r_v, d, generator=g, dtype=torch.float64) / math.sqrt(r_v)
+    W_O = torch.randn(wl.Hq * d, wl.hidden, generator=g,
+                      dtype=torch.float64) / math.sqrt(wl.Hq * d)
+    return {"A_V": _bf16(A_V), "P_K": _bf16(P_K), "U_K": _bf16(U_K),
+            "B_V": _bf16(B_V), "W_O": _bf16(W_O)}
+
+
+def _dev_gen(device, seed: int) -> torch.Generator:
+    return torch.Generator(device=device).manual_seed(seed)
+
+
+def make_cache(wl: Workload, factors: dict, device="cpu", layer: int = 0) -> dict:
+    """Logical caches [B][Hkv][capacity][*] holding T tokens per sequence."""
+    dev = torch.device(device)
+    gen = _dev_gen(dev, wl.seed * 1000 + 1 + 100003 * layer)
+    B, Hkv, T, cap = wl.B, wl.Hkv, wl.T, wl.capacity_tokens()
+    P_K = factors["P_K"].to(dev, torch.float32)
+    U_K = factors["U_K"].to(dev, torch.float32)
+    Z = torch.full((B, Hkv, cap, wl.r_v), FILLER, dtype=torch.bfloat16, device=dev)
+    E = torch.full((B, Hkv, cap, wl.r_k), FILLER, dtype=torch.bfloat16, device=dev)
+    K = torch.full((B, Hkv, cap, wl.d), FILLER, dtype=torch.bfloat16, device=dev)
+    for b in range(B):  # one sequence at a time bounds the fp32 temporaries
+        z = torch.randn(Hkv, T, wl.r_v, generator=gen, device=dev).bfloat16()
+        e = torch.randn(Hkv, T, wl.r_k, generator=gen, device=dev).bfloat16()
+        noise = torch.randn(Hkv, T, wl.d, generator=gen, device=dev) * 0.1
+        k = torch.bmm(z.float(), P_K) + torch.bmm(e.float(), U_K.transpose(1, 2)) + noise
+        Z[b, :, :T] = z
+        E[b, :, :T] = e
+        K[b, :, :T] = k.bfloat16()
+    return {"Z": Z, "E": E, "K": K}
+
+
+def planted_pages(wl: Workload, P: int | None = None) -> torch.Tensor:
+    """[B][Hkv][n_planted] distinct pages drawn from 1..P-2 (CPU)."""
+    P = wl.pages if P is None else P
+    g = torch.Generator().manual_seed(wl.seed * 1000 + 2)
+    n = min(wl.n_planted, max(P - 2, 0))
+    out = torch.empty(wl.B, wl.Hkv, n, dtype=torch.int64)
+    for b in range(wl.B):
+        for h in range(wl.Hkv):
+            out[b, h] = torch.randperm(P - 2, generator=g)[:n] + 1
+    return out
+
+
+def make_query(wl: Workload, K: torch.Tensor, T: int, step: int = 0) -> tuple:
+    """Planted queries q [B][Hq][d] (bf16) built from cached keys.
+
+    Returns (q, used) where used[b][h] lists the two planted pages that
+    query head h drew from."""
+    dev = K.device
+    P = -(-T // wl.page_size)
+    planted = planted_pages(wl, P)
+    g = torch.Generator().manual_seed(wl.seed * 1000 + 2 + 7 * (step + 1))
+    gen = _dev_gen(dev, wl.seed * 1000 + 5 + step)
+    S = wl.page_size
+    q = torch.empty(wl.B, wl.Hq, wl.d, dtype=torch.float32, device=dev)
+    used = torch.zeros(wl.B, wl.Hq, 2, dtype=torch.int64)
+    for b in range(wl.B):
+        for h in range(wl.Hq):
+            grp = h // wl.G
+            cand = planted[b, grp]
+            if len(cand) >= 2:
+                pick = cand[torch.randperm(len(cand), generator=g)[:2]]
+            else:  # too few pages to plant: any two tokens of the context
+                pick = torch.tensor([0, P - 1])
+            acc = torch.zeros(wl.d, dtype=torch.float32, device=dev)
+            for j, p in enumerate(pick.tolist()):
+                lo, hi = p * S, min((p + 1) * S, T)
+                t = lo + int(torch.randint(hi - lo, (1,), generator=g))
+                acc += K[b, grp, t].float()
+                used[b, h, j] = p
+            q[b, h] = acc
+    q += torch.randn(q.shape, generator=gen, device=dev) * 0.1
+    return q.bfloat16(), used
+
+
+def make_tokens(wl: Workload, factors: dict, n: int, device="cpu",
+                stream_id: int = 0) -> tuple:
+    """n new tokens per sequence: (k, v) each [B][n][Hkv][d] bf16."""
+    dev = torch.device(device)
+    gen = _dev_gen(dev, wl.seed * 1000 + 3 + stream_id)
+    A_V = factors["A_V"].to(dev, torch.float32)
+    P_K = factors["P_K"].to(dev, torch.float32)
+    U_K = factors["U_K"].to(dev, torch.float32)
+    B, Hkv, d = wl.B, wl.Hkv, wl.d
+    v = torch.randn(B, n, Hkv, d, generator=gen, device=dev).bfloat16()
+    ep = torch.randn(B, n, Hkv, wl.r_k, generator=gen, device=dev)
+    noise = torch.randn(B, n, Hkv, d, generator=gen, device=dev) * 0.1
+    lat = torch.einsum("bnhd,hdr->bnhr", v.float(), A_V)
+    k = (torch.einsum("bnhr,hrd->bnhd", lat, P_K)
+         + torch.einsum("bnhr,hdr->bnhd", ep, U_K) + noise)
+    return k.bfloat16(), v
+
+
+def block_table(wl: Workload, device="cpu") -> torch.Tensor:
+    """[B][pages_capacity] int32 logical->physical page map (a permutation)."""
+    pc = wl.pages_capacity()
+    g = torch.Generator().manual_seed(wl.seed * 1000 + 4)
+    perm = torch.randperm(wl.B * pc, generator=g).to(torch.int32)
+    return perm.view(wl.B, pc).to(device)
+
+
+def paginate(logical: torch.Tensor, table: torch.Tensor, page_size: int,
+             num_phys: int) -> torch.Tensor:
+    """Scatter a logical cache [B][Hkv][cap][r] into the paged layout
+    [num_phys][Hkv][page_size][r] through the block table."""
+    B, Hkv, cap, r = logical.shape
+    pc = table.shape[1]
+    pad = pc * page_size - cap
+    if pad:
+        logical = torch.cat([logical, torch.full((B, Hkv, pad, r), FILLER,
+                            dtype=logical.dtype, device=logical.device)], 2)
+    tiles = logical.view(B, Hkv, pc, page_size, r).permute(0, 2, 1, 3, 4)
+    out = torch.full((num_phys, Hkv, page_size, r), FILLER, dtype=logical.dtype,
+                     device=logical.device)
+    out[table.long().reshape(-1).to(logical.device)] = tiles.reshape(B * pc, Hkv, page_size, r)
+    return out
+
+
+def logical_view(paged: torch.Tensor, table: torch.Tensor, b: int, g: int,
+                 n_tokens: int) -> torch.Tensor:
+    """Gather tokens [0, n_tokens) of (sequence b, KV head g) from a paged
+    cache, in logical order (used to hand the CUDA path's outputs to a
+    comparison)."""
+    S = paged.shape[2]
+    n_pages = -(-n_tokens // S)
+    phys = table[b, :n_pages].long().to(paged.device)
+    return paged[phys, g].reshape(n_pages * S, -1)[:n_tokens]
+
+
+@dataclass
+class Problem:
+    """Everything one decode-attention workload needs, on one device."""
+
+    wl: Workload
+    factors: dict
+    cache: dict
+    table: torch.Tensor
+    seq_lens: torch.Tensor
+    q: torch.Tensor
+    used_pages: torch.Tensor
+    extra: dict = field(default_factory=dict)
+
+    def paged(self) -> dict:
+        n = self.wl.B * self.wl.pages_capacity()
+        return {k: paginate(v, self.table.to(v.device), self.wl.page_size, n)
+                for k, v in self.cache.items()}
+
+
+def make_problem(wl: Workload, device="cpu", layer: int = 0) -> Problem:
+    factors = make_factors(wl, layer)
+    cache = make_cache(wl, factors, device, layer)
+    table = block_table(wl, device)
+    seq_lens = torch.full((wl.B,), wl.T, dtype=torch.int32, device=device)
+    q, used = make_query(wl, cache["K"], wl.T)
+    return Problem(wl, factors, cache, table, seq_lens, q, used)
+
+
+def with_sizes(wl: Workload, **kw) -> Workload:
+    """A copy of a workload with some sizes changed (ragged / edge cases)."""
+    return replace(wl, **kw)
