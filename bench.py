@@ -1,0 +1,415 @@
+"""Benchmark of the BasisKV decode-attention block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Workload (one step): the Llama-3.1-8B attention-layer shape at Value width 64,
+B = 16 sequences, 32K-token context, page 16, top-k 128 pages: one fused
+``basiskv_decode`` that appends one token per sequence, routes over the full
+context, attends over the selected pages and out-projects.  The context grows
+by one token per step (32768 -> 32768 + W + K); the algorithmic bytes are
+counted per step from the actual length.
+
+Metric: achieved HBM TB/s = algorithmic bytes / device time (higher is
+better), with microseconds per step beside it.  Algorithmic bytes per step:
+  route   B*Hkv*T*(r_v+r_k)*2          z and e of the whole context
+  attend  B*Hkv*min(k,P)*S*(d+r_v)*2   exact K and z of the selected pages
+  outproj Hq*r_v*H*2                   the folded out-projection W'
+  small   q, y, appended token state, folded queries, scores, selection,
+          latent outputs, and the factors read by the fold / append kernels.
+Inputs are far larger than L2 (about 1.9 GB of cache per step), so no L2
+flush is needed between steps.
+
+With N > 1 (torchrun) every rank runs an independent replica ("replicas
+only": sequences are independent and the single-GPU path has no exchange);
+the value is the bytes of all ranks over the slowest rank's time.
+
+``--impl reference`` times the CPU oracle (float64 numpy) on rank 0 on a
+bounded sample of the same workload: one (sequence, KV head) group per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from sparse_decode_attention_basiskv_b200 import synth  # noqa: E402
+
+METRIC = "BasisKV decode µs/step & achieved HBM TB/s vs peak (Llama-8B shape, 32K ctx)"
+WL = synth.LLAMA8B_T32K_B16
+N_QUERIES = 4  # distinct planted query sets cycled over the steps
+
+
+def algorithmic_bytes(wl, T: int, append: bool = True) -> dict:
+    """Bytes one decode step must move at context length T (after append)."""
+    S = wl.page_size
+    P = -(-T // S)
+    sel = min(wl.top_k, P)
+    route = wl.B * wl.Hkv * T * (wl.r_v + wl.r_k) * 2
+    attend = wl.B * wl.Hkv * sel * S * (wl.d + wl.r_v) * 2
+    outproj = wl.Hq * wl.r_v * wl.hidden * 2
+    small = (wl.B * wl.Hq * wl.d * 2                      # q (fold + attend)
+             + wl.B * wl.hidden * 2                       # y
+             + wl.B * wl.Hq * (wl.r_v + wl.r_k) * 4 * 2   # folded queries w + r
+             + wl.B * wl.Hkv * P * 4 * 2                  # scores w + r
+             + wl.B * wl.Hkv * wl.top_k * 4 * 2           # selection w + r
+             + wl.B * wl.Hq * wl.r_v * 2 * 2              # latent a (bf16) w + r
+             + wl.Hkv * (wl.r_v + wl.r_k) * wl.d * 2)     # P_K, U_K for the fold
+    if append:
+        small += (wl.B * wl.Hkv * (2 * wl.d + wl.d + wl.r_v + wl.r_k) * 2
+                  + wl.Hkv * wl.d * wl.r_v * 2)           # k, v in; K, z, e out; A_V
+    return {"route": route, "attend": attend, "outproj": outproj, "small": small,
+            "total": route + attend + outproj + small}
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                mhz.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------ oracle
+def oracle_sample(wl, device_cache=None):
+    """Inputs of one (sequence 0, KV head 0) group on the CPU, float64."""
+    import numpy as np
+    factors = synth.make_factors(wl)
+    cache = synth.make_cache(wl, factors, "cpu", seqs=[0])
+    q, _ = synth.make_query(wl, cache["K"], wl.T)
+    k, v = synth.make_tokens(wl, factors, 1, "cpu")
+    f = {n: t.double().numpy() for n, t in factors.items()}
+    c = {n: t[0, 0].double().numpy() for n, t in cache.items()}
+    return {"f": f, "c": c, "q": q[0, :wl.G].double().numpy(),
+            "k": k[0, 0, 0].double().numpy(), "v": v[0, 0, 0].double().numpy(), "np": np}
+
+
+def oracle_group_step(wl, s) -> None:
+    """One decode step of one group through the oracle: append, route,
+    select, attend, and the group's share of the out-projection."""
+    from oracle import basiskv_oracle as O
+    np = s["np"]
+    f, c = s["f"], s["c"]
+    T = wl.T
+    z, e = O.append_latents(s["k"][None], s["v"][None], f["A_V"][0], f["P_K"][0], f["U_K"][0])
+    Z = c["Z"].copy()
+    E = c["E"].copy()
+    K = c["K"].copy()
+    Z[T], E[T], K[T] = O.to_bf16(z[0]), O.to_bf16(e[0]), s["k"]
+    sc = O.page_scores(s["q"], Z, E, f["P_K"][0], f["U_K"][0], T + 1, wl.page_size)
+    sel, _ = O.select_pages(sc, wl.top_k)
+    a, _ = O.attend(s["q"], K, Z, sel, T + 1, wl.page_size)
+    W = O.fold_outproj(f["B_V"][:1], f["W_O"][:wl.G * wl.d], wl.G)
+    O.outproj(a, W)
+
+
+def oracle_bytes_per_group(wl) -> int:
+    one = synth.with_sizes(wl, B=1, Hkv=1, Hq=wl.G)
+    return algorithmic_bytes(one, wl.T + 1)["total"]
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:  # noqa: BLE001
+        return os.cpu_count()
+
+
+def cpu_baseline(wl, budget_s: float = 12.0) -> dict:
+    s = oracle_sample(wl)
+    oracle_group_step(wl, s)  # warm
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s or n == 0:
+        oracle_group_step(wl, s)
+        n += 1
+    dt = (time.perf_counter() - t0) / n
+    groups = wl.B * wl.Hkv
+    return {"value": oracle_bytes_per_group(wl) / dt / 1e12, "unit": "TB/s",
+            "cores": blas_threads(), "kind": "oracle",
+            "us_per_step_equiv": dt * groups * 1e6,
+            "sample": (f"{n} decode steps of one (sequence, KV head) group (1/{groups} of the "
+                       f"step; float64 numpy oracle), {dt * 1e3:.1f} ms each")}
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = synth.with_sizes(WL, steps=args.steps + args.warmup)
+    s = oracle_sample(wl)
+    for _ in range(args.warmup):
+        oracle_group_step(wl, s)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_group_step(wl, s)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = oracle_bytes_per_group(wl) / dt / 1e12
+    groups = wl.B * wl.Hkv
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * groups * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": WL.name, **{k: v for k, v in WL.describe().items()
+                                                if k != "name"}},
+            "cpu_baseline": {"kind": "oracle", "cores": blas_threads(), "value": value,
+                             "unit": "TB/s",
+                             "sample": "one (sequence, KV head) group per step, scaled "
+                                       f"x{groups} for ms_per_step"},
+            "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_gpu(args) -> None:
+    import sparse_decode_attention_basiskv_b200 as bkv
+    from sparse_decode_attention_basiskv_b200.layer import DecodeLayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    K, W = args.steps, args.warmup
+    wl = synth.with_sizes(WL, steps=K + W)
+    pb = synth.make_problem(wl, device="cuda")
+    layer = DecodeLayer.from_problem(pb)
+    T0 = wl.T
+    queries = [synth.make_query(wl, pb.cache["K"], T0, step=i)[0] for i in range(N_QUERIES)]
+    k_all, v_all = synth.make_tokens(wl, pb.factors, K + W, device="cuda")
+    k_steps = [k_all[:, i].contiguous() for i in range(K + W)]
+    v_steps = [v_all[:, i].contiguous() for i in range(K + W)]
+    del pb.cache
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream()
+
+    def step(i, T_after):
+        layer.decode(queries[i % N_QUERIES], k_steps[i], v_steps[i], max_seq_len=T_after)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ------------------------------------------------ device-timed region
+    for i in range(W):
+        step(i, T0 + i + 1)
+    barrier()
+    assert bkv.read_device_status() == 0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = bkv.launch_count()
+    with ClockSampler(local) as clocks:
+        barrier()
+        ev0.record(stream)
+        for i in range(W, W + K):
+            step(i, T0 + i + 1)
+        ev1.record(stream)
+        barrier()
+    launches = bkv.launch_count() - launches0
+    ms = ev0.elapsed_time(ev1)
+    assert bkv.read_device_status() == 0
+    ms_t = torch.tensor([ms], device="cuda")
+    if dist is not None:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    bytes_steps = [algorithmic_bytes(wl, T0 + i + 1) for i in range(W, W + K)]
+    total_bytes = sum(b["total"] for b in bytes_steps)
+    value = world * total_bytes / (ms_max / 1e3) / 1e12
+    ms_per_step = ms_max / K
+
+    # ------------------------------ roofline: the routing stage, timed alone
+    layer.seq_lens.fill_(T0 + W + K)
+    T_r = T0 + W + K
+    sel = torch.empty(wl.B, wl.Hkv, wl.top_k, dtype=torch.int32, device="cuda")
+    reps = max(20, min(200, K))
+    for _ in range(3):
+        bkv.basiskv_route(layer.dims, queries[0], layer.seq_lens, T_r, layer.block_table,
+                          layer.P_K, layer.U_K, layer.Z, layer.E, wl.top_k, None, sel,
+                          layer.workspace)
+    torch.cuda.synchronize()
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    for _ in range(reps):
+        bkv.basiskv_route(layer.dims, queries[0], layer.seq_lens, T_r, layer.block_table,
+                          layer.P_K, layer.U_K, layer.Z, layer.E, wl.top_k, None, sel,
+                          layer.workspace)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    route_ms = r0.elapsed_time(r1) / reps
+    route_bytes = wl.B * wl.Hkv * T_r * (wl.r_v + wl.r_k) * 2
+    peak, peak_kind = measured_peak()
+    achieved = route_bytes / (route_ms / 1e3) / 1e9
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "route_traffic.json")
+    if os.path.exists(tr_path):
+        with open(tr_path) as f:
+            tr = json.load(f)
+        if tr.get("kernel_source_sha") == _route_source_sha():
+            traffic = tr["bytes_per_launch_scaled"]
+
+    # ------------------------------------ end to end through the public API
+    layer.seq_lens.fill_(T0)
+    q_h = [q.cpu().pin_memory() for q in queries]
+    k_h = [k.cpu().pin_memory() for k in k_steps]
+    v_h = [v.cpu().pin_memory() for v in v_steps]
+    q_d = torch.empty_like(queries[0])
+    k_d = torch.empty_like(k_steps[0])
+    v_d = torch.empty_like(v_steps[0])
+    y_h = torch.empty(wl.B, wl.hidden, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step(i, T_after):
+        q_d.copy_(q_h[i % N_QUERIES], non_blocking=True)
+        k_d.copy_(k_h[i], non_blocking=True)
+        v_d.copy_(v_h[i], non_blocking=True)
+        y = layer.decode(q_d, k_d, v_d, max_seq_len=T_after)
+        y_h.copy_(y, non_blocking=True)
+
+    for i in range(W):
+        e2e_step(i, T0 + i + 1)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(W, W + K):
+        e2e_step(i, T0 + i + 1)
+    e1.record(stream)
+    barrier()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], device="cuda")
+    if dist is not None:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = world * total_bytes / (float(e2e_ms.item()) / 1e3) / 1e12
+    h2d = (queries[0].numel() + k_steps[0].numel() + v_steps[0].numel()) * 2
+    d2h = wl.B * wl.hidden * 2
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    cpu = cpu_baseline(wl) if world == 1 and not args.no_cpu_baseline else None
+    avg = {k: sum(b[k] for b in bytes_steps) / K for k in bytes_steps[0]}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
+        "tokens_per_s": world * wl.B / (ms_per_step / 1e3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generators; planted-page queries)",
+        "config": {"workload": WL.name, "global_batch": wl.B * world, "seq_len": T0,
+                   "context": f"{T0} -> {T0 + W + K} tokens (one appended per step)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (~1.9 GB of cache per step); no flush",
+                   **{k: v for k, v in WL.describe().items() if k not in ("name", "steps")}},
+        "bytes_per_step": avg,
+        "frac_of_peak": value / world / (peak / 1e3),
+        "roofline": {"bound": "hbm", "kernel": "route (fold + page scoring + select)",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                     "ms_per_launch": route_ms, "algorithmic_bytes": route_bytes},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TB/s", "us_per_step": float(e2e_ms.item()) / K * 1e3,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _route_source_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for n in ("route.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "sparse_decode_attention_basiskv_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -53,8 +53,9 @@ def to_bf16(x) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
-# (1) cache append — abstract ("Value compression"; Key-specific residual
-#     "stores what cannot be recovered from Value"), Table 4 rows.
+# (1) cache append — abstract (the Value is compressed to a latent; a
+#     Key-specific residual keeps the part of the Key the latent cannot
+#     predict), Table 4 rows.
 # --------------------------------------------------------------------------
 def append_latents(k: np.ndarray, v: np.ndarray, A_V: np.ndarray,
                    P_K: np.ndarray, U_K: np.ndarray) -> tuple:
@@ -69,8 +70,9 @@ def append_latents(k: np.ndarray, v: np.ndarray, A_V: np.ndarray,
 
 
 # --------------------------------------------------------------------------
-# (2a) routing scores — abstract ("predicts part of the Key information
-#      needed for routing"), Figure 1 caption, Table 4 "Full-context routing".
+# (2a) routing scores — abstract (the cached Value latent stands in for
+#      part of each Key when pages are ranked), Figure 1 caption, Table 4
+#      full-context routing column.
 # --------------------------------------------------------------------------
 def predicted_keys(z: np.ndarray, e: np.ndarray, P_K: np.ndarray,
                    U_K: np.ndarray) -> np.ndarray:
@@ -128,9 +130,9 @@ def select_pages(scores, top_k: int) -> tuple:
 
 
 # --------------------------------------------------------------------------
-# (3) exact attention on the selected pages — abstract ("The original Keys
-#     are then retrieved only for the selected pages to compute exact QK
-#     scores"), Table 4 "Selected attention" (exact Key + Value latent).
+# (3) exact attention on the selected pages — abstract (exact Keys are read
+#     only for the chosen pages), Table 4 selected-attention column (exact
+#     Key + Value latent).
 # --------------------------------------------------------------------------
 def selected_tokens(sel, T: int, S: int) -> np.ndarray:
     toks = [t for p in np.asarray(sel) if p >= 0
@@ -154,9 +156,9 @@ def attend(q_group: np.ndarray, K: np.ndarray, z: np.ndarray, sel, T: int,
 
 
 # --------------------------------------------------------------------------
-# (4) latent out-projection — abstract ("Value compression can be associated
-#     with the output projection"), Figure 1 caption (the complete output is
-#     reconstructed from the latents), Table 1 caption.
+# (4) latent out-projection — abstract (the Value factor is tied to the
+#     output projection), Figure 1 caption (the full output is rebuilt from
+#     the latents), Table 1 caption.
 # --------------------------------------------------------------------------
 def fold_outproj(B_V: np.ndarray, W_O: np.ndarray, Hq: int) -> np.ndarray:
     """W'_h = B_V,g(h) W_O,h for every query head: [Hq][r_v][hidden].

@@ -1,0 +1,549 @@
+// C-ABI of the BasisKV decode-attention block: argument validation,
+// workspace layout, tensor-map encoding and the launch sequences.
+//
+// Validation is pure host arithmetic and runs before any CUDA call, so an
+// invalid call neither launches nor changes state (and can be exercised on a
+// machine without a GPU).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/basiskv.h"
+#include "internal.h"
+#include "launch.cuh"
+
+namespace basiskv {
+
+__device__ unsigned int g_status;  // BASISKV_DEV_* bits, cleared by read_device_status
+std::atomic<unsigned long long> g_launches{0};
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned int* g_status_ptr[kMaxDevices];
+int g_sms[kMaxDevices];
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+unsigned int* device_status_ptr() {
+  const int dev = current_device();
+  if (dev < 0) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<unsigned int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+int num_sms() {
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      n = 148;
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+bool make_tmap_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t cols,
+                  uint64_t row_bytes, uint32_t box_rows, uint32_t box_cols,
+                  CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace basiskv
+
+using namespace basiskv;
+
+namespace {
+
+constexpr int kMaxKsplit = 16;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("BASISKV_NO_PDL");
+    return !(e && e[0] == '1');
+  }();
+  return on;
+}
+
+int check_dims(const basiskv_dims* d) {
+  if (!d) return BASISKV_ERR_INVALID_ARG;
+  if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->max_pages_per_seq < 1 ||
+      d->num_phys_pages < 1 || d->hidden < 1)
+    return BASISKV_ERR_INVALID_ARG;
+  if (d->Hq % d->Hkv) return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  const int G = d->Hq / d->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  if (d->d != 64 && d->d != 128) return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  if (d->r_v != 32 && d->r_v != 64 && d->r_v != 96 && d->r_v != 128)
+    return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  if (d->r_k != 16 && d->r_k != 32 && d->r_k != 64) return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  if (d->page_size != 8 && d->page_size != 16 && d->page_size != 32)
+    return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  if (d->hidden % 128) return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  if (((long)d->Hq * d->r_v) % 64) return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  if (d->B > 256) return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  // Tensor-map row coordinates are 32-bit.
+  if ((long long)d->num_phys_pages * d->Hkv * d->page_size >= (1ll << 31))
+    return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)d->max_pages_per_seq * d->page_size >= (1ll << 30))
+    return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  return BASISKV_OK;
+}
+
+int check_len_topk(const basiskv_dims* d, int top_k, int max_seq_len) {
+  if (top_k < 2) return BASISKV_ERR_INVALID_ARG;
+  if (max_seq_len < 1 || (long long)max_seq_len > (long long)d->max_pages_per_seq * d->page_size)
+    return BASISKV_ERR_INVALID_ARG;
+  // Page selection keeps one 32-bit key per page in shared memory.
+  const long long P = (max_seq_len + d->page_size - 1) / d->page_size;
+  if (P * 4 > 200 * 1024) return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  return BASISKV_OK;
+}
+
+struct WsLayout {
+  size_t qt, scores, sel, partial, a_f32, a_bf16, op_part, total;
+  int nsplit, ppi;
+};
+
+WsLayout ws_layout(const basiskv_dims* d, int top_k) {
+  WsLayout w{};
+  const int G = d->Hq / d->Hkv;
+  size_t off = 0;
+  w.qt = off;
+  off += align256((size_t)d->B * d->Hq * (d->r_v + d->r_k) * 4);
+  w.scores = off;
+  off += align256((size_t)d->B * d->Hkv * d->max_pages_per_seq * 4);
+  w.sel = off;
+  off += align256((size_t)d->B * d->Hkv * top_k * 4);
+  w.ppi = attend_pages_per_split(d->page_size);
+  w.nsplit = (top_k + w.ppi - 1) / w.ppi;
+  w.partial = off;
+  off += align256((size_t)d->B * d->Hkv * w.nsplit * G * (d->r_v + 2) * 4);
+  w.a_f32 = off;
+  off += align256((size_t)d->B * d->Hq * d->r_v * 4);
+  w.a_bf16 = off;
+  off += align256((size_t)d->B * d->Hq * d->r_v * 2);
+  w.op_part = off;
+  off += align256((size_t)kMaxKsplit * d->B * d->hidden * 4);
+  w.total = off;
+  return w;
+}
+
+int launch_status(cudaError_t e) {
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e == cudaSuccess ? BASISKV_OK : BASISKV_ERR_LAUNCH_FAILED;
+}
+
+CUtensorMapSwizzle swizzle_for_cols(int cols) {
+  return cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                    : (cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+// Tensor map over a paged cache viewed as [num_phys*Hkv*S rows][width].
+bool cache_map(CUtensorMap* m, const void* base, const basiskv_dims* d, int width, int box_cols) {
+  const uint64_t rows = (uint64_t)d->num_phys_pages * d->Hkv * d->page_size;
+  return make_tmap_2d(m, base, rows, width, (uint64_t)width * 2, d->page_size, box_cols,
+                      swizzle_for_cols(box_cols));
+}
+
+int z_box_cols(int r_v) { return r_v % 32 == 0 ? 32 : 16; }
+int e_box_cols(int r_k) { return r_k % 32 == 0 ? 32 : 16; }
+
+// ---------------------------------------------------------------- stages
+int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_bf16* v_new,
+               int n_new, int32_t* seq_lens, const int32_t* block_table, const basiskv_bf16* A_V,
+               const basiskv_bf16* P_K, const basiskv_bf16* U_K, basiskv_bf16* K_cache,
+               basiskv_bf16* Z_cache, basiskv_bf16* E_cache, cudaStream_t st, bool pdl) {
+  AppendArgs a{};
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.n_new = n_new;
+  a.seq_lens = seq_lens;
+  a.seq_lens_out = seq_lens;
+  a.block_table = block_table;
+  a.A_V = A_V;
+  a.P_K = P_K;
+  a.U_K = U_K;
+  a.K_cache = K_cache;
+  a.Z_cache = Z_cache;
+  a.E_cache = E_cache;
+  a.B = d->B;
+  a.Hkv = d->Hkv;
+  a.d = d->d;
+  a.r_v = d->r_v;
+  a.r_k = d->r_k;
+  a.S = d->page_size;
+  a.max_pages = d->max_pages_per_seq;
+  a.num_phys = d->num_phys_pages;
+  a.status = device_status_ptr();
+  if (!a.status) return BASISKV_ERR_CUDA;
+  int rc = launch_status(launch_append_small(a, st, pdl));
+  if (rc) return rc;
+  return launch_status(launch_bump_lengths(a, st, pdl));
+}
+
+int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_lens,
+              int max_seq_len, const int32_t* block_table, const basiskv_bf16* P_K,
+              const basiskv_bf16* U_K, const basiskv_bf16* Z_cache, const basiskv_bf16* E_cache,
+              int top_k, float* scores, int32_t* sel, uint8_t* ws, const WsLayout& L,
+              cudaStream_t st, bool pdl) {
+  unsigned int* status = device_status_ptr();
+  if (!status) return BASISKV_ERR_CUDA;
+  const int wz = z_box_cols(d->r_v), we = e_box_cols(d->r_k);
+  CUtensorMap tmZ, tmE;
+  if (!cache_map(&tmZ, Z_cache, d, d->r_v, wz) || !cache_map(&tmE, E_cache, d, d->r_k, we))
+    return BASISKV_ERR_CUDA;
+  float* qt = reinterpret_cast<float*>(ws + L.qt);
+  FoldQArgs f{q, P_K, U_K, qt, d->B, d->Hq, d->Hkv, d->d, d->r_v, d->r_k};
+  int rc = launch_status(launch_fold_query(f, st, pdl));
+  if (rc) return rc;
+  RouteArgs r{};
+  r.qt = qt;
+  r.seq_lens = seq_lens;
+  r.block_table = block_table;
+  r.scores = scores;
+  r.B = d->B;
+  r.Hkv = d->Hkv;
+  r.G = d->Hq / d->Hkv;
+  r.r_v = d->r_v;
+  r.r_k = d->r_k;
+  r.S = d->page_size;
+  r.max_pages = d->max_pages_per_seq;
+  r.num_phys = d->num_phys_pages;
+  r.max_seq_len = max_seq_len;
+  r.status = status;
+  rc = launch_status(launch_route_scores(r, tmZ, tmE, wz, we, st, pdl));
+  if (rc) return rc;
+  SelectArgs s{scores, seq_lens, sel, d->B, d->Hkv, d->page_size, d->max_pages_per_seq, top_k,
+               max_seq_len};
+  return launch_status(launch_select(s, st, pdl));
+}
+
+int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_lens,
+               const int32_t* block_table, const basiskv_bf16* K_cache,
+               const basiskv_bf16* Z_cache, const int32_t* sel, int top_k, float* a_lat,
+               uint16_t* a_bf16, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl) {
+  unsigned int* status = device_status_ptr();
+  if (!status) return BASISKV_ERR_CUDA;
+  const int wz = z_box_cols(d->r_v);
+  CUtensorMap tmK, tmZ;
+  if (!cache_map(&tmK, K_cache, d, d->d, 64) || !cache_map(&tmZ, Z_cache, d, d->r_v, wz))
+    return BASISKV_ERR_CUDA;
+  AttendArgs a{};
+  a.q = q;
+  a.seq_lens = seq_lens;
+  a.block_table = block_table;
+  a.sel = sel;
+  a.partial = reinterpret_cast<float*>(ws + L.partial);
+  a.B = d->B;
+  a.Hq = d->Hq;
+  a.Hkv = d->Hkv;
+  a.G = d->Hq / d->Hkv;
+  a.d = d->d;
+  a.r_v = d->r_v;
+  a.S = d->page_size;
+  a.max_pages = d->max_pages_per_seq;
+  a.num_phys = d->num_phys_pages;
+  a.top_k = top_k;
+  a.nsplit = L.nsplit;
+  a.pages_per_split = L.ppi;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d->d));
+  a.status = status;
+  int rc = launch_status(launch_attend(a, tmK, tmZ, wz, st, pdl));
+  if (rc) return rc;
+  CombineArgs c{a.partial, seq_lens, a_lat, a_bf16, d->B, d->Hq, d->Hkv, a.G, d->r_v,
+                d->page_size, top_k, L.nsplit, L.ppi};
+  return launch_status(launch_combine(c, st, pdl));
+}
+
+int run_outproj(const basiskv_dims* d, const uint16_t* a_bf16, const basiskv_bf16* W_fold,
+                basiskv_bf16* y, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl) {
+  unsigned int* status = device_status_ptr();
+  if (!status) return BASISKV_ERR_CUDA;
+  const int K = d->Hq * d->r_v;
+  const int bn = outproj_bn(d->B);
+  CUtensorMap tmW, tmA;
+  if (!make_tmap_2d(&tmW, W_fold, d->hidden, K, (uint64_t)K * 2, 128, 64,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tmA, a_bf16, d->B, K, (uint64_t)K * 2, bn, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BASISKV_ERR_CUDA;
+  OutprojArgs o{};
+  o.partial = reinterpret_cast<float*>(ws + L.op_part);
+  o.y = y;
+  o.B = d->B;
+  o.H = d->hidden;
+  o.K = K;
+  o.ksplit = outproj_ksplit(d->hidden, K, d->B);
+  if (o.ksplit > kMaxKsplit) o.ksplit = kMaxKsplit;
+  o.bn = bn;
+  o.status = status;
+  return launch_status(launch_outproj(o, tmW, tmA, st, pdl));
+}
+
+int check_ws(const basiskv_dims* d, int top_k, void* ws, size_t ws_bytes, WsLayout* L) {
+  *L = ws_layout(d, top_k);
+  if (!ws) return BASISKV_ERR_INVALID_ARG;
+  if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return BASISKV_ERR_INVALID_ARG;
+  if (ws_bytes < L->total) return BASISKV_ERR_WORKSPACE_TOO_SMALL;
+  return BASISKV_OK;
+}
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// bf16 tensors: non-null and 16-byte aligned (TMA and vector loads).
+#define BKV_REQUIRE(p)                                         \
+  do {                                                         \
+    if (!(p) || !aligned16(p)) return BASISKV_ERR_INVALID_ARG; \
+  } while (0)
+// int32 / fp32 arrays: non-null and 4-byte aligned.
+#define BKV_REQUIRE4(p)                                       \
+  do {                                                        \
+    if (!(p) || !aligned4(p)) return BASISKV_ERR_INVALID_ARG; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t basiskv_workspace_size(const basiskv_dims* dims, int top_k, int max_seq_len) {
+  if (check_dims(dims) != BASISKV_OK || check_len_topk(dims, top_k, max_seq_len) != BASISKV_OK)
+    return 0;
+  return ws_layout(dims, top_k).total;
+}
+
+int basiskv_fold_outproj(const basiskv_dims* dims, const basiskv_bf16* B_V,
+                         const basiskv_bf16* W_O, basiskv_bf16* W_fold, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  BKV_REQUIRE(B_V);
+  BKV_REQUIRE(W_O);
+  BKV_REQUIRE(W_fold);
+  FoldOutArgs a{B_V, W_O, W_fold, dims->Hq, dims->Hkv, dims->d, dims->r_v, dims->hidden};
+  return launch_status(launch_fold_outproj(a, static_cast<cudaStream_t>(stream)));
+}
+
+int basiskv_append(const basiskv_dims* dims, const basiskv_bf16* k_new, const basiskv_bf16* v_new,
+                   int n_new, int32_t* seq_lens, const int32_t* block_table,
+                   const basiskv_bf16* A_V, const basiskv_bf16* P_K, const basiskv_bf16* U_K,
+                   basiskv_bf16* K_cache, basiskv_bf16* Z_cache, basiskv_bf16* E_cache,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (n_new < 1 || (long long)n_new > (long long)dims->max_pages_per_seq * dims->page_size)
+    return BASISKV_ERR_INVALID_ARG;
+  BKV_REQUIRE(k_new);
+  BKV_REQUIRE(v_new);
+  BKV_REQUIRE4(seq_lens);
+  BKV_REQUIRE4(block_table);
+  BKV_REQUIRE(A_V);
+  BKV_REQUIRE(P_K);
+  BKV_REQUIRE(U_K);
+  BKV_REQUIRE(K_cache);
+  BKV_REQUIRE(Z_cache);
+  BKV_REQUIRE(E_cache);
+  (void)workspace;
+  (void)workspace_bytes;
+  return run_append(dims, k_new, v_new, n_new, seq_lens, block_table, A_V, P_K, U_K, K_cache,
+                    Z_cache, E_cache, static_cast<cudaStream_t>(stream), pdl_enabled());
+}
+
+int basiskv_route(const basiskv_dims* dims, const basiskv_bf16* q, const int32_t* seq_lens,
+                  int max_seq_len, const int32_t* block_table, const basiskv_bf16* P_K,
+                  const basiskv_bf16* U_K, const basiskv_bf16* Z_cache,
+                  const basiskv_bf16* E_cache, int top_k, float* page_scores, int32_t* sel,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_len_topk(dims, top_k, max_seq_len);
+  if (rc) return rc;
+  BKV_REQUIRE(q);
+  BKV_REQUIRE4(seq_lens);
+  BKV_REQUIRE4(block_table);
+  BKV_REQUIRE(P_K);
+  BKV_REQUIRE(U_K);
+  BKV_REQUIRE(Z_cache);
+  BKV_REQUIRE(E_cache);
+  BKV_REQUIRE4(sel);
+  if (page_scores && !aligned4(page_scores)) return BASISKV_ERR_INVALID_ARG;
+  WsLayout L;
+  rc = check_ws(dims, top_k, workspace, workspace_bytes, &L);
+  if (rc) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* scores = page_scores ? page_scores : reinterpret_cast<float*>(ws + L.scores);
+  return run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache, top_k,
+                   scores, sel, ws, L, static_cast<cudaStream_t>(stream), pdl_enabled());
+}
+
+int basiskv_attend(const basiskv_dims* dims, const basiskv_bf16* q, const int32_t* seq_lens,
+                   int max_seq_len, const int32_t* block_table, const basiskv_bf16* K_cache,
+                   const basiskv_bf16* Z_cache, const int32_t* sel, int top_k, float* a_lat,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_len_topk(dims, top_k, max_seq_len);
+  if (rc) return rc;
+  BKV_REQUIRE(q);
+  BKV_REQUIRE4(seq_lens);
+  BKV_REQUIRE4(block_table);
+  BKV_REQUIRE(K_cache);
+  BKV_REQUIRE(Z_cache);
+  BKV_REQUIRE4(sel);
+  BKV_REQUIRE4(a_lat);
+  WsLayout L;
+  rc = check_ws(dims, top_k, workspace, workspace_bytes, &L);
+  if (rc) return rc;
+  return run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel, top_k, a_lat, nullptr,
+                    static_cast<uint8_t*>(workspace), L, static_cast<cudaStream_t>(stream),
+                    pdl_enabled());
+}
+
+int basiskv_outproj(const basiskv_dims* dims, const float* a_lat, const basiskv_bf16* W_fold,
+                    basiskv_bf16* y, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  BKV_REQUIRE4(a_lat);
+  BKV_REQUIRE(W_fold);
+  BKV_REQUIRE(y);
+  WsLayout L;
+  rc = check_ws(dims, 2, workspace, workspace_bytes, &L);
+  if (rc) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* a16 = reinterpret_cast<uint16_t*>(ws + L.a_bf16);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool pdl = pdl_enabled();
+  rc = launch_status(launch_cast_bf16(a_lat, a16, (size_t)dims->B * dims->Hq * dims->r_v, st, pdl));
+  if (rc) return rc;
+  return run_outproj(dims, a16, W_fold, y, ws, L, st, pdl);
+}
+
+int basiskv_decode(const basiskv_dims* dims, const basiskv_bf16* q, const basiskv_bf16* k_new,
+                   const basiskv_bf16* v_new, int32_t* seq_lens, int max_seq_len,
+                   const int32_t* block_table, const basiskv_bf16* A_V, const basiskv_bf16* P_K,
+                   const basiskv_bf16* U_K, const basiskv_bf16* W_fold, basiskv_bf16* K_cache,
+                   basiskv_bf16* Z_cache, basiskv_bf16* E_cache, int top_k, int32_t* sel,
+                   basiskv_bf16* y, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_len_topk(dims, top_k, max_seq_len);
+  if (rc) return rc;
+  const bool append = k_new || v_new;
+  if (append) {
+    BKV_REQUIRE(k_new);
+    BKV_REQUIRE(v_new);
+    BKV_REQUIRE(A_V);
+    BKV_REQUIRE(K_cache);
+    BKV_REQUIRE(E_cache);
+  }
+  BKV_REQUIRE(q);
+  BKV_REQUIRE4(seq_lens);
+  BKV_REQUIRE4(block_table);
+  BKV_REQUIRE(P_K);
+  BKV_REQUIRE(U_K);
+  BKV_REQUIRE(W_fold);
+  BKV_REQUIRE(K_cache);
+  BKV_REQUIRE(Z_cache);
+  BKV_REQUIRE(E_cache);
+  BKV_REQUIRE(y);
+  if (sel && !aligned4(sel)) return BASISKV_ERR_INVALID_ARG;
+  WsLayout L;
+  rc = check_ws(dims, top_k, workspace, workspace_bytes, &L);
+  if (rc) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool pdl = pdl_enabled();
+  int32_t* sel_buf = sel ? sel : reinterpret_cast<int32_t*>(ws + L.sel);
+  if (append) {
+    rc = run_append(dims, k_new, v_new, 1, seq_lens, block_table, A_V, P_K, U_K, K_cache, Z_cache,
+                    E_cache, st, pdl);
+    if (rc) return rc;
+  }
+  rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache, top_k,
+                 reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl);
+  if (rc) return rc;
+  uint16_t* a16 = reinterpret_cast<uint16_t*>(ws + L.a_bf16);
+  rc = run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel_buf, top_k, nullptr, a16,
+                  ws, L, st, pdl);
+  if (rc) return rc;
+  return run_outproj(dims, a16, W_fold, y, ws, L, st, pdl);
+}
+
+int basiskv_read_device_status(void* stream, uint32_t* flags) {
+  if (!flags) return BASISKV_ERR_INVALID_ARG;
+  *flags = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BASISKV_ERR_CUDA;
+  unsigned int* p = device_status_ptr();
+  if (!p) return BASISKV_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return BASISKV_ERR_CUDA;
+  if (v && cudaMemset(p, 0, sizeof(v)) != cudaSuccess) return BASISKV_ERR_CUDA;
+  *flags = v;
+  return v ? BASISKV_ERR_DEVICE : BASISKV_OK;
+}
+
+uint64_t basiskv_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* basiskv_strerror(int status) {
+  switch (status) {
+    case BASISKV_OK: return "ok";
+    case BASISKV_ERR_INVALID_ARG: return "invalid argument (null/misaligned pointer or bad count)";
+    case BASISKV_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case BASISKV_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case BASISKV_ERR_LAUNCH_FAILED: return "kernel launch failed";
+    case BASISKV_ERR_DEVICE: return "device reported an error (see device status bits)";
+    case BASISKV_ERR_CUDA: return "CUDA runtime call failed";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

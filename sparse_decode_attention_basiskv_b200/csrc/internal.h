@@ -1,0 +1,121 @@
+// Host-side interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/basiskv.h"
+
+namespace basiskv {
+
+// Encodes a 2-D bf16 tensor map: `rows` rows of `cols` elements with a row
+// pitch of `row_bytes`, boxes of box_rows x box_cols, the given swizzle.
+// Returns false when the driver rejects the description.
+bool make_tmap_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t cols,
+                  uint64_t row_bytes, uint32_t box_rows, uint32_t box_cols,
+                  CUtensorMapSwizzle swizzle);
+
+// Address of this library's device status word on the current device.
+unsigned int* device_status_ptr();
+
+int num_sms();
+
+// ------------------------------------------------------------------ append
+struct AppendArgs {
+  const uint16_t* k_new;  // [B][n_new][Hkv][d]
+  const uint16_t* v_new;
+  int n_new;
+  const int32_t* seq_lens;
+  int32_t* seq_lens_out;
+  const int32_t* block_table;
+  const uint16_t* A_V;
+  const uint16_t* P_K;
+  const uint16_t* U_K;
+  uint16_t* K_cache;
+  uint16_t* Z_cache;
+  uint16_t* E_cache;
+  int B, Hkv, d, r_v, r_k, S, max_pages, num_phys;
+  unsigned int* status;
+};
+cudaError_t launch_append_small(const AppendArgs& a, cudaStream_t st, bool pdl);
+cudaError_t launch_bump_lengths(const AppendArgs& a, cudaStream_t st, bool pdl);
+
+// ------------------------------------------------------------------- route
+struct FoldQArgs {
+  const uint16_t* q;    // [B][Hq][d]
+  const uint16_t* P_K;  // [Hkv][r_v][d]
+  const uint16_t* U_K;  // [Hkv][d][r_k]
+  float* qt;            // [B][Hq][r_v + r_k]
+  int B, Hq, Hkv, d, r_v, r_k;
+};
+cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl);
+
+struct RouteArgs {
+  const float* qt;  // [B][Hq][r_v + r_k]
+  const int32_t* seq_lens;
+  const int32_t* block_table;
+  float* scores;  // [B][Hkv][max_pages]
+  int B, Hkv, G, r_v, r_k, S, max_pages, num_phys, max_seq_len;
+  unsigned int* status;
+};
+cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
+                                const CUtensorMap& tmE, int wz, int we, cudaStream_t st,
+                                bool pdl);
+
+struct SelectArgs {
+  const float* scores;
+  const int32_t* seq_lens;
+  int32_t* sel;  // [B][Hkv][top_k]
+  int B, Hkv, S, max_pages, top_k, max_seq_len;
+};
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
+
+// ------------------------------------------------------------------ attend
+struct AttendArgs {
+  const uint16_t* q;
+  const int32_t* seq_lens;
+  const int32_t* block_table;
+  const int32_t* sel;
+  float* partial;  // [B*Hkv][nsplit][G][r_v + 2]
+  int B, Hq, Hkv, G, d, r_v, S, max_pages, num_phys, top_k, nsplit, pages_per_split;
+  float scale_log2;  // log2(e) / sqrt(d)
+  unsigned int* status;
+};
+int attend_pages_per_split(int S);
+cudaError_t launch_attend(const AttendArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmZ,
+                          int wz, cudaStream_t st, bool pdl);
+
+struct CombineArgs {
+  const float* partial;
+  const int32_t* seq_lens;
+  float* a_lat;        // [B][Hq][r_v] fp32 (may be null)
+  uint16_t* a_bf16;    // [B][Hq][r_v] bf16 (may be null)
+  int B, Hq, Hkv, G, r_v, S, top_k, nsplit, pages_per_split;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st, bool pdl);
+
+// ----------------------------------------------------------------- outproj
+struct OutprojArgs {
+  float* partial;  // [ksplit][B][H] fp32 (ksplit > 1)
+  uint16_t* y;     // [B][H] bf16
+  int B, H, K, ksplit, bn;
+  unsigned int* status;
+};
+// Chooses the K split for a given problem.
+int outproj_ksplit(int H, int K, int B);
+int outproj_bn(int B);
+cudaError_t launch_outproj(const OutprojArgs& a, const CUtensorMap& tmW, const CUtensorMap& tmA,
+                           cudaStream_t st, bool pdl);
+cudaError_t launch_cast_bf16(const float* x, uint16_t* y, size_t n, cudaStream_t st, bool pdl);
+
+struct FoldOutArgs {
+  const uint16_t* B_V;  // [Hkv][r_v][d]
+  const uint16_t* W_O;  // [Hq*d][H]
+  uint16_t* W_fold;     // [H][Hq*r_v]
+  int Hq, Hkv, d, r_v, H;
+};
+cudaError_t launch_fold_outproj(const FoldOutArgs& a, cudaStream_t st);
+
+}  // namespace basiskv

@@ -1,0 +1,34 @@
+// Kernel launch with optional Programmatic Dependent Launch: with `pdl` set,
+// the kernel may start while its predecessor on the stream is finishing;
+// every kernel here executes griddepcontrol.wait before touching data that
+// a predecessor writes, which is a no-op for a plain launch.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <utility>
+
+namespace basiskv {
+
+// Kernels launched by this library in this process (basiskv_launch_count).
+extern std::atomic<unsigned long long> g_launches;
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t st, bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+}  // namespace basiskv

@@ -1,0 +1,453 @@
+// Routing: BasisKV scores every page of the full context from the narrow
+// per-token state (Value latent z and Key residual e) instead of the exact
+// Keys (abstract: the cached latent stands in for part of each Key when
+// pages are ranked; Table 4, full-context routing column).
+//
+// The predicted key of token t is khat_t = z_t P_K + e_t U_K^T, and
+//   q_h . khat_t = z_t . (P_K q_h) + e_t . (U_K^T q_h),
+// so the query is folded once per step (fold_query_kernel) and the hot loop
+// streams only z and e: (r_v + r_k) * 2 bytes per token and KV head.
+//
+// route_kernel is HBM-bound.  A persistent grid of one CTA per SM walks a
+// contiguous range of (sequence, KV head, page-tile) work; a producer warp
+// gathers each tile's pages through the block table with 2-D TMA loads
+// (swizzled boxes, so the consumers' row-per-thread reads are free of bank
+// conflicts) into a ring of shared-memory stages; eight consumer warps own
+// one token each per stage, do the G head dot products in fp32, and reduce
+// the page maximum with warp shuffles.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "launch.cuh"
+
+namespace basiskv {
+
+namespace {
+
+// ----------------------------------------------------------- query folding
+// qt[b][h][j]       = sum_i P_K[g][j][i] q[b][h][i]          j < r_v
+// qt[b][h][r_v + c] = sum_i q[b][h][i] U_K[g][i][c]           c < r_k
+constexpr int kFoldThreads = 128;
+
+__global__ void __launch_bounds__(kFoldThreads) fold_query_kernel(FoldQArgs a) {
+  const int bg = blockIdx.x, b = bg / a.Hkv, g = bg % a.Hkv, tid = threadIdx.x;
+  const int G = a.Hq / a.Hkv, rq = a.r_v + a.r_k;
+  extern __shared__ float qs[];  // [G][d]
+  pdl_wait();
+  for (int i = tid; i < G * a.d; i += blockDim.x)
+    qs[i] = bf16_to_f(a.q[((size_t)b * a.Hq + g * G) * a.d + i]);
+  __syncthreads();
+  for (int j = tid; j < rq; j += blockDim.x) {
+    float acc[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) acc[h] = 0.f;
+    if (j < a.r_v) {
+      const uint16_t* P = a.P_K + ((size_t)g * a.r_v + j) * a.d;
+      for (int i = 0; i < a.d; ++i) {
+        const float p = bf16_to_f(P[i]);
+#pragma unroll
+        for (int h = 0; h < 8; ++h)
+          if (h < G) acc[h] = fmaf(p, qs[h * a.d + i], acc[h]);
+      }
+    } else {
+      const uint16_t* U = a.U_K + (size_t)g * a.d * a.r_k + (j - a.r_v);
+      for (int i = 0; i < a.d; ++i) {
+        const float u = bf16_to_f(U[(size_t)i * a.r_k]);
+#pragma unroll
+        for (int h = 0; h < 8; ++h)
+          if (h < G) acc[h] = fmaf(u, qs[h * a.d + i], acc[h]);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+      if (h < G) a.qt[((size_t)b * a.Hq + g * G + h) * rq + j] = acc[h];
+  }
+}
+
+// ------------------------------------------------------------ page scoring
+constexpr int kRouteConsumers = 256;  // one token per consumer thread per stage
+constexpr int kRouteThreads = kRouteConsumers + 32;
+constexpr int kRouteConsumerWarps = kRouteConsumers / 32;
+
+struct RouteGeom {
+  int np;           // pages per stage (kRouteConsumers / S)
+  int page_bytes;   // shared-memory bytes of one page slot (1 KB multiple)
+  int q_off;        // offset of the folded-query slot in a stage
+  int q_bytes;      // G * (r_v + r_k) * 4
+  int stage_bytes;  // 1 KB multiple
+  int stages;
+  int wz, we;       // box widths (columns) of the z and e tensor maps
+  int nzb, neb;     // boxes per page
+  int zbox, ebox;   // bytes per box
+  uint32_t zmask, emask;  // swizzle masks
+};
+
+__device__ __forceinline__ void decode_tile(long tile, int tiles_per_bg, int Hkv, int& bg,
+                                            int& b, int& g, int& ti) {
+  bg = (int)(tile / tiles_per_bg);
+  ti = (int)(tile % tiles_per_bg);
+  b = bg / Hkv;
+  g = bg % Hkv;
+}
+
+__device__ __forceinline__ int clamp_len(int T, int max_seq_len, unsigned int* status,
+                                         bool report) {
+  if (T < 0 || T > max_seq_len) {
+    if (report) raise_status(status, BASISKV_DEV_BAD_LENGTH);
+    T = T < 0 ? 0 : max_seq_len;
+  }
+  return T;
+}
+
+// Adds the contribution of one 8-wide chunk of a token row to the G head
+// accumulators.  `xa` is the swizzled shared address of the row chunk, `qa`
+// the address of the chunk in head 0's folded query; heads are rq floats
+// apart.
+template <int G>
+__device__ __forceinline__ void chunk_fma(uint32_t xa, uint32_t qa, uint32_t qstride,
+                                          float (&acc)[G][2]) {
+  const uint4 w = lds128(xa);
+  const float x0 = bf16lo(w.x), x1 = bf16hi(w.x), x2 = bf16lo(w.y), x3 = bf16hi(w.y);
+  const float x4 = bf16lo(w.z), x5 = bf16hi(w.z), x6 = bf16lo(w.w), x7 = bf16hi(w.w);
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const float4 q0 = lds128f(qa + h * qstride);
+    const float4 q1 = lds128f(qa + h * qstride + 16);
+    acc[h][0] = fmaf(x0, q0.x, acc[h][0]);
+    acc[h][1] = fmaf(x1, q0.y, acc[h][1]);
+    acc[h][0] = fmaf(x2, q0.z, acc[h][0]);
+    acc[h][1] = fmaf(x3, q0.w, acc[h][1]);
+    acc[h][0] = fmaf(x4, q1.x, acc[h][0]);
+    acc[h][1] = fmaf(x5, q1.y, acc[h][1]);
+    acc[h][0] = fmaf(x6, q1.z, acc[h][0]);
+    acc[h][1] = fmaf(x7, q1.w, acc[h][1]);
+  }
+}
+
+template <int G>
+__global__ void __launch_bounds__(kRouteThreads, 1)
+    route_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmE,
+                 RouteArgs a, RouteGeom geo) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)geo.stages * geo.stage_bytes);
+  uint64_t* empty = full + geo.stages;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < geo.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kRouteConsumerWarps);
+    }
+    fence_barrier_init();
+  }
+  if (warp == kRouteConsumerWarps && lane == 0) {
+    prefetch_tmap(&tmZ);
+    prefetch_tmap(&tmE);
+  }
+  __syncthreads();
+  pdl_wait();
+
+  const int S = a.S, rq = a.r_v + a.r_k;
+  const int P_max = (a.max_seq_len + S - 1) / S;
+  const int tiles_per_bg = (P_max + geo.np - 1) / geo.np;
+  const long total = (long)a.B * a.Hkv * tiles_per_bg;
+  const long t_begin = total * blockIdx.x / gridDim.x;
+  const long t_end = total * (blockIdx.x + 1) / gridDim.x;
+
+  if (warp == kRouteConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      for (long tile = t_begin; tile < t_end; ++tile) {
+        int bg, b, g, ti;
+        decode_tile(tile, tiles_per_bg, a.Hkv, bg, b, g, ti);
+        const int T = clamp_len(a.seq_lens[b], a.max_seq_len, a.status, false);
+        const int P = (T + S - 1) / S, p0 = ti * geo.np;
+        if (p0 >= P) continue;
+        const int npg = min(geo.np, P - p0);
+        const int s = it % geo.stages;
+        if (!mbar_wait(&empty[s], ((it / geo.stages) & 1) ^ 1, a.status)) break;
+        uint8_t* st = smem + (size_t)s * geo.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], geo.q_bytes + npg * S * rq * 2);
+        bulk_load(st + geo.q_off, a.qt + ((size_t)b * a.Hkv * G + (size_t)g * G) * rq,
+                  geo.q_bytes, &full[s]);
+        const int32_t* bt = a.block_table + (size_t)b * a.max_pages + p0;
+        for (int j = 0; j < npg; ++j) {
+          int pp = bt[j];
+          if (pp < 0 || pp >= a.num_phys) {
+            raise_status(a.status, BASISKV_DEV_BAD_PAGE);
+            pp = 0;  // keep the byte count; the page's score is flagged garbage
+          }
+          const int row = (pp * a.Hkv + g) * S;
+          uint8_t* pg = st + j * geo.page_bytes;
+          for (int k = 0; k < geo.nzb; ++k)
+            tma_load_2d(pg + k * geo.zbox, &tmZ, k * geo.wz, row, &full[s]);
+          uint8_t* pe = pg + geo.nzb * geo.zbox;
+          for (int k = 0; k < geo.neb; ++k)
+            tma_load_2d(pe + k * geo.ebox, &tmE, k * geo.we, row, &full[s]);
+        }
+        ++it;
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------- consumers
+  const int page_local = tid / S, row = tid % S;
+  const uint32_t qstride = rq * 4;
+  const int zc_per_box = geo.wz / 8, ec_per_box = geo.we / 8;
+  const int nzc = a.r_v / 8, nec = a.r_k / 8;
+  int it = 0;
+  for (long tile = t_begin; tile < t_end; ++tile) {
+    int bg, b, g, ti;
+    decode_tile(tile, tiles_per_bg, a.Hkv, bg, b, g, ti);
+    const int T = clamp_len(a.seq_lens[b], a.max_seq_len, a.status, tid == 0 && ti == 0);
+    const int P = (T + S - 1) / S, p0 = ti * geo.np;
+    if (p0 >= P) continue;
+    const int npg = min(geo.np, P - p0);
+    const int s = it % geo.stages;
+    if (!mbar_wait(&full[s], (it / geo.stages) & 1, a.status)) break;
+    const uint32_t st = smem_u32(smem + (size_t)s * geo.stage_bytes);
+    float best = -INFINITY;
+    const int p = p0 + page_local;
+    if (page_local < npg && p * S + row < T) {
+      float acc[G][2];
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = 0.f;
+      const uint32_t pgb = st + page_local * geo.page_bytes;
+      const uint32_t qb = st + geo.q_off;
+#pragma unroll 4
+      for (int c = 0; c < nzc; ++c) {
+        const int box = c / zc_per_box, cc = c - box * zc_per_box;
+        const uint32_t xa = swz(pgb + box * geo.zbox + row * geo.wz * 2 + cc * 16, geo.zmask);
+        chunk_fma<G>(xa, qb + c * 32, qstride, acc);
+      }
+      const uint32_t peb = pgb + geo.nzb * geo.zbox;
+#pragma unroll 4
+      for (int c = 0; c < nec; ++c) {
+        const int box = c / ec_per_box, cc = c - box * ec_per_box;
+        const uint32_t xa = swz(peb + box * geo.ebox + row * geo.we * 2 + cc * 16, geo.emask);
+        chunk_fma<G>(xa, qb + (a.r_v + c * 8) * 4, qstride, acc);
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) best = fmaxf(best, acc[h][0] + acc[h][1]);
+    }
+    for (int o = S >> 1; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+    if (row == 0 && page_local < npg) a.scores[(size_t)bg * a.max_pages + p] = best;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    ++it;
+  }
+}
+
+// -------------------------------------------------------- page selection
+// Per (sequence, KV head): sink page 0 and newest page P-1 always; the other
+// top_k - 2 slots go to the best remaining pages by (score desc, index asc),
+// found exactly with an MSB-first radix select over order-preserving 32-bit
+// keys; ties at the threshold are taken in index order.  Output ascending.
+constexpr int kSelThreads = 512;
+constexpr int kSelWarps = kSelThreads / 32;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f == 0.f) f = 0.f;  // -0 ranks as +0
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive prefix sum over the block; *total receives the sum of all v.
+__device__ int block_excl_scan(int v, int* sh, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kSelWarps ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    sh[lane] = w;
+  }
+  __syncthreads();
+  const int res = (warp ? sh[warp - 1] : 0) + x - v;
+  *total = sh[kSelWarps - 1];
+  __syncthreads();
+  return res;
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
+  extern __shared__ uint32_t keys[];
+  __shared__ int hist[256];
+  __shared__ int sh[32];
+  __shared__ uint32_t s_digit;
+  __shared__ int s_rem;
+  pdl_wait();
+  const int bg = blockIdx.x, b = bg / a.Hkv, tid = threadIdx.x;
+  int T = a.seq_lens[b];
+  T = T < 0 ? 0 : (T > a.max_seq_len ? a.max_seq_len : T);
+  const int P = (T + a.S - 1) / a.S;
+  int32_t* out = a.sel + (size_t)bg * a.top_k;
+  if (a.top_k >= P) {
+    for (int i = tid; i < a.top_k; i += kSelThreads) out[i] = i < P ? i : -1;
+    return;
+  }
+  const int n = P - 2, need = a.top_k - 2;
+  const float* sc = a.scores + (size_t)bg * a.max_pages + 1;
+  for (int i = tid; i < n; i += kSelThreads) keys[i] = order_key(sc[i]);
+  __syncthreads();
+
+  uint32_t prefix = 0, pmask = 0;
+  int rem = need;
+  if (need > 0) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      if (tid < 256) hist[tid] = 0;
+      __syncthreads();
+      for (int i = tid; i < n; i += kSelThreads) {
+        const uint32_t k = keys[i];
+        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255], 1);
+      }
+      __syncthreads();
+      if (tid < 32) {  // lane l covers digits 255-8l .. 248-8l, high to low
+        int local = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) local += hist[255 - 8 * tid - j];
+        int cum = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, cum, o);
+          if (tid >= o) cum += y;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, cum >= rem);
+        const int L = __ffs(hit) - 1;
+        if (tid == L) {
+          int start = cum - local;
+          for (int j = 0; j < 8; ++j) {
+            const int dg = 255 - 8 * L - j;
+            if (start + hist[dg] >= rem) {
+              s_digit = (uint32_t)dg;
+              s_rem = rem - start;
+              break;
+            }
+            start += hist[dg];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= s_digit << shift;
+      pmask |= 0xffu << shift;
+      rem = s_rem;
+      __syncthreads();
+    }
+  }
+  const uint32_t thr = prefix;
+  // Contiguous candidate chunk per thread, so prefix sums follow index order.
+  const int E = (n + kSelThreads - 1) / kSelThreads;
+  const int i0 = min(tid * E, n), i1 = min(i0 + E, n);
+  int total;
+  int n_eq = 0;
+  if (need > 0)
+    for (int i = i0; i < i1; ++i) n_eq += keys[i] == thr;
+  int eq_rank = block_excl_scan(n_eq, sh, &total);
+  int n_take = 0;
+  if (need > 0) {
+    int r = eq_rank;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t k = keys[i];
+      n_take += (k > thr) || (k == thr && r < rem);
+      r += k == thr;
+    }
+  }
+  int pos = 1 + block_excl_scan(n_take, sh, &total);
+  if (need > 0) {
+    int r = eq_rank;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t k = keys[i];
+      if ((k > thr) || (k == thr && r < rem)) out[pos++] = i + 1;
+      r += k == thr;
+    }
+  }
+  if (tid == 0) {
+    out[0] = 0;
+    out[a.top_k - 1] = P - 1;
+  }
+}
+
+RouteGeom route_geometry(int G, int r_v, int r_k, int S, int wz, int we) {
+  RouteGeom g{};
+  g.np = kRouteConsumers / S;
+  g.wz = wz;
+  g.we = we;
+  g.nzb = r_v / wz;
+  g.neb = r_k / we;
+  g.zbox = S * wz * 2;
+  g.ebox = S * we * 2;
+  g.zmask = wz == 64 ? 7u : (wz == 32 ? 3u : 1u);
+  g.emask = we == 64 ? 7u : (we == 32 ? 3u : 1u);
+  g.page_bytes = ((S * (r_v + r_k) * 2) + 1023) / 1024 * 1024;
+  g.q_off = g.np * g.page_bytes;
+  g.q_bytes = G * (r_v + r_k) * 4;
+  g.stage_bytes = (g.q_off + g.q_bytes + 1023) / 1024 * 1024;
+  const int budget = 220 * 1024;
+  g.stages = budget / g.stage_bytes;
+  if (g.stages > 8) g.stages = 8;
+  return g;
+}
+
+template <int G>
+cudaError_t launch_route_g(const RouteArgs& a, const CUtensorMap& tmZ, const CUtensorMap& tmE,
+                           const RouteGeom& geo, cudaStream_t st, bool pdl) {
+  const size_t smem = (size_t)geo.stages * geo.stage_bytes + 2 * geo.stages * 8 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<G>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int P_max = (a.max_seq_len + a.S - 1) / a.S;
+  const long tiles = (long)a.B * a.Hkv * ((P_max + geo.np - 1) / geo.np);
+  long grid = num_sms();
+  if (grid > tiles) grid = tiles;
+  if (grid < 1) grid = 1;
+  return launch_k(route_kernel<G>, dim3((unsigned)grid), dim3(kRouteThreads), smem, st, pdl,
+                  tmZ, tmE, a, geo);
+}
+
+}  // namespace
+
+cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl) {
+  const int G = a.Hq / a.Hkv;
+  return launch_k(fold_query_kernel, dim3(a.B * a.Hkv), dim3(kFoldThreads),
+                  (size_t)G * a.d * sizeof(float), st, pdl, a);
+}
+
+cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
+                                const CUtensorMap& tmE, int wz, int we, cudaStream_t st,
+                                bool pdl) {
+  const RouteGeom geo = route_geometry(a.G, a.r_v, a.r_k, a.S, wz, we);
+  if (geo.stages < 2) return cudaErrorInvalidConfiguration;
+  switch (a.G) {
+    case 1: return launch_route_g<1>(a, tmZ, tmE, geo, st, pdl);
+    case 2: return launch_route_g<2>(a, tmZ, tmE, geo, st, pdl);
+    case 4: return launch_route_g<4>(a, tmZ, tmE, geo, st, pdl);
+    case 8: return launch_route_g<8>(a, tmZ, tmE, geo, st, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
+  const int P_max = (a.max_seq_len + a.S - 1) / a.S;
+  const size_t smem = (size_t)(P_max > 2 ? P_max : 2) * sizeof(uint32_t);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_k(select_kernel, dim3(a.B * a.Hkv), dim3(kSelThreads), smem, st, pdl, a);
+}
+
+}  // namespace basiskv

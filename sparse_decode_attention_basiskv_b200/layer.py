@@ -1,0 +1,58 @@
+"""Device state of one BasisKV attention layer and its decode call.
+
+Holds the paged caches, block table, lengths, factors, folded out-projection
+and workspace of one layer on one GPU, and forwards each decode step to the
+C-ABI (``basiskv_decode``).  Allocation is PyTorch's; all compute is the
+library's.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (Dims, basiskv_decode, basiskv_fold_outproj, workspace_size)
+
+
+class DecodeLayer:
+    def __init__(self, dims: Dims, factors: dict, caches: dict, block_table: torch.Tensor,
+                 seq_lens: torch.Tensor, top_k: int, max_seq_len: int, stream=None):
+        self.dims = dims
+        self.top_k = top_k
+        self.max_seq_len = max_seq_len
+        self.A_V, self.P_K, self.U_K = factors["A_V"], factors["P_K"], factors["U_K"]
+        self.K, self.Z, self.E = caches["K"], caches["Z"], caches["E"]
+        self.block_table = block_table
+        self.seq_lens = seq_lens
+        dev = self.K.device
+        self.W_fold = torch.empty(dims.hidden, dims.Hq * dims.r_v, dtype=torch.bfloat16,
+                                  device=dev)
+        basiskv_fold_outproj(dims, factors["B_V"], factors["W_O"], self.W_fold, stream)
+        n = workspace_size(dims, top_k, max_seq_len)
+        if n == 0:
+            raise ValueError("unsupported dims for the BasisKV library")
+        self.workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+        self.y = torch.empty(dims.B, dims.hidden, dtype=torch.bfloat16, device=dev)
+
+    @classmethod
+    def from_problem(cls, pb, device="cuda", stream=None) -> "DecodeLayer":
+        """Builds the layer of a synthetic workload (``synth.Problem``)."""
+        wl = pb.wl
+        pc = wl.pages_capacity()
+        dims = Dims(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, hidden=wl.hidden, r_v=wl.r_v,
+                    r_k=wl.r_k, page_size=wl.page_size, max_pages_per_seq=pc,
+                    num_phys_pages=wl.B * pc)
+        factors = {k: v.to(device).contiguous() for k, v in pb.factors.items()}
+        caches = {k: v.contiguous() for k, v in pb.paged().items()}
+        return cls(dims, factors, caches, pb.table.to(device).contiguous(),
+                   pb.seq_lens.to(device).clone(), wl.top_k, pc * wl.page_size, stream)
+
+    def decode(self, q, k_new=None, v_new=None, sel=None, max_seq_len=None, y=None,
+               stream=None) -> torch.Tensor:
+        """One decode step: optional append of (k_new, v_new), then routing,
+        exact attention on the selected pages and the latent out-projection.
+        Returns y [B][hidden] (bf16, on the device)."""
+        y = self.y if y is None else y
+        basiskv_decode(self.dims, q, k_new, v_new, self.seq_lens,
+                       self.max_seq_len if max_seq_len is None else max_seq_len,
+                       self.block_table, self.A_V, self.P_K, self.U_K, self.W_fold, self.K,
+                       self.Z, self.E, self.top_k, sel, y, self.workspace, stream)
+        return y

@@ -14,7 +14,8 @@ per-token state of Table 4; model shapes of Figure 3's caption):
   of each column fixed so diag(R) > 0); B_V [r_v][d] ~ N(0, 1/r_v);
   W_O [Hq*d][hidden] ~ N(0, 1/(Hq*d)).  Every factor is rounded to bf16 once.
 * Cache contents for tokens t < T of every (sequence b, KV head g), drawn
-  with ``torch.Generator(device).manual_seed(seed*1000 + 1)``: z ~ N(0,1),
+  per sequence with ``torch.Generator(device).manual_seed(seed*1000 + 1 +
+  100003*layer + 7919*b)`` (so one sequence can be drawn alone): z ~ N(0,1),
   e ~ N(0,1) (both bf16), and the exact key
   K = z.P_K + e.U_K^T + N(0, 0.1^2), rounded to bf16.  This makes part of
   each key predictable from the Value latent, the structure BasisKV's router
@@ -152,24 +153,28 @@ def _dev_gen(device, seed: int) -> torch.Generator:
     return torch.Generator(device=device).manual_seed(seed)
 
 
-def make_cache(wl: Workload, factors: dict, device="cpu", layer: int = 0) -> dict:
-    """Logical caches [B][Hkv][capacity][*] holding T tokens per sequence."""
+def make_cache(wl: Workload, factors: dict, device="cpu", layer: int = 0,
+               seqs=None) -> dict:
+    """Logical caches [len(seqs)][Hkv][capacity][*] holding T tokens for each
+    sequence in ``seqs`` (default: all B)."""
     dev = torch.device(device)
-    gen = _dev_gen(dev, wl.seed * 1000 + 1 + 100003 * layer)
-    B, Hkv, T, cap = wl.B, wl.Hkv, wl.T, wl.capacity_tokens()
+    seqs = list(range(wl.B)) if seqs is None else list(seqs)
+    Hkv, T, cap = wl.Hkv, wl.T, wl.capacity_tokens()
     P_K = factors["P_K"].to(dev, torch.float32)
     U_K = factors["U_K"].to(dev, torch.float32)
-    Z = torch.full((B, Hkv, cap, wl.r_v), FILLER, dtype=torch.bfloat16, device=dev)
-    E = torch.full((B, Hkv, cap, wl.r_k), FILLER, dtype=torch.bfloat16, device=dev)
-    K = torch.full((B, Hkv, cap, wl.d), FILLER, dtype=torch.bfloat16, device=dev)
-    for b in range(B):  # one sequence at a time bounds the fp32 temporaries
+    n = len(seqs)
+    Z = torch.full((n, Hkv, cap, wl.r_v), FILLER, dtype=torch.bfloat16, device=dev)
+    E = torch.full((n, Hkv, cap, wl.r_k), FILLER, dtype=torch.bfloat16, device=dev)
+    K = torch.full((n, Hkv, cap, wl.d), FILLER, dtype=torch.bfloat16, device=dev)
+    for i, b in enumerate(seqs):  # one sequence at a time bounds the temporaries
+        gen = _dev_gen(dev, wl.seed * 1000 + 1 + 100003 * layer + 7919 * b)
         z = torch.randn(Hkv, T, wl.r_v, generator=gen, device=dev).bfloat16()
         e = torch.randn(Hkv, T, wl.r_k, generator=gen, device=dev).bfloat16()
         noise = torch.randn(Hkv, T, wl.d, generator=gen, device=dev) * 0.1
         k = torch.bmm(z.float(), P_K) + torch.bmm(e.float(), U_K.transpose(1, 2)) + noise
-        Z[b, :, :T] = z
-        E[b, :, :T] = e
-        K[b, :, :T] = k.bfloat16()
+        Z[i, :, :T] = z
+        E[i, :, :T] = e
+        K[i, :, :T] = k.bfloat16()
     return {"Z": Z, "E": E, "K": K}
 
 

@@ -1,0 +1,115 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The library must load, export every entry point include/basiskv.h declares,
+and reject invalid calls on the host, before any CUDA call, with the status
+the header documents.  Only fake (aligned, never dereferenced) addresses are
+passed, so nothing reaches a device.
+"""
+import ctypes
+import subprocess
+
+import pytest
+
+import sparse_decode_attention_basiskv_b200 as bkv
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _dims(**kw):
+    base = dict(B=2, Hq=8, Hkv=2, d=128, hidden=256, r_v=64, r_k=32, page_size=16,
+                max_pages_per_seq=64, num_phys_pages=128)
+    base.update(kw)
+    return bkv.Dims(**base)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return bkv.load_library()
+
+
+def test_header_symbols_are_exported(lib):
+    names = bkv.header_symbols()
+    assert len(names) == 10
+    out = subprocess.run(["nm", "-D", "--defined-only", bkv.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    for n in names:
+        assert n in exported, n
+        assert getattr(lib, n)
+
+
+def test_strerror_every_status(lib):
+    for s in range(-6, 1):
+        assert bkv.strerror(s) and "unknown" not in bkv.strerror(s)
+    assert "unknown" in bkv.strerror(-99)
+
+
+def test_workspace_size(lib):
+    d = _dims()
+    n = bkv.workspace_size(d, 8, 1000)
+    assert n > 0 and n % 256 == 0
+    assert bkv.workspace_size(d, 1, 1000) == 0           # top_k < 2
+    assert bkv.workspace_size(d, 8, 64 * 16 + 1) == 0    # longer than a block-table row
+    assert bkv.workspace_size(_dims(d=96), 8, 100) == 0  # unsupported head dim
+    assert bkv.workspace_size(_dims(Hq=6), 8, 100) == 0  # G = 3
+    assert bkv.workspace_size(d, 16, 1000) >= n
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("d", 80, bkv.ERR_UNSUPPORTED_SHAPE),
+    ("r_v", 48, bkv.ERR_UNSUPPORTED_SHAPE),
+    ("r_k", 8, bkv.ERR_UNSUPPORTED_SHAPE),
+    ("page_size", 12, bkv.ERR_UNSUPPORTED_SHAPE),
+    ("hidden", 200, bkv.ERR_UNSUPPORTED_SHAPE),
+    ("Hq", 3, bkv.ERR_UNSUPPORTED_SHAPE),
+    ("B", 0, bkv.ERR_INVALID_ARG),
+    ("num_phys_pages", 0, bkv.ERR_INVALID_ARG),
+])
+def test_route_rejects_bad_dims(lib, field, value, status):
+    d = _dims(**{field: value})
+    rc = lib.basiskv_route(ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, FAKE, FAKE, FAKE, 8,
+                           None, FAKE, FAKE, 1 << 30, None)
+    assert rc == status
+
+
+def test_route_rejects_bad_args(lib):
+    d = _dims()
+    args = [ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, FAKE, FAKE, FAKE, 8, None, FAKE, FAKE,
+            1 << 30, None]
+
+    def call(i, v):
+        a = list(args)
+        a[i] = v
+        return lib.basiskv_route(*a)
+
+    assert call(1, None) == bkv.ERR_INVALID_ARG          # q null
+    assert call(1, FAKE + 2) == bkv.ERR_INVALID_ARG      # q misaligned
+    assert call(11, None) == bkv.ERR_INVALID_ARG         # sel null
+    assert call(9, 1) == bkv.ERR_INVALID_ARG             # top_k < 2
+    assert call(3, 0) == bkv.ERR_INVALID_ARG             # empty context bound
+    assert call(3, 64 * 16 + 1) == bkv.ERR_INVALID_ARG   # past the block-table row
+    assert call(12, FAKE + 16) == bkv.ERR_INVALID_ARG    # workspace not 256-aligned
+    assert call(13, 64) == bkv.ERR_WORKSPACE_TOO_SMALL
+
+
+def test_other_entry_points_validate(lib):
+    d = _dims()
+    big = 1 << 30
+    assert lib.basiskv_attend(ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, FAKE, None, 8, FAKE,
+                              FAKE, big, None) == bkv.ERR_INVALID_ARG
+    assert lib.basiskv_outproj(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 16,
+                               None) == bkv.ERR_WORKSPACE_TOO_SMALL
+    assert lib.basiskv_append(ctypes.byref(d), FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                              FAKE, FAKE, FAKE, big, None) == bkv.ERR_INVALID_ARG
+    assert lib.basiskv_append(ctypes.byref(d), FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                              None, FAKE, FAKE, big, None) == bkv.ERR_INVALID_ARG
+    assert lib.basiskv_decode(ctypes.byref(d), FAKE, FAKE, None, FAKE, 100, FAKE, FAKE, FAKE,
+                              FAKE, FAKE, FAKE, FAKE, FAKE, 8, None, FAKE, FAKE, big,
+                              None) == bkv.ERR_INVALID_ARG  # k_new without v_new
+    assert lib.basiskv_decode(ctypes.byref(d), FAKE, None, None, FAKE, 100, FAKE, FAKE, FAKE,
+                              FAKE, FAKE, FAKE, FAKE, FAKE, 8, None, None, FAKE, big,
+                              None) == bkv.ERR_INVALID_ARG  # y null
+    assert lib.basiskv_fold_outproj(ctypes.byref(_dims(d=72)), FAKE, FAKE, FAKE,
+                                    None) == bkv.ERR_UNSUPPORTED_SHAPE
+    flags = ctypes.c_uint32(7)
+    assert lib.basiskv_read_device_status(None, None) == bkv.ERR_INVALID_ARG

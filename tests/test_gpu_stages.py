@@ -1,0 +1,236 @@
+"""Stage-by-stage parity of the CUDA path (through the C-ABI) with the CPU
+oracle, at sizes the oracle finishes in seconds that still span several
+tiles and a ragged tail, plus the edge cases of the method."""
+import numpy as np
+import pytest
+import torch
+
+import sparse_decode_attention_basiskv_b200 as bkv
+from oracle import basiskv_oracle as O
+from sparse_decode_attention_basiskv_b200 import synth
+
+from harness import (A_REL, S_REL, Y_ABS, Y_REL, ZE_REL, assert_within, compare_selection,
+                     factors_np, gpu_layer, np64, oracle_route, status_clean)
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": synth.TINY,
+    "llama4k": synth.LLAMA8B_T4K,
+    # the headline layer shape (r_v 64, B 16) at a context the oracle finishes fast
+    "llama_b16_t2k": synth.with_sizes(synth.LLAMA8B_T32K_B16, T=2000, top_k=32),
+    # the Qwen3-32B layer shape (G 8, page 32) at a short context
+    "qwen_b2_t3k": synth.with_sizes(synth.QWEN32B_T64K_B8, B=2, T=3000, prefill_tokens=0),
+}
+
+
+@pytest.fixture(scope="module", params=list(SMALL))
+def setup(request):
+    wl = SMALL[request.param]
+    pb, layer = gpu_layer(wl)
+    return wl, pb, layer
+
+
+def test_fold_outproj(setup):
+    wl, pb, layer = setup
+    f = factors_np(pb)
+    ref = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)  # [Hq][r_v][H]
+    got = np64(layer.W_fold).reshape(wl.hidden, wl.Hq, wl.r_v).transpose(1, 2, 0)
+    tol = 2.0 ** -8 * np.abs(ref) + 1e-5 * np.abs(ref).max()
+    assert (np.abs(got - ref) <= tol).all()
+
+
+def test_route_and_select(setup):
+    wl, pb, layer = setup
+    B, Hkv = wl.B, wl.Hkv
+    scores = torch.full((B, Hkv, layer.dims.max_pages_per_seq), float("nan"), device="cuda")
+    sel = torch.empty(B, Hkv, wl.top_k, dtype=torch.int32, device="cuda")
+    bkv.basiskv_route(layer.dims, pb.q, layer.seq_lens, wl.T, layer.block_table, layer.P_K,
+                      layer.U_K, layer.Z, layer.E, wl.top_k, scores, sel, layer.workspace)
+    status_clean()
+    P = wl.pages
+    stats = {}
+    for b in range(B):
+        for g in range(Hkv):
+            sc, ref_sel, tie = oracle_route(pb, b, g, wl.T)
+            assert_within(np64(scores[b, g, :P]), sc, S_REL, what=f"scores b{b} g{g}")
+            compare_selection(sel[b, g].cpu().numpy(), ref_sel, tie, stats)
+    assert stats.get("clean_mismatch", 0) == 0, stats
+
+
+def test_attend_on_oracle_selection(setup):
+    wl, pb, layer = setup
+    B, Hkv, G = wl.B, wl.Hkv, wl.G
+    f = factors_np(pb)
+    ref_sel = np.zeros((B, Hkv, wl.top_k), dtype=np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            ref_sel[b, g] = oracle_route(pb, b, g, wl.T)[1]
+    sel = torch.from_numpy(ref_sel).cuda()
+    a = torch.empty(B, wl.Hq, wl.r_v, device="cuda")
+    bkv.basiskv_attend(layer.dims, pb.q, layer.seq_lens, wl.T, layer.block_table, layer.K,
+                       layer.Z, sel, wl.top_k, a, layer.workspace)
+    status_clean()
+    for b in range(B):
+        for g in range(Hkv):
+            qg = np64(pb.q[b, g * G:(g + 1) * G])
+            ref, _ = O.attend(qg, np64(pb.cache["K"][b, g]), np64(pb.cache["Z"][b, g]),
+                              ref_sel[b, g], wl.T, wl.page_size)
+            assert_within(np64(a[b, g * G:(g + 1) * G]), ref, A_REL, what=f"a b{b} g{g}")
+
+
+def test_outproj(setup):
+    wl, pb, layer = setup
+    gen = torch.Generator(device="cuda").manual_seed(11)
+    a = torch.randn(wl.B, wl.Hq, wl.r_v, generator=gen, device="cuda")
+    y = torch.empty(wl.B, wl.hidden, dtype=torch.bfloat16, device="cuda")
+    bkv.basiskv_outproj(layer.dims, a, layer.W_fold, y, layer.workspace)
+    status_clean()
+    f = factors_np(pb)
+    W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
+    for b in range(wl.B):
+        assert_within(np64(y[b]), O.outproj(np64(a[b]), W), Y_REL, Y_ABS, what=f"y b{b}")
+
+
+def test_decode_step_with_append(setup):
+    """Fused step: append one token per sequence, then route, attend and
+    out-project over T + 1 tokens; compared with the oracle's own append."""
+    wl, pb, layer = setup
+    f = factors_np(pb)
+    k_new, v_new = synth.make_tokens(wl, pb.factors, 1, device="cuda")
+    k_new, v_new = k_new[:, 0].contiguous(), v_new[:, 0].contiguous()
+    sel = torch.empty(wl.B, wl.Hkv, wl.top_k, dtype=torch.int32, device="cuda")
+    seq0 = layer.seq_lens.clone()
+    y = layer.decode(pb.q, k_new, v_new, sel=sel, max_seq_len=wl.T + 1).clone()
+    status_clean()
+    assert torch.equal(layer.seq_lens, seq0 + 1)
+    W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
+    stats = {}
+    for b in range(wl.B):
+        c = {k: np64(v[b]) for k, v in pb.cache.items()}
+        out = O.decode_sequence(np64(pb.q[b]), c["K"], c["Z"], c["E"], wl.T, wl.page_size,
+                                wl.top_k, f["P_K"], f["U_K"], W, k_new=np64(k_new[b]),
+                                v_new=np64(v_new[b]), A_V=f["A_V"])
+        # appended state, read back from the paged caches
+        for g in range(wl.Hkv):
+            slot = (layer.block_table[b, wl.T // wl.page_size].item(), g, wl.T % wl.page_size)
+            assert_within(np64(layer.Z[slot]), out["z_new"][g], ZE_REL, what="z")
+            assert_within(np64(layer.E[slot]), out["e_new"][g], ZE_REL, what="e")
+            assert torch.equal(layer.K[slot], k_new[b, g])
+            compare_selection(sel[b, g].cpu().numpy(), out["sel"][g], out["near_tie"][g], stats)
+        if not out["near_tie"].any():
+            assert_within(np64(y[b]), out["y"], Y_REL, Y_ABS, what=f"y b{b}")
+    assert stats.get("clean_mismatch", 0) == 0, stats
+    # undo the append for the other tests of this module
+    layer.seq_lens.copy_(seq0)
+
+
+def test_ragged_lengths_and_degenerate_pages():
+    """Lengths that end mid-page, exactly on a page, inside the first page
+    (sink == newest), and contexts with fewer pages than top_k."""
+    wl = synth.with_sizes(synth.LLAMA8B_T4K, B=6, T=1200, top_k=16)
+    lens = [1, 15, 16, 17, 700, 1200]
+    pb, layer = gpu_layer(wl, seq_lens=lens)
+    sel = torch.empty(wl.B, wl.Hkv, wl.top_k, dtype=torch.int32, device="cuda")
+    y = layer.decode(pb.q, sel=sel, max_seq_len=max(lens)).clone()
+    status_clean()
+    f = factors_np(pb)
+    W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
+    for b, T in enumerate(lens):
+        c = {k: np64(v[b]) for k, v in pb.cache.items()}
+        out = O.decode_sequence(np64(pb.q[b]), c["K"], c["Z"], c["E"], T, wl.page_size,
+                                wl.top_k, f["P_K"], f["U_K"], W)
+        if not out["near_tie"].any():
+            assert np.array_equal(sel[b].cpu().numpy(), out["sel"]), b
+            assert_within(np64(y[b]), out["y"], Y_REL, Y_ABS, what=f"y b{b}")
+    assert sel[0, 0, 0].item() == 0 and (sel[0, 0, 1:] == -1).all()  # one page
+
+
+def test_dense_when_top_k_covers_context():
+    """top_k >= P: every page is attended, so the result is plain attention."""
+    wl = synth.with_sizes(synth.TINY, top_k=40)  # 32 pages
+    pb, layer = gpu_layer(wl)
+    sel = torch.empty(1, 1, 40, dtype=torch.int32, device="cuda")
+    y = layer.decode(pb.q, sel=sel, max_seq_len=wl.T).clone()
+    status_clean()
+    assert sel[0, 0].tolist() == list(range(32)) + [-1] * 8
+    f = factors_np(pb)
+    W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
+    c = {k: np64(v[0]) for k, v in pb.cache.items()}
+    out = O.decode_sequence(np64(pb.q[0]), c["K"], c["Z"], c["E"], wl.T, 16, 40, f["P_K"],
+                            f["U_K"], W)
+    assert_within(np64(y[0]), out["y"], Y_REL, Y_ABS)
+
+
+def test_block_table_permutation_invariance():
+    """Different physical placements of the same logical pages give
+    bit-identical scores, selection and output."""
+    wl = synth.with_sizes(synth.LLAMA8B_T4K, B=2, T=1000, top_k=16)
+    pb, layer = gpu_layer(wl)
+    sc1 = torch.zeros(2, 8, layer.dims.max_pages_per_seq, device="cuda")
+    sel1 = torch.empty(2, 8, 16, dtype=torch.int32, device="cuda")
+    bkv.basiskv_route(layer.dims, pb.q, layer.seq_lens, wl.T, layer.block_table, layer.P_K,
+                      layer.U_K, layer.Z, layer.E, 16, sc1, sel1, layer.workspace)
+    y1 = layer.decode(pb.q, max_seq_len=wl.T).clone()
+    # a second placement: reverse the physical order
+    n = layer.dims.num_phys_pages
+    table2 = (n - 1 - layer.block_table).contiguous()
+    perm = (n - 1 - torch.arange(n, device="cuda"))
+    for name in ("K", "Z", "E"):
+        getattr(layer, name).copy_(getattr(layer, name)[perm].clone())
+    layer.block_table = table2
+    sc2 = torch.zeros_like(sc1)
+    sel2 = torch.empty_like(sel1)
+    bkv.basiskv_route(layer.dims, pb.q, layer.seq_lens, wl.T, layer.block_table, layer.P_K,
+                      layer.U_K, layer.Z, layer.E, 16, sc2, sel2, layer.workspace)
+    y2 = layer.decode(pb.q, max_seq_len=wl.T).clone()
+    status_clean()
+    assert torch.equal(sc1, sc2) and torch.equal(sel1, sel2) and torch.equal(y1, y2)
+
+
+def test_prefill_chunk_append():
+    """A 4096-token prefill chunk appended to one sequence of the Qwen3-32B
+    layer shape (B = 1 view of the batch), compared token by token."""
+    wl = synth.with_sizes(synth.QWEN32B_T64K_B8, B=2, T=96, prefill_tokens=4096)
+    pb, layer = gpu_layer(wl)
+    f = factors_np(pb)
+    k, v = synth.make_tokens(wl, pb.factors, 4096, device="cuda", stream_id=99)
+    b = 1
+    dims1 = bkv.Dims(B=1, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, hidden=wl.hidden, r_v=wl.r_v,
+                     r_k=wl.r_k, page_size=wl.page_size,
+                     max_pages_per_seq=layer.dims.max_pages_per_seq,
+                     num_phys_pages=layer.dims.num_phys_pages)
+    bkv.basiskv_append(dims1, k[b].contiguous(), v[b].contiguous(), 4096, layer.seq_lens[b:],
+                       layer.block_table[b], layer.A_V, layer.P_K, layer.U_K, layer.K, layer.Z,
+                       layer.E, layer.workspace)
+    status_clean()
+    assert layer.seq_lens.tolist() == [wl.T, wl.T + 4096]
+    for g in range(wl.Hkv):
+        z_ref, e_ref = O.append_latents(np64(k[b, :, g]), np64(v[b, :, g]), f["A_V"][g],
+                                        f["P_K"][g], f["U_K"][g])
+        toks = np.arange(wl.T, wl.T + 4096)
+        phys = layer.block_table[b, toks // wl.page_size].long().cpu()
+        rows = torch.as_tensor(toks % wl.page_size)
+        assert_within(np64(layer.Z[phys, g, rows]), z_ref, ZE_REL, what="prefill z")
+        assert_within(np64(layer.E[phys, g, rows]), e_ref, ZE_REL, what="prefill e")
+        assert torch.equal(layer.K[phys, g, rows], k[b, :, g])
+
+
+def test_device_status_reports_bad_inputs():
+    """A block-table entry outside the cache and an append past the
+    block-table row are caught by the kernels' own checks: the work is
+    skipped and the status word says why."""
+    wl = synth.with_sizes(synth.TINY, T=100)
+    pb, layer = gpu_layer(wl)
+    status_clean()
+    layer.block_table[0, 3] = layer.dims.num_phys_pages + 5
+    layer.decode(pb.q, max_seq_len=wl.T)
+    assert bkv.read_device_status() & bkv.DEV_BAD_PAGE
+    assert bkv.read_device_status() == 0  # cleared
+    layer.block_table[0, 3] = 3
+    cap = layer.dims.max_pages_per_seq * wl.page_size
+    layer.seq_lens.fill_(cap)
+    k_new, v_new = synth.make_tokens(wl, pb.factors, 1, device="cuda")
+    layer.decode(pb.q, k_new[:, 0].contiguous(), v_new[:, 0].contiguous(), max_seq_len=cap)
+    assert bkv.read_device_status() & bkv.DEV_OVERFLOW
+    assert layer.seq_lens.item() == cap
