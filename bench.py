@@ -244,7 +244,7 @@ def run_gpu(args) -> None:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
 
     K, W = args.steps, args.warmup
-    wl = synth.with_sizes(WL, steps=K + W)
+    wl = synth.with_sizes(WL, steps=K + W, B=args.batch or WL.B, T=args.context or WL.T)
     pb = synth.make_problem(wl, device="cuda")
     layer = DecodeLayer.from_problem(pb)
     T0 = wl.T
@@ -366,11 +366,13 @@ def run_gpu(args) -> None:
         "tokens_per_s": world * wl.B / (ms_per_step / 1e3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded generators; planted-page queries)",
-        "config": {"workload": WL.name, "global_batch": wl.B * world, "seq_len": T0,
+        "config": {"workload": WL.name if (wl.B, wl.T) == (WL.B, WL.T) else
+                   f"{WL.name} at B={wl.B}, T={wl.T}",
+                   "global_batch": wl.B * world, "seq_len": T0,
                    "context": f"{T0} -> {T0 + W + K} tokens (one appended per step)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (~1.9 GB of cache per step); no flush",
-                   **{k: v for k, v in WL.describe().items() if k not in ("name", "steps")}},
+                   **{k: v for k, v in wl.describe().items() if k not in ("name", "steps")}},
         "bytes_per_step": avg,
         "frac_of_peak": value / world / (peak / 1e3),
         "roofline": {"bound": "hbm", "kernel": "route (fold + page scoring + select)",
@@ -402,6 +404,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the batch (smaller cases for profiling)")
+    ap.add_argument("--context", type=int, default=0,
+                    help="override the context length (smaller cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

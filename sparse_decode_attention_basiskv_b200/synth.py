@@ -78,8 +78,10 @@ class Workload:
         return -(-self.T // self.page_size)
 
     def capacity_tokens(self) -> int:
-        """Token slots per sequence: context plus every token appended."""
-        return self.T + self.append_tokens * self.steps + self.prefill_tokens
+        """Token slots per sequence: context, every token appended, and one
+        page of slack (room for an extra decode token in any workload)."""
+        return (self.T + self.append_tokens * self.steps + self.prefill_tokens
+                + self.page_size)
 
     def pages_capacity(self) -> int:
         return -(-self.capacity_tokens() // self.page_size)
