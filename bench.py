@@ -142,7 +142,7 @@ def oracle_sample(wl, device_cache=None):
     import numpy as np
     factors = synth.make_factors(wl)
     cache = synth.make_cache(wl, factors, "cpu", seqs=[0])
-    q, _ = synth.make_query(wl, cache["K"], wl.T)
+    q, _ = synth.make_query(synth.with_sizes(wl, B=1), cache["K"], wl.T)
     k, v = synth.make_tokens(wl, factors, 1, "cpu")
     f = {n: t.double().numpy() for n, t in factors.items()}
     c = {n: t[0, 0].double().numpy() for n, t in cache.items()}

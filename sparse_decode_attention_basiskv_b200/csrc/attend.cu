@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                                              ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + geo.smem_bytes);
   uint64_t* empty = full + geo.stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + geo.stages);
   float* qs = reinterpret_cast<float*>(smem + geo.q_off);     // [G][d], pre-scaled
   float* ps = reinterpret_cast<float*>(smem + geo.p_off);     // [128][G]
   float* red = reinterpret_cast<float*>(smem + geo.red_off);  // [2][warps][G]
@@ -58,6 +59,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kAttConsumerWarps);
     }
+    *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == kAttConsumerWarps && lane == 0) {
@@ -83,10 +85,12 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         for (int k = 0; k < geo.ppi && j * geo.ppi + k < a.top_k; ++k) npg += sel[k] >= 0;
         if (npg == 0) continue;
         const int s = it % geo.stages;
-        if (!mbar_wait(&empty[s], ((it / geo.stages) & 1) ^ 1, a.status)) break;
+        ++it;
+        if (!mbar_wait_or_abort(&empty[s], (((it - 1) / geo.stages) & 1) ^ 1, a.status,
+                                abort_flag))
+          continue;  // aborted: issue nothing more
         uint8_t* st = smem + (size_t)s * geo.stage_bytes;
         mbar_arrive_expect_tx(&full[s], npg * S * (d + r_v) * 2);
-        int slot = 0;
         for (int k = 0; k < geo.ppi && j * geo.ppi + k < a.top_k; ++k) {
           const int lp = sel[k];
           if (lp < 0) continue;
@@ -102,9 +106,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
           for (int zb = 0; zb < geo.nzb; ++zb)
             tma_load_2d(st + geo.z_off + (k * geo.nzb + zb) * geo.zbox, &tmZ, zb * geo.wz, row,
                         &full[s]);
-          ++slot;
         }
-        ++it;
       }
     }
     return;
@@ -128,7 +130,9 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     int T = a.seq_lens[b];
     T = T < 0 ? 0 : T;
     const int s = it % geo.stages;
-    if (!mbar_wait(&full[s], (it / geo.stages) & 1, a.status)) break;
+    // On a timeout every later wait fails at once; the item is skipped but
+    // the barrier sequence below is kept, so all consumer warps stay in step.
+    const bool ready = mbar_wait_or_abort(&full[s], (it / geo.stages) & 1, a.status, abort_flag);
     const uint32_t st = smem_u32(smem + (size_t)s * geo.stage_bytes);
 
     // Query of the group, scaled so that exp2 gives the softmax.
@@ -137,7 +141,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     named_bar_sync(1, kAttTokens);
 
     const int lp = page_local < nk ? sel[page_local] : -1;
-    const bool valid = lp >= 0 && lp * S + row < T;
+    const bool valid = ready && lp >= 0 && lp * S + row < T;
     float sc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) sc[h] = -INFINITY;
@@ -194,7 +198,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     }
     named_bar_sync(1, kAttTokens);
     // Latent accumulation: thread = (head, 8-wide chunk) slot x token group.
-    if (tid < nact) {
+    if (ready && tid < nact) {
       const int slot = tid % nslot, grp = tid / nslot;
       const int h = slot / (r_v / 8), c = slot % (r_v / 8);
       const int box = c / zc_per_box, cc = c - box * zc_per_box;
@@ -225,13 +229,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     // All reads of the stage are done: release it to the producer.
     if (lane == 0) mbar_arrive(&empty[s]);
     float* out = a.partial + ((size_t)bg * a.nsplit + j) * G * (r_v + 2);
-    for (int i = tid; i < G * r_v; i += kAttTokens) {
+    for (int i = tid; ready && i < G * r_v; i += kAttTokens) {
       const int h = i / r_v, jj = i % r_v;
       float v = 0.f;
       for (int gi = 0; gi < ngrp; ++gi) v += accs[(size_t)gi * G * r_v + i];
       out[h * (r_v + 2) + 2 + jj] = v;
     }
-    if (tid < G) {
+    if (ready && tid < G) {
       float l = 0.f;
       for (int w = 0; w < kAttConsumerWarps; ++w) l += red[(kAttConsumerWarps + w) * G + tid];
       out[tid * (r_v + 2)] = mh[tid];
@@ -301,7 +305,7 @@ AttendGeom attend_geometry(int G, int d, int r_v, int S, int wz) {
 template <int G>
 cudaError_t launch_attend_g(const AttendArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmZ,
                             const AttendGeom& geo, cudaStream_t st, bool pdl) {
-  const size_t smem = (size_t)geo.smem_bytes + 2 * geo.stages * 8 + 1024;
+  const size_t smem = (size_t)geo.smem_bytes + 2 * geo.stages * 8 + 16 + 1024;
   cudaError_t e = cudaFuncSetAttribute(attend_kernel<G>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -83,6 +83,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return true;
 }
 
+// Like mbar_wait, for kernels whose threads also meet at named barriers: a
+// timeout sets the CTA-wide `abort` flag, and once it is set every later wait
+// returns false at once.  Callers then skip their work but keep executing the
+// same sequence of barriers, so no thread is ever left waiting for one that
+// stopped early.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t parity,
+                                                   unsigned int* status, volatile int* abort) {
+  if (*abort) return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      raise_status(status, BASISKV_DEV_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
 // ------------------------------------------------------------ TMA and bulk
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -135,6 +156,19 @@ __device__ __forceinline__ uint32_t swz(uint32_t addr, uint32_t mask) {
 // bf16 pair (one 32-bit word) -> two fp32 values: exact bit placement.
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// A bf16 pair as (even, odd) fp32 values.
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// d += a * b on two fp32 lanes with one instruction (fma.rn.f32x2, sm_100).
+__device__ __forceinline__ void ffma2(float2& d, const float2& a, const float2& b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;"
+      : "+l"(reinterpret_cast<unsigned long long&>(d))
+      : "l"(reinterpret_cast<const unsigned long long&>(a)),
+        "l"(reinterpret_cast<const unsigned long long&>(b)));
+}
 
 __device__ __forceinline__ float bf16_to_f(uint16_t h) {
   return __uint_as_float(static_cast<uint32_t>(h) << 16);

@@ -242,6 +242,185 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   }
 }
 
+
+// ----------------------------------------------- page scoring, specialised
+// The same stream with the head count and the state widths fixed at compile
+// time.  Each consumer thread copies its token's whole row (r_v + r_k bf16)
+// from the stage into registers and releases the stage at once, so shared
+// memory holds data in flight rather than data being computed on; the folded
+// queries live in a per-group buffer that is refreshed when the (sequence,
+// KV head) changes.  Two groups of seven consumer warps take alternate
+// stages, and the G dot products use packed fp32x2 FMAs.
+constexpr int kRsGroupThreads = 224;  // tokens per stage (7 warps: 16 warps per CTA in all)
+constexpr int kRsGroups = 2;
+constexpr int kRsThreads = kRsGroups * kRsGroupThreads + 32;
+constexpr int kRsProducerWarp = kRsGroups * kRsGroupThreads / 32;
+
+struct RsGeom {
+  int np;           // pages per stage
+  int page_bytes;   // 1 KB multiple
+  int stage_bytes;  // 1 KB multiple
+  int stages;
+  int q_off;        // per-group folded-query buffers, after the ring
+  int bar_off;
+};
+
+template <int G, int RV, int RK>
+__global__ void __launch_bounds__(kRsThreads, 1)
+    route_rs_kernel(const __grid_constant__ CUtensorMap tmZ,
+                    const __grid_constant__ CUtensorMap tmE, RouteArgs a, RsGeom geo) {
+  constexpr int WZ = 32, WE = (RK % 32 == 0) ? 32 : 16;
+  constexpr int NZB = RV / WZ, NEB = RK / WE;
+  constexpr int NZC = RV / 8, NEC = RK / 8, NCH = NZC + NEC, RQ = RV + RK;
+  constexpr uint32_t ZM = 3u, EM = (WE == 32) ? 3u : 1u;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + geo.bar_off);
+  uint64_t* empty = full + geo.stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + geo.stages);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = a.S;
+  const int zbox = S * WZ * 2, ebox = S * WE * 2;
+  if (tid == 0) {
+    for (int s = 0; s < geo.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kRsGroupThreads / 32);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kRsProducerWarp && lane == 0) {
+    prefetch_tmap(&tmZ);
+    prefetch_tmap(&tmE);
+  }
+  __syncthreads();
+  pdl_wait();
+
+  const int P_max = (a.max_seq_len + S - 1) / S;
+  const int tiles_per_bg = (P_max + geo.np - 1) / geo.np;
+  const long total = (long)a.B * a.Hkv * tiles_per_bg;
+  const long t_begin = total * blockIdx.x / gridDim.x;
+  const long t_end = total * (blockIdx.x + 1) / gridDim.x;
+
+  if (warp == kRsProducerWarp) {
+    // ------------------------------------------------------------ producer
+    // The whole warp: lane j fetches page j's block-table entry and issues
+    // that page's boxes, so a tile's gathers go out in parallel.
+    int it = 0, cur_b = -1, T = 0;
+    for (long tile = t_begin; tile < t_end; ++tile) {
+      int bg, b, g, ti;
+      decode_tile(tile, tiles_per_bg, a.Hkv, bg, b, g, ti);
+      if (b != cur_b) {
+        T = clamp_len(a.seq_lens[b], a.max_seq_len, a.status, false);
+        cur_b = b;
+      }
+      const int P = (T + S - 1) / S, p0 = ti * geo.np;
+      if (p0 >= P) continue;
+      const int npg = min(geo.np, P - p0);
+      const int s = it % geo.stages;
+      ++it;
+      int pp = 0;
+      if (lane < npg) pp = a.block_table[(size_t)b * a.max_pages + p0 + lane];
+      bool go = true;
+      if (lane == 0) {
+        go = mbar_wait_or_abort(&empty[s], (((it - 1) / geo.stages) & 1) ^ 1, a.status,
+                                abort_flag);
+        if (go) mbar_arrive_expect_tx(&full[s], npg * S * RQ * 2);
+      }
+      go = __shfl_sync(0xffffffffu, go, 0);
+      if (!go) continue;  // aborted: issue nothing more
+      if (lane < npg) {
+        if (pp < 0 || pp >= a.num_phys) {
+          raise_status(a.status, BASISKV_DEV_BAD_PAGE);
+          pp = 0;  // keep the byte count; the page's score is flagged garbage
+        }
+        const int row = (pp * a.Hkv + g) * S;
+        uint8_t* pg = smem + (size_t)s * geo.stage_bytes + lane * geo.page_bytes;
+#pragma unroll
+        for (int k = 0; k < NZB; ++k) tma_load_2d(pg + k * zbox, &tmZ, k * WZ, row, &full[s]);
+#pragma unroll
+        for (int k = 0; k < NEB; ++k)
+          tma_load_2d(pg + NZB * zbox + k * ebox, &tmE, k * WE, row, &full[s]);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------- consumers
+  const int group = tid / kRsGroupThreads, gtid = tid % kRsGroupThreads;
+  const int page_local = gtid / S, row = gtid % S;
+  float* qbuf = reinterpret_cast<float*>(smem + geo.q_off) + group * G * RQ;
+  int cur_bg = -1, cur_b = -1, T = 0;
+  int it = 0;
+  for (long tile = t_begin; tile < t_end; ++tile) {
+    int bg, b, g, ti;
+    decode_tile(tile, tiles_per_bg, a.Hkv, bg, b, g, ti);
+    if (b != cur_b) {
+      T = clamp_len(a.seq_lens[b], a.max_seq_len, a.status, tid == 0);
+      cur_b = b;
+    }
+    const int P = (T + S - 1) / S, p0 = ti * geo.np;
+    if (p0 >= P) continue;
+    const int my = it++;
+    if ((my % kRsGroups) != group) continue;
+    const int npg = min(geo.np, P - p0);
+    if (bg != cur_bg) {  // refresh the group's folded queries (uniform control flow)
+      named_bar_sync(1 + group, kRsGroupThreads);
+      const float* src = a.qt + ((size_t)b * a.Hkv * G + (size_t)g * G) * RQ;
+      for (int i = gtid; i < G * RQ; i += kRsGroupThreads) qbuf[i] = src[i];
+      named_bar_sync(1 + group, kRsGroupThreads);
+      cur_bg = bg;
+    }
+    const int s = my % geo.stages;
+    const bool ready = mbar_wait_or_abort(&full[s], (my / geo.stages) & 1, a.status, abort_flag);
+    const int p = p0 + page_local;
+    const bool valid = ready && page_local < npg && p * S + row < T;
+    uint4 x[NCH];
+    if (valid) {
+      const uint8_t* pg = smem + (size_t)s * geo.stage_bytes + page_local * geo.page_bytes;
+#pragma unroll
+      for (int c = 0; c < NZC; ++c) {
+        const uint32_t off = (c / 4) * zbox + row * (WZ * 2) + (c % 4) * 16;
+        x[c] = *reinterpret_cast<const uint4*>(pg + swz(off, ZM));
+      }
+#pragma unroll
+      for (int c = 0; c < NEC; ++c) {
+        const uint32_t off =
+            NZB * zbox + (c / (WE / 8)) * ebox + row * (WE * 2) + (c % (WE / 8)) * 16;
+        x[NZC + c] = *reinterpret_cast<const uint4*>(pg + swz(off, EM));
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);  // the rows are in registers now
+    float best = -INFINITY;
+    if (valid) {
+      float2 acc[G][2];
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        const float2 p0v = bf16x2_to_f2(x[c].x), p1v = bf16x2_to_f2(x[c].y);
+        const float2 p2v = bf16x2_to_f2(x[c].z), p3v = bf16x2_to_f2(x[c].w);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float4 qa = *reinterpret_cast<const float4*>(qbuf + h * RQ + c * 8);
+          const float4 qb = *reinterpret_cast<const float4*>(qbuf + h * RQ + c * 8 + 4);
+          ffma2(acc[h][0], p0v, make_float2(qa.x, qa.y));
+          ffma2(acc[h][1], p1v, make_float2(qa.z, qa.w));
+          ffma2(acc[h][0], p2v, make_float2(qb.x, qb.y));
+          ffma2(acc[h][1], p3v, make_float2(qb.z, qb.w));
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        best = fmaxf(best, (acc[h][0].x + acc[h][1].x) + (acc[h][0].y + acc[h][1].y));
+    }
+    for (int o = S >> 1; o > 0; o >>= 1) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+    if (ready && row == 0 && page_local < npg) a.scores[(size_t)bg * a.max_pages + p] = best;
+  }
+}
+
 // -------------------------------------------------------- page selection
 // Per (sequence, KV head): sink page 0 and newest page P-1 always; the other
 // top_k - 2 slots go to the best remaining pages by (score desc, index asc),
@@ -417,6 +596,33 @@ cudaError_t launch_route_g(const RouteArgs& a, const CUtensorMap& tmZ, const CUt
                   tmZ, tmE, a, geo);
 }
 
+template <int G, int RV, int RK>
+cudaError_t launch_route_rs(const RouteArgs& a, const CUtensorMap& tmZ, const CUtensorMap& tmE,
+                            cudaStream_t st, bool pdl) {
+  RsGeom geo{};
+  geo.np = kRsGroupThreads / a.S;
+  geo.page_bytes = (a.S * (RV + RK) * 2 + 1023) / 1024 * 1024;
+  geo.stage_bytes = geo.np * geo.page_bytes;
+  const int qbytes = kRsGroups * G * (RV + RK) * 4;
+  const int budget = 224 * 1024 - qbytes - 1024 - 256;
+  geo.stages = budget / geo.stage_bytes;
+  if (geo.stages > 8) geo.stages = 8;
+  if (geo.stages < kRsGroups + 1) return cudaErrorInvalidConfiguration;
+  geo.q_off = geo.stages * geo.stage_bytes;
+  geo.bar_off = geo.q_off + qbytes;
+  const size_t smem = (size_t)geo.bar_off + 2 * geo.stages * 8 + 16 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(route_rs_kernel<G, RV, RK>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int P_max = (a.max_seq_len + a.S - 1) / a.S;
+  const long tiles = (long)a.B * a.Hkv * ((P_max + geo.np - 1) / geo.np);
+  long grid = num_sms();
+  if (grid > tiles) grid = tiles;
+  if (grid < 1) grid = 1;
+  return launch_k(route_rs_kernel<G, RV, RK>, dim3((unsigned)grid), dim3(kRsThreads), smem, st,
+                  pdl, tmZ, tmE, a, geo);
+}
+
 }  // namespace
 
 cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl) {
@@ -428,6 +634,18 @@ cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl) {
 cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
                                 const CUtensorMap& tmE, int wz, int we, cudaStream_t st,
                                 bool pdl) {
+  if (wz == 32 && we == (a.r_k % 32 == 0 ? 32 : 16)) {
+#define BKV_RS(GG, V, K) \
+  if (a.G == GG && a.r_v == V && a.r_k == K) return launch_route_rs<GG, V, K>(a, tmZ, tmE, st, pdl);
+    BKV_RS(4, 32, 16)
+    BKV_RS(4, 64, 32)
+    BKV_RS(4, 96, 32)
+    BKV_RS(4, 128, 32)
+    BKV_RS(8, 64, 32)
+    BKV_RS(8, 96, 32)
+    BKV_RS(8, 128, 32)
+#undef BKV_RS
+  }
   const RouteGeom geo = route_geometry(a.G, a.r_v, a.r_k, a.S, wz, we);
   if (geo.stages < 2) return cudaErrorInvalidConfiguration;
   switch (a.G) {
