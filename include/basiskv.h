@@ -98,7 +98,8 @@ enum basiskv_status {
   BASISKV_ERR_WORKSPACE_TOO_SMALL = -3,
   BASISKV_ERR_LAUNCH_FAILED = -4,     /* a kernel launch was rejected */
   BASISKV_ERR_DEVICE = -5,            /* the device status word was non-zero */
-  BASISKV_ERR_CUDA = -6               /* another CUDA runtime call failed */
+  BASISKV_ERR_CUDA = -6,              /* another CUDA runtime call failed */
+  BASISKV_ERR_SCRATCH_LIMIT = -7      /* needs more than the static scratch holds */
 };
 
 /* Device status bits (basiskv_read_device_status). */
@@ -206,6 +207,39 @@ BASISKV_API int basiskv_decode(const basiskv_dims* dims, const basiskv_bf16* q,
                    basiskv_bf16* Z_cache, basiskv_bf16* E_cache, int top_k,
                    int32_t* sel, basiskv_bf16* y, void* workspace,
                    size_t workspace_bytes, void* stream);
+
+/* Size of the static device scratch array behind basiskv_decode_noalloc. */
+#define BASISKV_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* basiskv_decode for callers that cannot allocate device memory.  The paper
+ * has no counterpart: this is a deployment variant of the fused decode step.
+ *
+ * Some callers cannot call cudaMalloc when they run a step: a runtime that
+ * owns all device memory through its own pool and forbids side allocations,
+ * a plug-in invoked where allocation is not allowed, or a service that must
+ * keep its footprint fixed after start-up.  This entry point takes the same
+ * arguments as basiskv_decode minus the workspace; the scratch comes from a
+ * static __device__ array of BASISKV_NOALLOC_SCRATCH_BYTES (32 MiB) compiled
+ * into the library, which every GPU that loads the library holds until the
+ * process exits.  It allocates nothing itself.
+ *   - Shapes whose basiskv_workspace_size exceeds the array return
+ *     BASISKV_ERR_SCRATCH_LIMIT and launch nothing.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents (nothing in it needs to start at zero).  Calls that may
+ *     overlap on the GPU (two streams, two host threads) race on it: order
+ *     them on one stream, or use basiskv_decode with separate workspaces. */
+BASISKV_API int basiskv_decode_noalloc(const basiskv_dims* dims, const basiskv_bf16* q,
+                                       const basiskv_bf16* k_new,
+                                       const basiskv_bf16* v_new, int32_t* seq_lens,
+                                       int max_seq_len, const int32_t* block_table,
+                                       const basiskv_bf16* A_V, const basiskv_bf16* P_K,
+                                       const basiskv_bf16* U_K, const basiskv_bf16* W_fold,
+                                       basiskv_bf16* K_cache, basiskv_bf16* Z_cache,
+                                       basiskv_bf16* E_cache, int top_k, int32_t* sel,
+                                       basiskv_bf16* y, void* stream);
 
 /* Waits for `stream`, then returns the device status word in *flags (a
  * HOST pointer; BASISKV_DEV_* bits, 0 = clean) and clears it.  Returns

@@ -25,6 +25,8 @@ ERR_WORKSPACE_TOO_SMALL = -3
 ERR_LAUNCH_FAILED = -4
 ERR_DEVICE = -5
 ERR_CUDA = -6
+ERR_SCRATCH_LIMIT = -7
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 DEV_BAD_PAGE = 0x1
 DEV_OVERFLOW = 0x2
@@ -65,6 +67,8 @@ _SIGNATURES = {
     "basiskv_outproj": (_I, [_DIMS, _P, _P, _P, _P, _SZ, _P]),
     "basiskv_decode": (_I, [_DIMS, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I,
                             _P, _P, _P, _SZ, _P]),
+    "basiskv_decode_noalloc": (_I, [_DIMS, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
+                                    _I, _P, _P, _P]),
     "basiskv_read_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "basiskv_strerror": (ctypes.c_char_p, [_I]),
     "basiskv_launch_count": (ctypes.c_uint64, []),
@@ -170,6 +174,18 @@ def basiskv_decode(dims: Dims, q, k_new, v_new, seq_lens, max_seq_len: int, bloc
         _ptr(block_table), _ptr(A_V), _ptr(P_K), _ptr(U_K), _ptr(W_fold), _ptr(K_cache),
         _ptr(Z_cache), _ptr(E_cache), top_k, _ptr(sel), _ptr(y), _ptr(workspace),
         _nbytes(workspace), _stream(stream)), "basiskv_decode")
+
+
+def basiskv_decode_noalloc(dims: Dims, q, k_new, v_new, seq_lens, max_seq_len: int,
+                           block_table, A_V, P_K, U_K, W_fold, K_cache, Z_cache, E_cache,
+                           top_k: int, sel, y, stream=None) -> None:
+    """basiskv_decode without a workspace, for callers that cannot allocate:
+    the scratch is the library's static device array (see the header)."""
+    _check(load_library().basiskv_decode_noalloc(
+        ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(seq_lens), max_seq_len,
+        _ptr(block_table), _ptr(A_V), _ptr(P_K), _ptr(U_K), _ptr(W_fold), _ptr(K_cache),
+        _ptr(Z_cache), _ptr(E_cache), top_k, _ptr(sel), _ptr(y), _stream(stream)),
+        "basiskv_decode_noalloc")
 
 
 def read_device_status(stream=None) -> int:

@@ -542,6 +542,8 @@ const char* basiskv_strerror(int status) {
     case BASISKV_ERR_LAUNCH_FAILED: return "kernel launch failed";
     case BASISKV_ERR_DEVICE: return "device reported an error (see device status bits)";
     case BASISKV_ERR_CUDA: return "CUDA runtime call failed";
+    case BASISKV_ERR_SCRATCH_LIMIT:
+      return "problem needs more scratch than the static no-alloc buffer holds";
     default: return "unknown status";
   }
 }

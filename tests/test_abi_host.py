@@ -29,7 +29,7 @@ def lib():
 
 def test_header_symbols_are_exported(lib):
     names = bkv.header_symbols()
-    assert len(names) == 10
+    assert len(names) == 11
     out = subprocess.run(["nm", "-D", "--defined-only", bkv.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
@@ -39,7 +39,7 @@ def test_header_symbols_are_exported(lib):
 
 
 def test_strerror_every_status(lib):
-    for s in range(-6, 1):
+    for s in range(-7, 1):
         assert bkv.strerror(s) and "unknown" not in bkv.strerror(s)
     assert "unknown" in bkv.strerror(-99)
 
