@@ -195,14 +195,16 @@ bool cache_map(CUtensorMap* m, const void* base, const basiskv_dims* d, int widt
                       swizzle_for_cols(box_cols));
 }
 
-int z_box_cols(int r_v) { return r_v % 32 == 0 ? 32 : 16; }
+// z boxes: full 128-byte rows when r_v allows (fewer, larger TMA requests).
+int z_box_cols(int r_v) { return r_v % 64 == 0 ? 64 : (r_v % 32 == 0 ? 32 : 16); }
 int e_box_cols(int r_k) { return r_k % 32 == 0 ? 32 : 16; }
 
 // ---------------------------------------------------------------- stages
 int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_bf16* v_new,
                int n_new, int32_t* seq_lens, const int32_t* block_table, const basiskv_bf16* A_V,
                const basiskv_bf16* P_K, const basiskv_bf16* U_K, basiskv_bf16* K_cache,
-               basiskv_bf16* Z_cache, basiskv_bf16* E_cache, cudaStream_t st, bool pdl) {
+               basiskv_bf16* Z_cache, basiskv_bf16* E_cache, cudaStream_t st, bool pdl,
+               bool bump = true) {
   AppendArgs a{};
   a.k_new = k_new;
   a.v_new = v_new;
@@ -227,7 +229,7 @@ int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_b
   a.status = device_status_ptr();
   if (!a.status) return BASISKV_ERR_CUDA;
   int rc = launch_status(launch_append_small(a, st, pdl));
-  if (rc) return rc;
+  if (rc || !bump) return rc;
   return launch_status(launch_bump_lengths(a, st, pdl));
 }
 
@@ -235,7 +237,7 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
               int max_seq_len, const int32_t* block_table, const basiskv_bf16* P_K,
               const basiskv_bf16* U_K, const basiskv_bf16* Z_cache, const basiskv_bf16* E_cache,
               int top_k, float* scores, int32_t* sel, uint8_t* ws, const WsLayout& L,
-              cudaStream_t st, bool pdl) {
+              cudaStream_t st, bool pdl, int len_offset = 0) {
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   const int wz = z_box_cols(d->r_v), we = e_box_cols(d->r_k);
@@ -260,18 +262,20 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   r.max_pages = d->max_pages_per_seq;
   r.num_phys = d->num_phys_pages;
   r.max_seq_len = max_seq_len;
+  r.len_offset = len_offset;
   r.status = status;
   rc = launch_status(launch_route_scores(r, tmZ, tmE, wz, we, st, pdl));
   if (rc) return rc;
   SelectArgs s{scores, seq_lens, sel, d->B, d->Hkv, d->page_size, d->max_pages_per_seq, top_k,
-               max_seq_len};
+               max_seq_len, len_offset};
   return launch_status(launch_select(s, st, pdl));
 }
 
 int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_lens,
                const int32_t* block_table, const basiskv_bf16* K_cache,
                const basiskv_bf16* Z_cache, const int32_t* sel, int top_k, float* a_lat,
-               uint16_t* a_bf16, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl) {
+               uint16_t* a_bf16, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl,
+               int len_offset = 0) {
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   const int wz = z_box_cols(d->r_v);
@@ -296,17 +300,19 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
   a.top_k = top_k;
   a.nsplit = L.nsplit;
   a.pages_per_split = L.ppi;
+  a.len_offset = len_offset;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d->d));
   a.status = status;
   int rc = launch_status(launch_attend(a, tmK, tmZ, wz, st, pdl));
   if (rc) return rc;
   CombineArgs c{a.partial, seq_lens, a_lat, a_bf16, d->B, d->Hq, d->Hkv, a.G, d->r_v,
-                d->page_size, top_k, L.nsplit, L.ppi};
+                d->page_size, top_k, L.nsplit, L.ppi, len_offset};
   return launch_status(launch_combine(c, st, pdl));
 }
 
 int run_outproj(const basiskv_dims* d, const uint16_t* a_bf16, const basiskv_bf16* W_fold,
-                basiskv_bf16* y, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl) {
+                basiskv_bf16* y, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl,
+                int32_t* bump_lens = nullptr) {
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   const int K = d->Hq * d->r_v;
@@ -326,6 +332,9 @@ int run_outproj(const basiskv_dims* d, const uint16_t* a_bf16, const basiskv_bf1
   if (o.ksplit > kMaxKsplit) o.ksplit = kMaxKsplit;
   o.bn = bn;
   o.status = status;
+  o.bump_lens = bump_lens;
+  o.bump_n = 1;
+  o.bump_cap = d->max_pages_per_seq * d->page_size;
   return launch_status(launch_outproj(o, tmW, tmA, st, pdl));
 }
 
@@ -502,19 +511,23 @@ int basiskv_decode(const basiskv_dims* dims, const basiskv_bf16* q, const basisk
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool pdl = pdl_enabled();
   int32_t* sel_buf = sel ? sel : reinterpret_cast<int32_t*>(ws + L.sel);
+  // With an append, the new token is written first; the lengths are bumped
+  // only at the end of the step (by the out-projection launch), and the
+  // stages in between read seq_lens[b] + 1.
+  const int off = append ? 1 : 0;
   if (append) {
     rc = run_append(dims, k_new, v_new, 1, seq_lens, block_table, A_V, P_K, U_K, K_cache, Z_cache,
-                    E_cache, st, pdl);
+                    E_cache, st, pdl, /*bump=*/false);
     if (rc) return rc;
   }
   rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache, top_k,
-                 reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl);
+                 reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl, off);
   if (rc) return rc;
   uint16_t* a16 = reinterpret_cast<uint16_t*>(ws + L.a_bf16);
   rc = run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel_buf, top_k, nullptr, a16,
-                  ws, L, st, pdl);
+                  ws, L, st, pdl, off);
   if (rc) return rc;
-  return run_outproj(dims, a16, W_fold, y, ws, L, st, pdl);
+  return run_outproj(dims, a16, W_fold, y, ws, L, st, pdl, append ? seq_lens : nullptr);
 }
 
 int basiskv_read_device_status(void* stream, uint32_t* flags) {

@@ -4,9 +4,9 @@
 //   z = v A_V,g        e = (k - z P_K,g) U_K,g       K <- k
 //
 // One CTA per (KV head, token, sequence); each output element is one
-// thread's fp32 dot product over factor rows that stay resident in L2.  The
-// work is a few hundred thousand FMAs per decode step, so the kernel is
-// bounded by launch latency, not by any pipe.
+// thread's fp32 dot product over the head's factors, staged in shared memory.
+// The work is a few hundred thousand FMAs per decode step, so the kernel is
+// bounded by latency (factor staging from L2, launch), not by any pipe.
 #include "common.cuh"
 #include "internal.h"
 #include "launch.cuh"
@@ -17,11 +17,32 @@ namespace {
 
 constexpr int kAppendThreads = 128;  // >= max(d, r_v, r_k) of every supported shape
 
+// Copies n bf16 values (n % 8 == 0, both pointers 16-byte aligned) with
+// independent 16-byte loads spread over the block.
+__device__ __forceinline__ void stage_bf16(uint16_t* dst, const uint16_t* src, int n) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  for (int i = threadIdx.x; i < n / 8; i += blockDim.x) d4[i] = s4[i];
+}
+
+// One CTA per (KV head, token, sequence).  The head's three factors (at most
+// 128x128 + 128x128 + 128x64 bf16 = 80 KB) are first staged in shared memory
+// with independent 16-byte loads, so the dot products below read shared
+// memory instead of waiting on one global load per step.
 __global__ void __launch_bounds__(kAppendThreads) append_small_kernel(AppendArgs a) {
-  pdl_wait();
-  const int g = blockIdx.x, j = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  extern __shared__ __align__(16) uint16_t fac[];  // A_V | P_K | U_K of head g
   __shared__ float vs[kAppendThreads], ks[kAppendThreads], zs[kAppendThreads],
       rs[kAppendThreads];
+  const int g = blockIdx.x, j = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+  const int d = a.d, r_v = a.r_v, r_k = a.r_k;
+  uint16_t* A = fac;
+  uint16_t* Pk = fac + d * r_v;
+  uint16_t* U = Pk + r_v * d;
+  // Factors are inputs no predecessor writes: stage them before the wait.
+  stage_bf16(A, a.A_V + (size_t)g * d * r_v, d * r_v);
+  stage_bf16(Pk, a.P_K + (size_t)g * r_v * d, r_v * d);
+  stage_bf16(U, a.U_K + (size_t)g * d * r_k, d * r_k);
+  pdl_wait();
   const int len = a.seq_lens[b];
   const int cap = a.max_pages * a.S;
   if (len < 0 || len + a.n_new > cap) {
@@ -35,34 +56,34 @@ __global__ void __launch_bounds__(kAppendThreads) append_small_kernel(AppendArgs
     return;
   }
   const size_t slot = ((size_t)pp * a.Hkv + g) * a.S + pos % a.S;
-  const size_t tok = (((size_t)b * a.n_new + j) * a.Hkv + g) * a.d;
-  if (tid < a.d) {
+  const size_t tok = (((size_t)b * a.n_new + j) * a.Hkv + g) * d;
+  if (tid < d) {
     const uint16_t kb = a.k_new[tok + tid];
     ks[tid] = bf16_to_f(kb);
     vs[tid] = bf16_to_f(a.v_new[tok + tid]);
-    a.K_cache[slot * a.d + tid] = kb;
+    a.K_cache[slot * d + tid] = kb;
   }
   __syncthreads();
-  if (tid < a.r_v) {  // z_j = sum_i v_i A_V[i][j]
-    const uint16_t* A = a.A_V + (size_t)g * a.d * a.r_v + tid;
+  if (tid < r_v) {  // z_j = sum_i v_i A_V[i][j]
     float acc = 0.f;
-    for (int i = 0; i < a.d; ++i) acc = fmaf(vs[i], bf16_to_f(A[(size_t)i * a.r_v]), acc);
+#pragma unroll 8
+    for (int i = 0; i < d; ++i) acc = fmaf(vs[i], bf16_to_f(A[i * r_v + tid]), acc);
     zs[tid] = acc;
-    a.Z_cache[slot * a.r_v + tid] = f_to_bf16(acc);
+    a.Z_cache[slot * r_v + tid] = f_to_bf16(acc);
   }
   __syncthreads();
-  if (tid < a.d) {  // residual_i = k_i - sum_j z_j P_K[j][i]   (z unrounded)
-    const uint16_t* P = a.P_K + (size_t)g * a.r_v * a.d + tid;
+  if (tid < d) {  // residual_i = k_i - sum_j z_j P_K[j][i]   (z unrounded)
     float acc = ks[tid];
-    for (int jj = 0; jj < a.r_v; ++jj) acc = fmaf(-zs[jj], bf16_to_f(P[(size_t)jj * a.d]), acc);
+#pragma unroll 8
+    for (int jj = 0; jj < r_v; ++jj) acc = fmaf(-zs[jj], bf16_to_f(Pk[jj * d + tid]), acc);
     rs[tid] = acc;
   }
   __syncthreads();
-  if (tid < a.r_k) {  // e_c = sum_i residual_i U_K[i][c]
-    const uint16_t* U = a.U_K + (size_t)g * a.d * a.r_k + tid;
+  if (tid < r_k) {  // e_c = sum_i residual_i U_K[i][c]
     float acc = 0.f;
-    for (int i = 0; i < a.d; ++i) acc = fmaf(rs[i], bf16_to_f(U[(size_t)i * a.r_k]), acc);
-    a.E_cache[slot * a.r_k + tid] = f_to_bf16(acc);
+#pragma unroll 8
+    for (int i = 0; i < d; ++i) acc = fmaf(rs[i], bf16_to_f(U[i * r_k + tid]), acc);
+    a.E_cache[slot * r_k + tid] = f_to_bf16(acc);
   }
 }
 
@@ -85,7 +106,13 @@ __global__ void bump_lengths_kernel(const int32_t* seq_lens, int32_t* out, int B
 
 cudaError_t launch_append_small(const AppendArgs& a, cudaStream_t st, bool pdl) {
   dim3 grid(a.Hkv, a.n_new, a.B);
-  return launch_k(append_small_kernel, grid, dim3(kAppendThreads), 0, st, pdl, a);
+  const size_t smem = (size_t)(2 * a.d * a.r_v + a.d * a.r_k) * sizeof(uint16_t);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(append_small_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_k(append_small_kernel, grid, dim3(kAppendThreads), smem, st, pdl, a);
 }
 
 cudaError_t launch_bump_lengths(const AppendArgs& a, cudaStream_t st, bool pdl) {

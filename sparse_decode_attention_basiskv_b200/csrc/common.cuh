@@ -31,6 +31,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Rounds a dynamic shared-memory base up to 1024 bytes (the repeat of the
+// 128-byte TMA swizzle).  Pointer arithmetic on the __shared__ array itself
+// keeps the compiler aware that loads through the result are shared-memory
+// loads; a round trip through an integer would turn them into generic loads.
+__device__ __forceinline__ uint8_t* align_smem_1k(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)

@@ -58,6 +58,7 @@ struct RouteArgs {
   const int32_t* block_table;
   float* scores;  // [B][Hkv][max_pages]
   int B, Hkv, G, r_v, r_k, S, max_pages, num_phys, max_seq_len;
+  int len_offset;  // added to seq_lens[b] (tokens appended in this step, not yet counted)
   unsigned int* status;
 };
 cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
@@ -69,6 +70,7 @@ struct SelectArgs {
   const int32_t* seq_lens;
   int32_t* sel;  // [B][Hkv][top_k]
   int B, Hkv, S, max_pages, top_k, max_seq_len;
+  int len_offset;
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
 
@@ -80,6 +82,7 @@ struct AttendArgs {
   const int32_t* sel;
   float* partial;  // [B*Hkv][nsplit][G][r_v + 2]
   int B, Hq, Hkv, G, d, r_v, S, max_pages, num_phys, top_k, nsplit, pages_per_split;
+  int len_offset;
   float scale_log2;  // log2(e) / sqrt(d)
   unsigned int* status;
 };
@@ -93,6 +96,7 @@ struct CombineArgs {
   float* a_lat;        // [B][Hq][r_v] fp32 (may be null)
   uint16_t* a_bf16;    // [B][Hq][r_v] bf16 (may be null)
   int B, Hq, Hkv, G, r_v, S, top_k, nsplit, pages_per_split;
+  int len_offset;  // added to seq_lens[b] (tokens appended in this step, not yet counted)
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st, bool pdl);
 
@@ -102,6 +106,11 @@ struct OutprojArgs {
   uint16_t* y;     // [B][H] bf16
   int B, H, K, ksplit, bn;
   unsigned int* status;
+  // Deferred length update of a fused decode step: when bump_lens is set,
+  // seq_lens[b] += bump_n (unless that passes bump_cap), done once every
+  // earlier kernel of the step has finished reading the lengths.
+  int32_t* bump_lens;
+  int bump_n, bump_cap;
 };
 // Chooses the K split for a given problem.
 int outproj_ksplit(int H, int K, int B);

@@ -92,8 +92,7 @@ __global__ void __launch_bounds__(kOpThreads, 1)
   constexpr int kOpStages = op_stages<BN>();
   constexpr int kTmemCols = BN <= 32 ? 32 : (BN <= 64 ? 64 : (BN <= 128 ? 128 : 256));
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   uint8_t* a_tiles = smem;                              // kOpStages x 16 KB
   uint8_t* b_tiles = smem + kOpStages * kOpATile;       // kOpStages x kBTile
   uint64_t* full = reinterpret_cast<uint64_t*>(b_tiles + kOpStages * kBTile);
@@ -131,6 +130,12 @@ __global__ void __launch_bounds__(kOpThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_wait();
+  if (a.bump_lens && blockIdx.x == 0 && blockIdx.y == 0) {
+    for (int b = tid; b < a.B; b += kOpThreads) {
+      const int len = a.bump_lens[b];
+      if (len >= 0 && len + a.bump_n <= a.bump_cap) a.bump_lens[b] = len + a.bump_n;
+    }
+  }
 
   if (warp == 0) {
     if (lane == 0) {  // ---------------------------------------- TMA producer

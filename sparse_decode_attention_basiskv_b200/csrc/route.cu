@@ -28,40 +28,62 @@ namespace {
 // ----------------------------------------------------------- query folding
 // qt[b][h][j]       = sum_i P_K[g][j][i] q[b][h][i]          j < r_v
 // qt[b][h][r_v + c] = sum_i q[b][h][i] U_K[g][i][c]           c < r_k
-constexpr int kFoldThreads = 128;
+constexpr int kFoldThreads = 128;  // 32 outputs x 4 quarters of the head dim
 
+// CTA = (sequence, KV head, 32 consecutive outputs j).  Warp w sums the
+// products over the w-th quarter of the head dimension for every head of
+// the group; the four partial sums meet in shared memory.  All loads of a
+// thread are independent, so the kernel costs about one memory round trip.
 __global__ void __launch_bounds__(kFoldThreads) fold_query_kernel(FoldQArgs a) {
-  const int bg = blockIdx.x, b = bg / a.Hkv, g = bg % a.Hkv, tid = threadIdx.x;
-  const int G = a.Hq / a.Hkv, rq = a.r_v + a.r_k;
-  extern __shared__ float qs[];  // [G][d]
+  const int bg = blockIdx.x, b = bg / a.Hkv, g = bg % a.Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, quarter = tid >> 5;
+  const int G = a.Hq / a.Hkv, rq = a.r_v + a.r_k, d = a.d;
+  const int j = blockIdx.y * 32 + lane;
+  const int i0 = quarter * (d / 4), n = d / 4;
+  extern __shared__ float fsm[];
+  float* qs = fsm;               // [G][d]
+  float* part = fsm + G * d;     // [4][G][32]
   pdl_wait();
-  for (int i = tid; i < G * a.d; i += blockDim.x)
-    qs[i] = bf16_to_f(a.q[((size_t)b * a.Hq + g * G) * a.d + i]);
+  for (int i = tid; i < G * d; i += kFoldThreads)
+    qs[i] = bf16_to_f(a.q[((size_t)b * a.Hq + g * G) * d + i]);
   __syncthreads();
-  for (int j = tid; j < rq; j += blockDim.x) {
-    float acc[8];
+  float acc[8];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) acc[h] = 0.f;
-    if (j < a.r_v) {
-      const uint16_t* P = a.P_K + ((size_t)g * a.r_v + j) * a.d;
-      for (int i = 0; i < a.d; ++i) {
-        const float p = bf16_to_f(P[i]);
+  for (int h = 0; h < 8; ++h) acc[h] = 0.f;
+  if (j < a.r_v) {  // row j of P_K, this quarter: n contiguous bf16 (16-byte aligned)
+    const uint4* row = reinterpret_cast<const uint4*>(a.P_K + ((size_t)g * a.r_v + j) * d + i0);
+    for (int c = 0; c < n / 8; ++c) {
+      const uint4 w = row[c];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int h = 0; h < 8; ++h)
-          if (h < G) acc[h] = fmaf(p, qs[h * a.d + i], acc[h]);
-      }
-    } else {
-      const uint16_t* U = a.U_K + (size_t)g * a.d * a.r_k + (j - a.r_v);
-      for (int i = 0; i < a.d; ++i) {
-        const float u = bf16_to_f(U[(size_t)i * a.r_k]);
+      for (int e = 0; e < 4; ++e) {
+        const float p0 = bf16lo(ws[e]), p1 = bf16hi(ws[e]);
+        const int ii = i0 + c * 8 + 2 * e;
 #pragma unroll
         for (int h = 0; h < 8; ++h)
-          if (h < G) acc[h] = fmaf(u, qs[h * a.d + i], acc[h]);
+          if (h < G) acc[h] = fmaf(p1, qs[h * d + ii + 1], fmaf(p0, qs[h * d + ii], acc[h]));
       }
     }
+  } else if (j < rq) {  // column j - r_v of U_K, this quarter (coalesced across lanes)
+    const uint16_t* col = a.U_K + (size_t)g * d * a.r_k + (j - a.r_v);
+    for (int i = i0; i < i0 + n; ++i) {
+      const float u = bf16_to_f(col[(size_t)i * a.r_k]);
 #pragma unroll
-    for (int h = 0; h < 8; ++h)
-      if (h < G) a.qt[((size_t)b * a.Hq + g * G + h) * rq + j] = acc[h];
+      for (int h = 0; h < 8; ++h)
+        if (h < G) acc[h] = fmaf(u, qs[h * d + i], acc[h]);
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 8; ++h)
+    if (h < G) part[(quarter * G + h) * 32 + lane] = acc[h];
+  __syncthreads();
+  for (int o = tid; o < G * 32; o += kFoldThreads) {
+    const int h = o / 32, jj = blockIdx.y * 32 + (o % 32);
+    if (jj < rq) {
+      const float v = part[(0 * G + h) * 32 + o % 32] + part[(1 * G + h) * 32 + o % 32] +
+                      part[(2 * G + h) * 32 + o % 32] + part[(3 * G + h) * 32 + o % 32];
+      a.qt[((size_t)b * a.Hq + g * G + h) * rq + jj] = v;
+    }
   }
 }
 
@@ -100,6 +122,41 @@ __device__ __forceinline__ int clamp_len(int T, int max_seq_len, unsigned int* s
   return T;
 }
 
+// Walks a contiguous range of (sequence, KV head, page-tile) work without a
+// division per tile: one division at the start, then increments.  The
+// length of the current sequence is cached and reloaded only when the
+// sequence changes.
+struct TileCursor {
+  int bg, b, g, ti;  // flat (sequence, KV head), sequence, KV head, tile in it
+  int T, P;          // length (clamped) and pages of sequence b
+  __device__ void init(long tile, int tiles_per_bg, int Hkv) {
+    bg = (int)(tile / tiles_per_bg);
+    ti = (int)(tile - (long)bg * tiles_per_bg);
+    b = bg / Hkv;
+    g = bg - b * Hkv;
+    T = -1;
+  }
+  __device__ void next(int tiles_per_bg, int Hkv) {
+    if (++ti == tiles_per_bg) {
+      ti = 0;
+      ++bg;
+      if (++g == Hkv) {
+        g = 0;
+        ++b;
+        T = -1;
+      }
+    }
+  }
+  // Loads the length when the sequence changed since the last call.
+  __device__ void length(const int32_t* seq_lens, int len_offset, int max_seq_len, int S,
+                         unsigned int* status, bool report) {
+    if (T < 0) {
+      T = clamp_len(seq_lens[b] + len_offset, max_seq_len, status, report);
+      P = (T + S - 1) / S;
+    }
+  }
+};
+
 // Adds the contribution of one 8-wide chunk of a token row to the G head
 // accumulators.  `xa` is the swizzled shared address of the row chunk, `qa`
 // the address of the chunk in head 0's folded query; heads are rq floats
@@ -130,8 +187,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
     route_kernel(const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmE,
                  RouteArgs a, RouteGeom geo) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)geo.stages * geo.stage_bytes);
   uint64_t* empty = full + geo.stages;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -163,7 +219,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
       for (long tile = t_begin; tile < t_end; ++tile) {
         int bg, b, g, ti;
         decode_tile(tile, tiles_per_bg, a.Hkv, bg, b, g, ti);
-        const int T = clamp_len(a.seq_lens[b], a.max_seq_len, a.status, false);
+        const int T = clamp_len(a.seq_lens[b] + a.len_offset, a.max_seq_len, a.status, false);
         const int P = (T + S - 1) / S, p0 = ti * geo.np;
         if (p0 >= P) continue;
         const int npg = min(geo.np, P - p0);
@@ -203,7 +259,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
   for (long tile = t_begin; tile < t_end; ++tile) {
     int bg, b, g, ti;
     decode_tile(tile, tiles_per_bg, a.Hkv, bg, b, g, ti);
-    const int T = clamp_len(a.seq_lens[b], a.max_seq_len, a.status, tid == 0 && ti == 0);
+    const int T = clamp_len(a.seq_lens[b] + a.len_offset, a.max_seq_len, a.status, tid == 0 && ti == 0);
     const int P = (T + S - 1) / S, p0 = ti * geo.np;
     if (p0 >= P) continue;
     const int npg = min(geo.np, P - p0);
@@ -248,13 +304,22 @@ __global__ void __launch_bounds__(kRouteThreads, 1)
 // time.  Each consumer thread copies its token's whole row (r_v + r_k bf16)
 // from the stage into registers and releases the stage at once, so shared
 // memory holds data in flight rather than data being computed on; the folded
-// queries live in a per-group buffer that is refreshed when the (sequence,
-// KV head) changes.  Two groups of seven consumer warps take alternate
-// stages, and the G dot products use packed fp32x2 FMAs.
-constexpr int kRsGroupThreads = 224;  // tokens per stage (7 warps: 16 warps per CTA in all)
-constexpr int kRsGroups = 2;
+// queries live in a per-CTA buffer that is refreshed when the (sequence, KV
+// head) changes.  The G dot products use packed fp32x2 FMAs.
+//
+// Pipeline shape (measured on B200 at the 32K-context, B = 16 workload): one
+// producer/consumer ring per CTA caps at about 29 GB/s per SM however deep
+// it is, so the kernel runs three small independent rings per SM (3 CTAs of
+// 4 consumer warps, 128 tokens per stage) rather than one large one; z
+// boxes are 64 columns (full 128-byte rows) whenever r_v allows.
+constexpr int kRsGroupThreads = 128;  // tokens per stage (4 consumer warps)
+constexpr int kRsGroups = 1;
+constexpr int kRsCtasPerSm = 3;
 constexpr int kRsThreads = kRsGroups * kRsGroupThreads + 32;
 constexpr int kRsProducerWarp = kRsGroups * kRsGroupThreads / 32;
+
+// Box width of the z tensor map the specialised kernel expects.
+__host__ __device__ constexpr int rs_z_box_cols(int r_v) { return r_v % 64 == 0 ? 64 : 32; }
 
 struct RsGeom {
   int np;           // pages per stage
@@ -266,16 +331,15 @@ struct RsGeom {
 };
 
 template <int G, int RV, int RK>
-__global__ void __launch_bounds__(kRsThreads, 1)
+__global__ void __launch_bounds__(kRsThreads, kRsCtasPerSm)
     route_rs_kernel(const __grid_constant__ CUtensorMap tmZ,
                     const __grid_constant__ CUtensorMap tmE, RouteArgs a, RsGeom geo) {
-  constexpr int WZ = 32, WE = (RK % 32 == 0) ? 32 : 16;
+  constexpr int WZ = rs_z_box_cols(RV), WE = (RK % 32 == 0) ? 32 : 16;
   constexpr int NZB = RV / WZ, NEB = RK / WE;
   constexpr int NZC = RV / 8, NEC = RK / 8, NCH = NZC + NEC, RQ = RV + RK;
-  constexpr uint32_t ZM = 3u, EM = (WE == 32) ? 3u : 1u;
+  constexpr uint32_t ZM = (WZ == 64) ? 7u : 3u, EM = (WE == 32) ? 3u : 1u;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + geo.bar_off);
   uint64_t* empty = full + geo.stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + geo.stages);
@@ -306,22 +370,41 @@ __global__ void __launch_bounds__(kRsThreads, 1)
   if (warp == kRsProducerWarp) {
     // ------------------------------------------------------------ producer
     // The whole warp: lane j fetches page j's block-table entry and issues
-    // that page's boxes, so a tile's gathers go out in parallel.
-    int it = 0, cur_b = -1, T = 0;
-    for (long tile = t_begin; tile < t_end; ++tile) {
-      int bg, b, g, ti;
-      decode_tile(tile, tiles_per_bg, a.Hkv, bg, b, g, ti);
-      if (b != cur_b) {
-        T = clamp_len(a.seq_lens[b], a.max_seq_len, a.status, false);
-        cur_b = b;
+    // that page's boxes, so a tile's gathers go out in parallel.  Entries are
+    // fetched kBtAhead tiles ahead into a per-lane register ring: the table is
+    // evicted from L2 by the cache stream, and one dependent round trip per
+    // tile would otherwise pace the whole pipeline.
+    constexpr int kBtAhead = 8;
+    const int count = (int)(t_end - t_begin);
+    TileCursor pre, cur;
+    pre.init(t_begin, tiles_per_bg, a.Hkv);
+    cur = pre;
+    auto fetch = [&](int n) -> int {  // entry of tile t_begin + n, then advance
+      int v = 0;
+      if (n < count) {
+        pre.length(a.seq_lens, a.len_offset, a.max_seq_len, S, a.status, false);
+        const int p0_ = pre.ti * geo.np;
+        if (lane < min(geo.np, pre.P - p0_))
+          v = a.block_table[(size_t)pre.b * a.max_pages + p0_ + lane];
+        pre.next(tiles_per_bg, a.Hkv);
       }
-      const int P = (T + S - 1) / S, p0 = ti * geo.np;
+      return v;
+    };
+    int ring[kBtAhead];
+#pragma unroll
+    for (int k = 0; k < kBtAhead; ++k) ring[k] = fetch(k);
+    int it = 0;
+    for (int n = 0; n < count; ++n, cur.next(tiles_per_bg, a.Hkv)) {
+      int pp = ring[0];
+#pragma unroll
+      for (int k = 0; k + 1 < kBtAhead; ++k) ring[k] = ring[k + 1];
+      ring[kBtAhead - 1] = fetch(n + kBtAhead);
+      cur.length(a.seq_lens, a.len_offset, a.max_seq_len, S, a.status, false);
+      const int b = cur.b, g = cur.g, P = cur.P, p0 = cur.ti * geo.np;
       if (p0 >= P) continue;
       const int npg = min(geo.np, P - p0);
       const int s = it % geo.stages;
       ++it;
-      int pp = 0;
-      if (lane < npg) pp = a.block_table[(size_t)b * a.max_pages + p0 + lane];
       bool go = true;
       if (lane == 0) {
         go = mbar_wait_or_abort(&empty[s], (((it - 1) / geo.stages) & 1) ^ 1, a.status,
@@ -351,16 +434,15 @@ __global__ void __launch_bounds__(kRsThreads, 1)
   const int group = tid / kRsGroupThreads, gtid = tid % kRsGroupThreads;
   const int page_local = gtid / S, row = gtid % S;
   float* qbuf = reinterpret_cast<float*>(smem + geo.q_off) + group * G * RQ;
-  int cur_bg = -1, cur_b = -1, T = 0;
+  int cur_bg = -1;
   int it = 0;
-  for (long tile = t_begin; tile < t_end; ++tile) {
-    int bg, b, g, ti;
-    decode_tile(tile, tiles_per_bg, a.Hkv, bg, b, g, ti);
-    if (b != cur_b) {
-      T = clamp_len(a.seq_lens[b], a.max_seq_len, a.status, tid == 0);
-      cur_b = b;
-    }
-    const int P = (T + S - 1) / S, p0 = ti * geo.np;
+  const int count = (int)(t_end - t_begin);
+  TileCursor cur;
+  cur.init(t_begin, tiles_per_bg, a.Hkv);
+  for (int n = 0; n < count; ++n, cur.next(tiles_per_bg, a.Hkv)) {
+    cur.length(a.seq_lens, a.len_offset, a.max_seq_len, S, a.status, tid == 0);
+    const int bg = cur.bg, b = cur.b, g = cur.g, T = cur.T, P = cur.P;
+    const int p0 = cur.ti * geo.np;
     if (p0 >= P) continue;
     const int my = it++;
     if ((my % kRsGroups) != group) continue;
@@ -381,7 +463,7 @@ __global__ void __launch_bounds__(kRsThreads, 1)
       const uint8_t* pg = smem + (size_t)s * geo.stage_bytes + page_local * geo.page_bytes;
 #pragma unroll
       for (int c = 0; c < NZC; ++c) {
-        const uint32_t off = (c / 4) * zbox + row * (WZ * 2) + (c % 4) * 16;
+        const uint32_t off = (c / (WZ / 8)) * zbox + row * (WZ * 2) + (c % (WZ / 8)) * 16;
         x[c] = *reinterpret_cast<const uint4*>(pg + swz(off, ZM));
       }
 #pragma unroll
@@ -470,7 +552,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   __shared__ int s_rem;
   pdl_wait();
   const int bg = blockIdx.x, b = bg / a.Hkv, tid = threadIdx.x;
-  int T = a.seq_lens[b];
+  int T = a.seq_lens[b] + a.len_offset;
   T = T < 0 ? 0 : (T > a.max_seq_len ? a.max_seq_len : T);
   const int P = (T + a.S - 1) / a.S;
   int32_t* out = a.sel + (size_t)bg * a.top_k;
@@ -604,10 +686,12 @@ cudaError_t launch_route_rs(const RouteArgs& a, const CUtensorMap& tmZ, const CU
   geo.page_bytes = (a.S * (RV + RK) * 2 + 1023) / 1024 * 1024;
   geo.stage_bytes = geo.np * geo.page_bytes;
   const int qbytes = kRsGroups * G * (RV + RK) * 4;
-  const int budget = 224 * 1024 - qbytes - 1024 - 256;
+  // 228 KB of shared memory per SM, 1 KB of it reserved per CTA; 1 KB of
+  // slack for the 1024-byte alignment of the base.
+  const int budget = 228 * 1024 / kRsCtasPerSm - 1024 - 1024 - qbytes - 256;
   geo.stages = budget / geo.stage_bytes;
   if (geo.stages > 8) geo.stages = 8;
-  if (geo.stages < kRsGroups + 1) return cudaErrorInvalidConfiguration;
+  if (geo.stages < 2) return cudaErrorInvalidConfiguration;
   geo.q_off = geo.stages * geo.stage_bytes;
   geo.bar_off = geo.q_off + qbytes;
   const size_t smem = (size_t)geo.bar_off + 2 * geo.stages * 8 + 16 + 1024;
@@ -616,7 +700,7 @@ cudaError_t launch_route_rs(const RouteArgs& a, const CUtensorMap& tmZ, const CU
   if (e != cudaSuccess) return e;
   const int P_max = (a.max_seq_len + a.S - 1) / a.S;
   const long tiles = (long)a.B * a.Hkv * ((P_max + geo.np - 1) / geo.np);
-  long grid = num_sms();
+  long grid = (long)num_sms() * kRsCtasPerSm;
   if (grid > tiles) grid = tiles;
   if (grid < 1) grid = 1;
   return launch_k(route_rs_kernel<G, RV, RK>, dim3((unsigned)grid), dim3(kRsThreads), smem, st,
@@ -627,14 +711,15 @@ cudaError_t launch_route_rs(const RouteArgs& a, const CUtensorMap& tmZ, const CU
 
 cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl) {
   const int G = a.Hq / a.Hkv;
-  return launch_k(fold_query_kernel, dim3(a.B * a.Hkv), dim3(kFoldThreads),
-                  (size_t)G * a.d * sizeof(float), st, pdl, a);
+  const size_t smem = (size_t)(G * a.d + 4 * G * 32) * sizeof(float);
+  dim3 grid(a.B * a.Hkv, (a.r_v + a.r_k + 31) / 32);
+  return launch_k(fold_query_kernel, grid, dim3(kFoldThreads), smem, st, pdl, a);
 }
 
 cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
                                 const CUtensorMap& tmE, int wz, int we, cudaStream_t st,
                                 bool pdl) {
-  if (wz == 32 && we == (a.r_k % 32 == 0 ? 32 : 16)) {
+  if (wz == rs_z_box_cols(a.r_v) && we == (a.r_k % 32 == 0 ? 32 : 16)) {
 #define BKV_RS(GG, V, K) \
   if (a.G == GG && a.r_v == V && a.r_k == K) return launch_route_rs<GG, V, K>(a, tmZ, tmE, st, pdl);
     BKV_RS(4, 32, 16)
