@@ -47,8 +47,7 @@ struct AttendGeom {
   int k_off, z_off, q_off, meta_off;  // regions inside a stage
   int stage_bytes;
   int stages;
-  int qs_off, ps_off, red_off, acc_off;  // single-buffered scratch after the ring
-  int qs_stride;                          // floats per head in qs (d + 8)
+  int ps_off, red_off;  // scratch after the ring, double-buffered by item parity
   int smem_bytes;
 };
 
@@ -74,7 +73,7 @@ struct ItemCursor {
   }
 };
 
-template <int G>
+template <int G, int D>
 __global__ void __launch_bounds__(kAttThreads, kAttCtasPerSm)
     attend_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmZ,
                   AttendArgs a, AttendGeom geo) {
@@ -83,10 +82,8 @@ __global__ void __launch_bounds__(kAttThreads, kAttCtasPerSm)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + geo.smem_bytes);
   uint64_t* empty = full + geo.stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + geo.stages);
-  float* qs = reinterpret_cast<float*>(smem + geo.qs_off);     // [G][d + 8], pre-scaled
-  float* ps = reinterpret_cast<float*>(smem + geo.ps_off);     // [128][G]
-  float* red = reinterpret_cast<float*>(smem + geo.red_off);   // [2][warps][G]
-  float* accs = reinterpret_cast<float*>(smem + geo.acc_off);  // [groups][G*r_v]
+  float* psb = reinterpret_cast<float*>(smem + geo.ps_off);    // [2][G][64] weights
+  float* redb = reinterpret_cast<float*>(smem + geo.red_off);  // [2][2][warps][G]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < geo.stages; ++s) {
@@ -103,7 +100,9 @@ __global__ void __launch_bounds__(kAttThreads, kAttCtasPerSm)
   __syncthreads();
   pdl_wait();
 
-  const int S = a.S, d = a.d, r_v = a.r_v;
+  constexpr int d = D;
+  const int S = a.S, r_v = a.r_v;
+  const int logS = 31 - __clz(S);  // S is a power of two
   const long total = (long)a.B * a.Hkv * a.nsplit;
   const long i_begin = total * blockIdx.x / gridDim.x;
   const long i_end = total * (blockIdx.x + 1) / gridDim.x;
@@ -189,14 +188,17 @@ __global__ void __launch_bounds__(kAttThreads, kAttCtasPerSm)
   }
 
   // --------------------------------------------------------------- consumers
-  const int tok = tid >> 1, half = tid & 1;
-  const int page_local = tok / S, row = tok % S;
+  // Warp w owns item tokens [16w, 16w + 16) for QK and latent tiles w, w+4,
+  // ... (16 latent dims each) for PV, both as warp-level tensor-core MMAs
+  // (mma.m16n8k16, bf16 operands, fp32 accumulation; heads are the N = 8
+  // columns).  Fragment layout: lane l holds accumulator rows l/4 and
+  // l/4 + 8, columns 2(l%4) and 2(l%4)+1.  QK multiplies the exact bf16
+  // products; PV splits each softmax weight into bf16 hi + lo parts (two
+  // MMAs), which keeps ~16 mantissa bits of the weights.
+  const int lq = lane >> 2, lr = lane & 3;
+  const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix index, row in it
   const int zc_per_box = geo.wz / 8;
-  const int nslot = G * r_v / 8;  // (head, 8-wide latent chunk) slots
-  const int ngrp = kAttConsumers / nslot > 0 ? kAttConsumers / nslot : 1;
-  const int nact = nslot < kAttConsumers ? nslot * ngrp : kAttConsumers;
-  const int QS = geo.qs_stride;
-  const int nch = d / 16;  // 16-byte chunks per half of a K row
+  const uint32_t zmask = geo.zmask;
   int it = 0;
   const int count = (int)(i_end - i_begin);
   ItemCursor cur;
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kAttThreads, kAttCtasPerSm)
     const int my = it++;
     // On a timeout every later wait fails at once; the item is skipped but
     // the barrier sequence below is kept, so all consumer warps stay in step.
-    bool ready = mbar_wait_or_abort(&full[s], (my / geo.stages) & 1, a.status, abort_flag);
+    const bool ready = mbar_wait_or_abort(&full[s], (my / geo.stages) & 1, a.status, abort_flag);
     const uint8_t* st = smem + (size_t)s * geo.stage_bytes;
     const int* meta = reinterpret_cast<const int*>(st + geo.meta_off);
     if (ready && meta[0] < 0) {  // empty split: nothing to attend, nothing to write
@@ -215,127 +217,151 @@ __global__ void __launch_bounds__(kAttThreads, kAttCtasPerSm)
       if (lane == 0) mbar_arrive(&empty[s]);
       continue;
     }
-
-    // Queries of the group, fp32 and scaled so that exp2 gives the softmax;
-    // the second half of each head is shifted by 4 floats (bank spread).
-    if (ready) {
-      const uint16_t* qb = reinterpret_cast<const uint16_t*>(st + geo.q_off);
-      for (int i = tid; i < G * d; i += kAttConsumers) {
-        const int h = i / d, c = i % d;
-        qs[h * QS + c + (c >= d / 2 ? 4 : 0)] = bf16_to_f(qb[i]) * a.scale_log2;
-      }
-    }
-    named_bar_sync(1, kAttConsumers);
-
+    float* red = redb + (my & 1) * 2 * kAttConsumerWarps * G;  // scratch by item parity
+    float* ps = psb + (my & 1) * G * kAttTokens;
     const int T = ready ? meta[31] : 0;
-    const int lp = (ready && page_local < geo.ppi) ? meta[page_local] : -1;
-    const bool valid = lp >= 0 && lp * S + row < T;
-    float sc[G];
+    auto tok_ok = [&](int t) -> bool {
+      const int lp = ready ? meta[t >> logS] : -1;
+      return lp >= 0 && (lp << logS) + (t & (S - 1)) < T;
+    };
+
+    // ---- QK: scores of the warp's 16 tokens for all heads
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    if (ready) {
+      const uint16_t* qb = reinterpret_cast<const uint16_t*>(st + geo.q_off);  // [G][D] bf16
+      const int t_ld = warp * 16 + (mi & 1) * 8 + mr;
+      const uint8_t* krow = st + geo.k_off + (t_ld >> logS) * geo.nkb * geo.kbox;
+      const int r_ld = t_ld & (S - 1);
 #pragma unroll
-    for (int h = 0; h < G; ++h) sc[h] = 0.f;
-    if (valid) {
-      float2 acc[G][2];
-#pragma unroll
-      for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = make_float2(0.f, 0.f);
-      const uint8_t* kb0 = st + geo.k_off + page_local * geo.nkb * geo.kbox;
-      for (int i = 0; i < nch; ++i) {
-        // half 1 walks its chunks in a rotated order so that the two halves of
-        // neighbouring tokens hit different banks
-        const int c = half ? nch + ((i + nch / 2) % nch) : i;
-        const uint32_t off = (c >> 3) * geo.kbox + swz(row * 128 + (c & 7) * 16, 7u);
-        const uint4 w = *reinterpret_cast<const uint4*>(kb0 + off);
-        const float2 x0 = bf16x2_to_f2(w.x), x1 = bf16x2_to_f2(w.y);
-        const float2 x2 = bf16x2_to_f2(w.z), x3 = bf16x2_to_f2(w.w);
-        const int qo = c * 8 + (half ? 4 : 0);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float4 q0 = *reinterpret_cast<const float4*>(qs + h * QS + qo);
-          const float4 q1 = *reinterpret_cast<const float4*>(qs + h * QS + qo + 4);
-          ffma2(acc[h][0], x0, make_float2(q0.x, q0.y));
-          ffma2(acc[h][1], x1, make_float2(q0.z, q0.w));
-          ffma2(acc[h][0], x2, make_float2(q1.x, q1.y));
-          ffma2(acc[h][1], x3, make_float2(q1.z, q1.w));
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const int cc = 2 * ks + (mi >> 1);  // 16-byte chunk of the K row
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(smem_u32(krow + (cc >> 3) * geo.kbox + swz(r_ld * 128 + (cc & 7) * 16, 7u)),
+                    a0, a1, a2, a3);
+        uint32_t b0 = 0u, b1 = 0u;
+        if (lq < G) {
+          b0 = *reinterpret_cast<const uint32_t*>(qb + lq * D + ks * 16 + 2 * lr);
+          b1 = *reinterpret_cast<const uint32_t*>(qb + lq * D + ks * 16 + 8 + 2 * lr);
         }
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-        sc[h] = (acc[h][0].x + acc[h][1].x) + (acc[h][0].y + acc[h][1].y);
-    }
-    // The two halves of a token sum their partial dot products.
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 1);
-      if (!valid) sc[h] = -INFINITY;
-    }
-    // Item maximum per head.
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float m = warp_max(sc[h]);
-      if (lane == 0) red[warp * G + h] = m;
-    }
-    named_bar_sync(1, kAttConsumers);
-    float mh[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float m = red[h];
-      for (int w = 1; w < kAttConsumerWarps; ++w) m = fmaxf(m, red[w * G + h]);
-      mh[h] = m;
-    }
-    // Weights and their sum per head (one thread of each token pair counts).
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float p = valid ? exp2f(sc[h] - mh[h]) : 0.f;
-      if (half == 0) ps[tok * G + h] = p;
-      const float l = warp_sum(half == 0 ? p : 0.f);
-      if (lane == 0) red[(kAttConsumerWarps + warp) * G + h] = l;
-    }
-    named_bar_sync(1, kAttConsumers);
-    // Latent accumulation: thread = (head, 8-wide chunk) slot x token group.
-    if (ready && tid < nact) {
-      const int slot = tid % nslot, grp = tid / nslot;
-      const int h = slot / (r_v / 8), c = slot % (r_v / 8);
-      const int box = c / zc_per_box, cc = c - box * zc_per_box;
-      float2 acc[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
-      const uint8_t* zb0 = st + geo.z_off + box * geo.zbox;
-      for (int t = grp; t < kAttTokens; t += ngrp) {
-        const float p = ps[t * G + h];
-        if (p > 0.f) {  // skips tokens never loaded (their slots hold stale data)
-          const int pl = t / S, rw = t % S;
-          const uint4 w = *reinterpret_cast<const uint4*>(
-              zb0 + pl * geo.nzb * geo.zbox + swz(rw * geo.wz * 2 + cc * 16, geo.zmask));
-          const float2 pp = make_float2(p, p);
-          ffma2(acc[0], pp, bf16x2_to_f2(w.x));
-          ffma2(acc[1], pp, bf16x2_to_f2(w.y));
-          ffma2(acc[2], pp, bf16x2_to_f2(w.z));
-          ffma2(acc[3], pp, bf16x2_to_f2(w.w));
-        }
-      }
-      float* dst = accs + (size_t)grp * G * r_v + h * r_v + c * 8;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        dst[2 * i] = acc[i].x;
-        dst[2 * i + 1] = acc[i].y;
+        mma_bf16_16816(c, a0, a1, a2, a3, b0, b1);
       }
     }
+    const int t0 = warp * 16 + lq, t1 = t0 + 8;
+    const bool v0 = tok_ok(t0), v1 = tok_ok(t1);
+    const int h0 = 2 * lr, h1 = 2 * lr + 1;
+    float sc[2][2];  // [token 0/1][head h0/h1], log2-scaled
+    sc[0][0] = (v0 && h0 < G) ? c[0] * a.scale_log2 : -INFINITY;
+    sc[0][1] = (v0 && h1 < G) ? c[1] * a.scale_log2 : -INFINITY;
+    sc[1][0] = (v1 && h0 < G) ? c[2] * a.scale_log2 : -INFINITY;
+    sc[1][1] = (v1 && h1 < G) ? c[3] * a.scale_log2 : -INFINITY;
+    // item maximum per head: over the warp's tokens (lanes with equal l%4),
+    // then over the warps
+    float mx0 = fmaxf(sc[0][0], sc[1][0]), mx1 = fmaxf(sc[0][1], sc[1][1]);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    if (lq == 0) {
+      if (h0 < G) red[warp * G + h0] = mx0;
+      if (h1 < G) red[warp * G + h1] = mx1;
+    }
     named_bar_sync(1, kAttConsumers);
-    // All reads of the stage are done: release it to the producer.
-    if (lane == 0) mbar_arrive(&empty[s]);
+    float m0 = -INFINITY, m1 = -INFINITY;
+    for (int w = 0; w < kAttConsumerWarps; ++w) {
+      if (h0 < G) m0 = fmaxf(m0, red[w * G + h0]);
+      if (h1 < G) m1 = fmaxf(m1, red[w * G + h1]);
+    }
+    // weights, their sums, and the weights for PV (ps[h][t])
+    const float p00 = sc[0][0] > -INFINITY ? exp2f(sc[0][0] - m0) : 0.f;
+    const float p01 = sc[0][1] > -INFINITY ? exp2f(sc[0][1] - m1) : 0.f;
+    const float p10 = sc[1][0] > -INFINITY ? exp2f(sc[1][0] - m0) : 0.f;
+    const float p11 = sc[1][1] > -INFINITY ? exp2f(sc[1][1] - m1) : 0.f;
+    if (h0 < G) {
+      ps[h0 * kAttTokens + t0] = p00;
+      ps[h0 * kAttTokens + t1] = p10;
+    }
+    if (h1 < G) {
+      ps[h1 * kAttTokens + t0] = p01;
+      ps[h1 * kAttTokens + t1] = p11;
+    }
+    float l0 = p00 + p10, l1 = p01 + p11;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+    }
+    if (lq == 0) {
+      if (h0 < G) red[(kAttConsumerWarps + warp) * G + h0] = l0;
+      if (h1 < G) red[(kAttConsumerWarps + warp) * G + h1] = l1;
+    }
+    // Latent rows of tokens that do not exist (past the length, or pages the
+    // split does not have) hold whatever the stage held before: zero them so
+    // a zero weight never meets a NaN.
+    if (ready && lane < 16) {
+      const int t = warp * 16 + lane;
+      if (!tok_ok(t)) {
+        const int pl = t >> logS, rw = t & (S - 1);
+        uint8_t* zb = const_cast<uint8_t*>(st) + geo.z_off + pl * geo.nzb * geo.zbox;
+        for (int cz = 0; cz < r_v / 8; ++cz)
+          *reinterpret_cast<uint4*>(zb + (cz / zc_per_box) * geo.zbox +
+                                    swz(rw * geo.wz * 2 + (cz % zc_per_box) * 16, zmask)) =
+              make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async();  // the stage is refilled by TMA (async proxy) later
+      }
+    }
+    named_bar_sync(1, kAttConsumers);
+
+    // ---- PV: a[h][j] = sum_t p[h][t] z[t][j], warp = 16-row latent tiles
     float* out = a.partial + ((size_t)bg * a.nsplit + j) * G * (r_v + 2);
-    for (int i = tid; ready && i < G * r_v; i += kAttConsumers) {
-      const int h = i / r_v, jj = i % r_v;
-      float v = 0.f;
-      for (int gi = 0; gi < ngrp; ++gi) v += accs[(size_t)gi * G * r_v + i];
-      out[h * (r_v + 2) + 2 + jj] = v;
+    for (int mt = warp; ready && mt < r_v / 16; mt += kAttConsumerWarps) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < kAttTokens / 16; ++ks) {
+        const int t_ld = ks * 16 + (mi >> 1) * 8 + mr;
+        const int jc = mt * 2 + (mi & 1);  // 16-byte chunk of the z row
+        const uint8_t* zrow = st + geo.z_off + (t_ld >> logS) * geo.nzb * geo.zbox;
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4_trans(smem_u32(zrow + (jc / zc_per_box) * geo.zbox +
+                                   swz((t_ld & (S - 1)) * geo.wz * 2 + (jc % zc_per_box) * 16,
+                                       zmask)),
+                          a0, a1, a2, a3);
+        float q00 = 0.f, q01 = 0.f, q10 = 0.f, q11 = 0.f;
+        if (lq < G) {
+          const float* pr = ps + lq * kAttTokens + ks * 16 + 2 * lr;
+          q00 = pr[0];
+          q01 = pr[1];
+          q10 = pr[8];
+          q11 = pr[9];
+        }
+        uint32_t bh0, bh1, bl0, bl1;
+        split_bf16x2(q00, q01, bh0, bl0);
+        split_bf16x2(q10, q11, bh1, bl1);
+        mma_bf16_16816(acc, a0, a1, a2, a3, bh0, bh1);
+        mma_bf16_16816(acc, a0, a1, a2, a3, bl0, bl1);
+      }
+      const int jr = mt * 16 + lq;
+      if (h0 < G) {
+        out[h0 * (r_v + 2) + 2 + jr] = acc[0];
+        out[h0 * (r_v + 2) + 2 + jr + 8] = acc[2];
+      }
+      if (h1 < G) {
+        out[h1 * (r_v + 2) + 2 + jr] = acc[1];
+        out[h1 * (r_v + 2) + 2 + jr + 8] = acc[3];
+      }
     }
+    // this warp has finished reading the stage
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
     if (ready && tid < G) {
-      float l = 0.f;
-      for (int w = 0; w < kAttConsumerWarps; ++w) l += red[(kAttConsumerWarps + w) * G + tid];
-      out[tid * (r_v + 2)] = mh[tid];
+      float l = 0.f, m = -INFINITY;
+      for (int w = 0; w < kAttConsumerWarps; ++w) {
+        l += red[(kAttConsumerWarps + w) * G + tid];
+        m = fmaxf(m, red[w * G + tid]);
+      }
+      out[tid * (r_v + 2)] = m;
       out[tid * (r_v + 2) + 1] = l;
     }
-    named_bar_sync(1, kAttConsumers);  // scratch is reused by the next item
   }
 }
 
@@ -419,36 +445,31 @@ AttendGeom attend_geometry(int G, int d, int r_v, int S, int wz) {
   g.q_off = g.z_off + round1k(g.ppi * g.nzb * g.zbox);
   g.meta_off = g.q_off + G * d * 2;
   g.stage_bytes = round1k(g.meta_off + kMetaInts * 4);
-  g.qs_stride = d + 8;
-  const int nslot = G * r_v / 8;
-  const int ngrp = kAttConsumers / nslot > 0 ? kAttConsumers / nslot : 1;
-  const int scratch = G * g.qs_stride * 4 + kAttTokens * G * 4 +
-                      2 * kAttConsumerWarps * G * 4 + ngrp * G * r_v * 4 + 2048;
+  // weights [2][G][64] and reductions [2][2][warps][G]
+  const int scratch = 2 * G * kAttTokens * 4 + 2 * 2 * kAttConsumerWarps * G * 4 + 64;
   // 228 KB of shared memory per SM, 1 KB reserved per CTA, 1 KB of slack for
   // the 1024-byte alignment of the base.
   const int budget = 228 * 1024 / kAttCtasPerSm - 2048 - 64 - scratch;
   g.stages = budget / g.stage_bytes;
   if (g.stages > 6) g.stages = 6;
-  g.qs_off = g.stages * g.stage_bytes;
-  g.ps_off = g.qs_off + G * g.qs_stride * 4;
-  g.red_off = g.ps_off + kAttTokens * G * 4;
-  g.acc_off = g.red_off + 2 * kAttConsumerWarps * G * 4;
-  g.smem_bytes = (g.acc_off + ngrp * G * r_v * 4 + 15) / 16 * 16;
+  g.ps_off = g.stages * g.stage_bytes;
+  g.red_off = g.ps_off + 2 * G * kAttTokens * 4;
+  g.smem_bytes = (g.red_off + 2 * 2 * kAttConsumerWarps * G * 4 + 15) / 16 * 16;
   return g;
 }
 
-template <int G>
+template <int G, int D>
 cudaError_t launch_attend_g(const AttendArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmZ,
                             const AttendGeom& geo, cudaStream_t st, bool pdl) {
   const size_t smem = (size_t)geo.smem_bytes + 2 * geo.stages * 8 + 16 + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attend_kernel<G>,
+  cudaError_t e = cudaFuncSetAttribute(attend_kernel<G, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long items = (long)a.B * a.Hkv * a.nsplit;
   long grid = (long)num_sms() * kAttCtasPerSm;
   if (grid > items) grid = items;
   if (grid < 1) grid = 1;
-  return launch_k(attend_kernel<G>, dim3((unsigned)grid), dim3(kAttThreads), smem, st, pdl, tmK,
+  return launch_k(attend_kernel<G, D>, dim3((unsigned)grid), dim3(kAttThreads), smem, st, pdl, tmK,
                   tmZ, a, geo);
 }
 
@@ -461,10 +482,15 @@ cudaError_t launch_attend(const AttendArgs& a, const CUtensorMap& tmK, const CUt
   const AttendGeom geo = attend_geometry(a.G, a.d, a.r_v, a.S, wz);
   if (geo.stages < 2 || geo.ppi > 31) return cudaErrorInvalidConfiguration;
   switch (a.G) {
-    case 1: return launch_attend_g<1>(a, tmK, tmZ, geo, st, pdl);
-    case 2: return launch_attend_g<2>(a, tmK, tmZ, geo, st, pdl);
-    case 4: return launch_attend_g<4>(a, tmK, tmZ, geo, st, pdl);
-    case 8: return launch_attend_g<8>(a, tmK, tmZ, geo, st, pdl);
+#define BKV_ATT(GG)                                                        \
+  case GG:                                                                 \
+    return a.d == 64 ? launch_attend_g<GG, 64>(a, tmK, tmZ, geo, st, pdl) \
+                     : launch_attend_g<GG, 128>(a, tmK, tmZ, geo, st, pdl);
+    BKV_ATT(1)
+    BKV_ATT(2)
+    BKV_ATT(4)
+    BKV_ATT(8)
+#undef BKV_ATT
     default: return cudaErrorInvalidValue;
   }
 }
