@@ -123,6 +123,18 @@ BASISKV_API int basiskv_fold_outproj(const basiskv_dims* dims, const basiskv_bf1
                          const basiskv_bf16* W_O, basiskv_bf16* W_fold,
                          void* stream);
 
+/* Offline fold of the append factors for the tensor-core prefill path.
+ * Per KV head g, with M_g = A_V,g P_K,g U_K,g (d x r_k, fp32):
+ *   W_app[g][n][i]     = A_V[g][i][n]      n < r_v, i < d     (z = v A_V)
+ *   W_app[g][n][d + i] = 0                 n < r_v
+ *   W_app[g][r_v+c][i]     = -M_g[i][c]    c < r_k, i < d
+ *   W_app[g][r_v+c][d + i] = U_K[g][i][c]               (e = k U_K - v M_g)
+ * so that [z | e] = [v | k] W_app^T.  W_app: bf16 [Hkv][r_v + r_k][2d].
+ * Uses no workspace. */
+BASISKV_API int basiskv_fold_append(const basiskv_dims* dims, const basiskv_bf16* A_V,
+                                    const basiskv_bf16* P_K, const basiskv_bf16* U_K,
+                                    basiskv_bf16* W_app, void* stream);
+
 /* Cache append: the Value is kept only as its latent and the Key as a
  * residual code beside the exact Key (abstract; Table 4 rows).  For each sequence b and its n_new new tokens j:
  *   position t = seq_lens[b] + j, KV head g:
@@ -135,12 +147,16 @@ BASISKV_API int basiskv_fold_outproj(const basiskv_dims* dims, const basiskv_bf1
  * BASISKV_DEV_OVERFLOW is raised; seq_lens[b] is then left unchanged.
  * A prefill chunk is an append with n_new > 1; to fill one sequence only,
  * pass dims->B = 1 and seq_lens / block_table offset to that sequence.
- * n_new*B >= 128 runs the tensor-core (tcgen05) path. */
+ * n_new*B >= 128 runs the tensor-core (tcgen05) path: [z | e] = [v | k]
+ * W_app^T with W_app as built by basiskv_fold_append (W_app may be NULL:
+ * the call then folds it into the workspace first); the residual then uses
+ * the bf16-rounded fold instead of the unrounded z.  Smaller appends run
+ * the two-step CUDA-core form and ignore W_app. */
 BASISKV_API int basiskv_append(const basiskv_dims* dims, const basiskv_bf16* k_new,
                    const basiskv_bf16* v_new, int n_new, int32_t* seq_lens,
                    const int32_t* block_table, const basiskv_bf16* A_V,
                    const basiskv_bf16* P_K, const basiskv_bf16* U_K,
-                   basiskv_bf16* K_cache, basiskv_bf16* Z_cache,
+                   const basiskv_bf16* W_app, basiskv_bf16* K_cache, basiskv_bf16* Z_cache,
                    basiskv_bf16* E_cache, void* workspace,
                    size_t workspace_bytes, void* stream);
 

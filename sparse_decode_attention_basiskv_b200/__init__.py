@@ -61,7 +61,8 @@ _DIMS = ctypes.POINTER(Dims)
 _SIGNATURES = {
     "basiskv_workspace_size": (_SZ, [_DIMS, _I, _I]),
     "basiskv_fold_outproj": (_I, [_DIMS, _P, _P, _P, _P]),
-    "basiskv_append": (_I, [_DIMS, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "basiskv_fold_append": (_I, [_DIMS, _P, _P, _P, _P, _P]),
+    "basiskv_append": (_I, [_DIMS, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "basiskv_route": (_I, [_DIMS, _P, _P, _I, _P, _P, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "basiskv_attend": (_I, [_DIMS, _P, _P, _I, _P, _P, _P, _P, _I, _P, _P, _SZ, _P]),
     "basiskv_outproj": (_I, [_DIMS, _P, _P, _P, _P, _SZ, _P]),
@@ -134,12 +135,18 @@ def basiskv_fold_outproj(dims: Dims, B_V, W_O, W_fold, stream=None) -> None:
         "basiskv_fold_outproj")
 
 
+def basiskv_fold_append(dims: Dims, A_V, P_K, U_K, W_app, stream=None) -> None:
+    _check(load_library().basiskv_fold_append(
+        ctypes.byref(dims), _ptr(A_V), _ptr(P_K), _ptr(U_K), _ptr(W_app), _stream(stream)),
+        "basiskv_fold_append")
+
+
 def basiskv_append(dims: Dims, k_new, v_new, n_new: int, seq_lens, block_table, A_V, P_K,
-                   U_K, K_cache, Z_cache, E_cache, workspace, stream=None) -> None:
+                   U_K, K_cache, Z_cache, E_cache, workspace, stream=None, W_app=None) -> None:
     _check(load_library().basiskv_append(
         ctypes.byref(dims), _ptr(k_new), _ptr(v_new), n_new, _ptr(seq_lens),
-        _ptr(block_table), _ptr(A_V), _ptr(P_K), _ptr(U_K), _ptr(K_cache), _ptr(Z_cache),
-        _ptr(E_cache), _ptr(workspace), _nbytes(workspace), _stream(stream)),
+        _ptr(block_table), _ptr(A_V), _ptr(P_K), _ptr(U_K), _ptr(W_app), _ptr(K_cache),
+        _ptr(Z_cache), _ptr(E_cache), _ptr(workspace), _nbytes(workspace), _stream(stream)),
         "basiskv_append")
 
 

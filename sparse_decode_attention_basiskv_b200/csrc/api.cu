@@ -94,6 +94,19 @@ bool make_tmap_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t co
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_3d(CUtensorMap* out, const void* base, const uint64_t dims[3],
+                  const uint64_t strides[2], const uint32_t box[3], CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t gd[3] = {dims[0], dims[1], dims[2]};
+  const cuuint64_t gs[2] = {strides[0], strides[1]};
+  const cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), gd, gs, bx, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace basiskv
 
 using namespace basiskv;
@@ -150,7 +163,7 @@ int check_len_topk(const basiskv_dims* d, int top_k, int max_seq_len) {
 }
 
 struct WsLayout {
-  size_t qt, scores, sel, partial, a_f32, a_bf16, op_part, total;
+  size_t qt, scores, sel, partial, a_f32, a_bf16, op_part, w_app, total;
   int nsplit, ppi;
 };
 
@@ -174,6 +187,8 @@ WsLayout ws_layout(const basiskv_dims* d, int top_k) {
   off += align256((size_t)d->B * d->Hq * d->r_v * 2);
   w.op_part = off;
   off += align256((size_t)kMaxKsplit * d->B * d->hidden * 4);
+  w.w_app = off;
+  off += align256(append_factor_bytes(d->Hkv, d->d, d->r_v, d->r_k));
   w.total = off;
   return w;
 }
@@ -204,7 +219,7 @@ int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_b
                int n_new, int32_t* seq_lens, const int32_t* block_table, const basiskv_bf16* A_V,
                const basiskv_bf16* P_K, const basiskv_bf16* U_K, basiskv_bf16* K_cache,
                basiskv_bf16* Z_cache, basiskv_bf16* E_cache, cudaStream_t st, bool pdl,
-               bool bump = true) {
+               bool bump = true, uint16_t* w_app = nullptr, bool fold_first = false) {
   AppendArgs a{};
   a.k_new = k_new;
   a.v_new = v_new;
@@ -228,7 +243,28 @@ int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_b
   a.num_phys = d->num_phys_pages;
   a.status = device_status_ptr();
   if (!a.status) return BASISKV_ERR_CUDA;
-  int rc = launch_status(launch_append_small(a, st, pdl));
+  int rc;
+  if (w_app) {  // prefill chunk: one tensor-core product per KV head
+    if (fold_first) {
+      FoldAppArgs f{A_V, P_K, U_K, w_app, d->Hkv, d->d, d->r_v, d->r_k};
+      rc = launch_status(launch_fold_append(f, st, pdl));
+      if (rc) return rc;
+    }
+    const int N = d->r_v + d->r_k;
+    const uint64_t rows = (uint64_t)d->B * n_new;
+    const uint64_t dims3[3] = {(uint64_t)d->d, (uint64_t)d->Hkv, rows};
+    const uint64_t str3[2] = {(uint64_t)d->d * 2, (uint64_t)d->Hkv * d->d * 2};
+    const uint32_t box3[3] = {64, 1, 128};
+    CUtensorMap tmV, tmK, tmW;
+    if (!make_tmap_3d(&tmV, v_new, dims3, str3, box3, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_3d(&tmK, k_new, dims3, str3, box3, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&tmW, w_app, (uint64_t)d->Hkv * N, 2 * d->d, (uint64_t)4 * d->d, N, 64,
+                      CU_TENSOR_MAP_SWIZZLE_128B))
+      return BASISKV_ERR_CUDA;
+    rc = launch_status(launch_append_tc(a, tmV, tmK, tmW, st, pdl));
+  } else {
+    rc = launch_status(launch_append_small(a, st, pdl));
+  }
   if (rc || !bump) return rc;
   return launch_status(launch_bump_lengths(a, st, pdl));
 }
@@ -381,10 +417,23 @@ int basiskv_fold_outproj(const basiskv_dims* dims, const basiskv_bf16* B_V,
   return launch_status(launch_fold_outproj(a, static_cast<cudaStream_t>(stream)));
 }
 
+int basiskv_fold_append(const basiskv_dims* dims, const basiskv_bf16* A_V,
+                        const basiskv_bf16* P_K, const basiskv_bf16* U_K, basiskv_bf16* W_app,
+                        void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  BKV_REQUIRE(A_V);
+  BKV_REQUIRE(P_K);
+  BKV_REQUIRE(U_K);
+  BKV_REQUIRE(W_app);
+  FoldAppArgs f{A_V, P_K, U_K, W_app, dims->Hkv, dims->d, dims->r_v, dims->r_k};
+  return launch_status(launch_fold_append(f, static_cast<cudaStream_t>(stream), false));
+}
+
 int basiskv_append(const basiskv_dims* dims, const basiskv_bf16* k_new, const basiskv_bf16* v_new,
                    int n_new, int32_t* seq_lens, const int32_t* block_table,
                    const basiskv_bf16* A_V, const basiskv_bf16* P_K, const basiskv_bf16* U_K,
-                   basiskv_bf16* K_cache, basiskv_bf16* Z_cache, basiskv_bf16* E_cache,
+                   const basiskv_bf16* W_app, basiskv_bf16* K_cache, basiskv_bf16* Z_cache, basiskv_bf16* E_cache,
                    void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
@@ -400,10 +449,21 @@ int basiskv_append(const basiskv_dims* dims, const basiskv_bf16* k_new, const ba
   BKV_REQUIRE(K_cache);
   BKV_REQUIRE(Z_cache);
   BKV_REQUIRE(E_cache);
-  (void)workspace;
-  (void)workspace_bytes;
+  // Chunks of at least 128 token rows take the tensor-core path; without a
+  // caller-folded W_app the fold goes to the workspace first.
+  uint16_t* w_ws = nullptr;
+  const bool tc = (long long)dims->B * n_new >= 128;
+  if (tc && W_app && !aligned16(W_app)) return BASISKV_ERR_INVALID_ARG;
+  if (tc && !W_app) {
+    WsLayout L;
+    rc = check_ws(dims, 2, workspace, workspace_bytes, &L);
+    if (rc) return rc;
+    w_ws = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) + L.w_app);
+  }
   return run_append(dims, k_new, v_new, n_new, seq_lens, block_table, A_V, P_K, U_K, K_cache,
-                    Z_cache, E_cache, static_cast<cudaStream_t>(stream), pdl_enabled());
+                    Z_cache, E_cache, static_cast<cudaStream_t>(stream), pdl_enabled(), true,
+                    tc ? (W_app ? const_cast<uint16_t*>(W_app) : w_ws) : nullptr,
+                    tc && !W_app);
 }
 
 int basiskv_route(const basiskv_dims* dims, const basiskv_bf16* q, const int32_t* seq_lens,

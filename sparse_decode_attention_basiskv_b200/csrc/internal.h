@@ -16,6 +16,9 @@ namespace basiskv {
 bool make_tmap_2d(CUtensorMap* out, const void* base, uint64_t rows, uint64_t cols,
                   uint64_t row_bytes, uint32_t box_rows, uint32_t box_cols,
                   CUtensorMapSwizzle swizzle);
+// 3-D bf16 tensor map, dims innermost first, byte strides of dims 1 and 2.
+bool make_tmap_3d(CUtensorMap* out, const void* base, const uint64_t dims[3],
+                  const uint64_t strides[2], const uint32_t box[3], CUtensorMapSwizzle swizzle);
 
 // Address of this library's device status word on the current device.
 unsigned int* device_status_ptr();
@@ -40,6 +43,22 @@ struct AppendArgs {
   unsigned int* status;
 };
 cudaError_t launch_append_small(const AppendArgs& a, cudaStream_t st, bool pdl);
+
+// Prefill path (tensor cores): W_app = [[A_V^T, 0], [-(A_V P_K U_K)^T, U_K^T]]
+// per KV head, [Hkv][r_v + r_k][2d] bf16, then [z | e] = [v | k] W_app^T.
+struct FoldAppArgs {
+  const uint16_t* A_V;
+  const uint16_t* P_K;
+  const uint16_t* U_K;
+  uint16_t* W_app;
+  int Hkv, d, r_v, r_k;
+};
+size_t append_factor_bytes(int Hkv, int d, int r_v, int r_k);
+cudaError_t launch_fold_append(const FoldAppArgs& a, cudaStream_t st, bool pdl);
+// tmV, tmK: 3-D maps over [rows][Hkv][d] (box 64 x 1 x 128); tmW: 2-D map over
+// [Hkv*(r_v+r_k)][2d] (box (r_v+r_k) x 64); all with 128-byte swizzle.
+cudaError_t launch_append_tc(const AppendArgs& a, const CUtensorMap& tmV, const CUtensorMap& tmK,
+                             const CUtensorMap& tmW, cudaStream_t st, bool pdl);
 cudaError_t launch_bump_lengths(const AppendArgs& a, cudaStream_t st, bool pdl);
 
 // ------------------------------------------------------------------- route

@@ -9,7 +9,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (Dims, basiskv_decode, basiskv_fold_outproj, workspace_size)
+from . import (Dims, basiskv_append, basiskv_decode, basiskv_fold_append, basiskv_fold_outproj,
+               workspace_size)
 
 
 class DecodeLayer:
@@ -26,6 +27,9 @@ class DecodeLayer:
         self.W_fold = torch.empty(dims.hidden, dims.Hq * dims.r_v, dtype=torch.bfloat16,
                                   device=dev)
         basiskv_fold_outproj(dims, factors["B_V"], factors["W_O"], self.W_fold, stream)
+        self.W_app = torch.empty(dims.Hkv, dims.r_v + dims.r_k, 2 * dims.d, dtype=torch.bfloat16,
+                                 device=dev)
+        basiskv_fold_append(dims, self.A_V, self.P_K, self.U_K, self.W_app, stream)
         n = workspace_size(dims, top_k, max_seq_len)
         if n == 0:
             raise ValueError("unsupported dims for the BasisKV library")
@@ -44,6 +48,13 @@ class DecodeLayer:
         caches = {k: v.contiguous() for k, v in pb.paged().items()}
         return cls(dims, factors, caches, pb.table.to(device).contiguous(),
                    pb.seq_lens.to(device).clone(), wl.top_k, pc * wl.page_size, stream)
+
+    def append(self, k_new, v_new, n_new: int, stream=None) -> None:
+        """Appends n_new tokens ([B][n_new][Hkv][d] bf16) to every sequence
+        (a prefill chunk runs on the tensor cores with the folded factor)."""
+        basiskv_append(self.dims, k_new, v_new, n_new, self.seq_lens, self.block_table, self.A_V,
+                       self.P_K, self.U_K, self.K, self.Z, self.E, self.workspace, stream,
+                       W_app=self.W_app)
 
     def decode(self, q, k_new=None, v_new=None, sel=None, max_seq_len=None, y=None,
                stream=None) -> torch.Tensor:

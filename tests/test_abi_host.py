@@ -29,7 +29,7 @@ def lib():
 
 def test_header_symbols_are_exported(lib):
     names = bkv.header_symbols()
-    assert len(names) == 11
+    assert len(names) == 12
     out = subprocess.run(["nm", "-D", "--defined-only", bkv.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
@@ -99,10 +99,16 @@ def test_other_entry_points_validate(lib):
                               FAKE, big, None) == bkv.ERR_INVALID_ARG
     assert lib.basiskv_outproj(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, 16,
                                None) == bkv.ERR_WORKSPACE_TOO_SMALL
-    assert lib.basiskv_append(ctypes.byref(d), FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
-                              FAKE, FAKE, FAKE, big, None) == bkv.ERR_INVALID_ARG
-    assert lib.basiskv_append(ctypes.byref(d), FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
-                              None, FAKE, FAKE, big, None) == bkv.ERR_INVALID_ARG
+    assert lib.basiskv_append(ctypes.byref(d), FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                              FAKE, FAKE, FAKE, FAKE, big, None) == bkv.ERR_INVALID_ARG
+    assert lib.basiskv_append(ctypes.byref(d), FAKE, FAKE, 1, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                              FAKE, None, FAKE, FAKE, big, None) == bkv.ERR_INVALID_ARG
+    # a chunk for the tensor-core path with a misaligned folded factor
+    assert lib.basiskv_append(ctypes.byref(d), FAKE, FAKE, 64, FAKE, FAKE, FAKE, FAKE, FAKE,
+                              FAKE + 2, FAKE, FAKE, FAKE, FAKE, big,
+                              None) == bkv.ERR_INVALID_ARG
+    assert lib.basiskv_fold_append(ctypes.byref(d), FAKE, None, FAKE, FAKE,
+                                   None) == bkv.ERR_INVALID_ARG
     assert lib.basiskv_decode(ctypes.byref(d), FAKE, FAKE, None, FAKE, 100, FAKE, FAKE, FAKE,
                               FAKE, FAKE, FAKE, FAKE, FAKE, 8, None, FAKE, FAKE, big,
                               None) == bkv.ERR_INVALID_ARG  # k_new without v_new

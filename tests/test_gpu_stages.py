@@ -188,9 +188,12 @@ def test_block_table_permutation_invariance():
     assert torch.equal(sc1, sc2) and torch.equal(sel1, sel2) and torch.equal(y1, y2)
 
 
-def test_prefill_chunk_append():
+@pytest.mark.parametrize("prefolded", [True, False], ids=["W_app", "fold_in_call"])
+def test_prefill_chunk_append(prefolded):
     """A 4096-token prefill chunk appended to one sequence of the Qwen3-32B
-    layer shape (B = 1 view of the batch), compared token by token."""
+    layer shape (B = 1 view of the batch; the tensor-core path), compared
+    token by token; the folded append factor is either built once up front
+    or folded inside the call."""
     wl = synth.with_sizes(synth.QWEN32B_T64K_B8, B=2, T=96, prefill_tokens=4096)
     pb, layer = gpu_layer(wl)
     f = factors_np(pb)
@@ -202,7 +205,7 @@ def test_prefill_chunk_append():
                      num_phys_pages=layer.dims.num_phys_pages)
     bkv.basiskv_append(dims1, k[b].contiguous(), v[b].contiguous(), 4096, layer.seq_lens[b:],
                        layer.block_table[b], layer.A_V, layer.P_K, layer.U_K, layer.K, layer.Z,
-                       layer.E, layer.workspace)
+                       layer.E, layer.workspace, W_app=layer.W_app if prefolded else None)
     status_clean()
     assert layer.seq_lens.tolist() == [wl.T, wl.T + 4096]
     for g in range(wl.Hkv):
