@@ -317,8 +317,11 @@ def run_gpu(args) -> None:
     if os.path.exists(tr_path):
         with open(tr_path) as f:
             tr = json.load(f)
+        # DRAM traffic of one launch, captured with ncu on a smaller batch of the
+        # same kernel (B = 4) and scaled by the units processed: traffic grows in
+        # proportion to the pages streamed.
         if tr.get("kernel_source_sha") == _route_source_sha():
-            traffic = tr["bytes_per_launch_scaled"]
+            traffic = tr["traffic_over_algorithmic"] * route_bytes
 
     # ------------------------------------ end to end through the public API
     layer.seq_lens.fill_(T0)
