@@ -163,7 +163,8 @@ int check_len_topk(const basiskv_dims* d, int top_k, int max_seq_len) {
 }
 
 struct WsLayout {
-  size_t qt, scores, sel, partial, a_f32, a_bf16, op_part, w_app, total;
+  size_t qt, scores, sel, partial, a_f32, a_bf16, op_part, w_app, counters, total;
+  int n_att_cnt, n_op_cnt;
   int nsplit, ppi;
 };
 
@@ -189,6 +190,12 @@ WsLayout ws_layout(const basiskv_dims* d, int top_k) {
   off += align256((size_t)kMaxKsplit * d->B * d->hidden * 4);
   w.w_app = off;
   off += align256(append_factor_bytes(d->Hkv, d->d, d->r_v, d->r_k));
+  // arrival counters of the fused decode: one per (sequence, KV head) for the
+  // attention merge, then one per 128-row tile of the out-projection
+  w.n_att_cnt = d->B * d->Hkv;
+  w.n_op_cnt = (d->hidden + 127) / 128;
+  w.counters = off;
+  off += align256((size_t)(w.n_att_cnt + w.n_op_cnt) * 4);
   w.total = off;
   return w;
 }
@@ -215,11 +222,11 @@ int z_box_cols(int r_v) { return r_v % 64 == 0 ? 64 : (r_v % 32 == 0 ? 32 : 16);
 int e_box_cols(int r_k) { return r_k % 32 == 0 ? 32 : 16; }
 
 // ---------------------------------------------------------------- stages
-int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_bf16* v_new,
-               int n_new, int32_t* seq_lens, const int32_t* block_table, const basiskv_bf16* A_V,
-               const basiskv_bf16* P_K, const basiskv_bf16* U_K, basiskv_bf16* K_cache,
-               basiskv_bf16* Z_cache, basiskv_bf16* E_cache, cudaStream_t st, bool pdl,
-               bool bump = true, uint16_t* w_app = nullptr, bool fold_first = false) {
+AppendArgs make_append_args(const basiskv_dims* d, const basiskv_bf16* k_new,
+                            const basiskv_bf16* v_new, int n_new, int32_t* seq_lens,
+                            const int32_t* block_table, const basiskv_bf16* A_V,
+                            const basiskv_bf16* P_K, const basiskv_bf16* U_K,
+                            basiskv_bf16* K_cache, basiskv_bf16* Z_cache, basiskv_bf16* E_cache) {
   AppendArgs a{};
   a.k_new = k_new;
   a.v_new = v_new;
@@ -242,6 +249,16 @@ int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_b
   a.max_pages = d->max_pages_per_seq;
   a.num_phys = d->num_phys_pages;
   a.status = device_status_ptr();
+  return a;
+}
+
+int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_bf16* v_new,
+               int n_new, int32_t* seq_lens, const int32_t* block_table, const basiskv_bf16* A_V,
+               const basiskv_bf16* P_K, const basiskv_bf16* U_K, basiskv_bf16* K_cache,
+               basiskv_bf16* Z_cache, basiskv_bf16* E_cache, cudaStream_t st, bool pdl,
+               bool bump = true, uint16_t* w_app = nullptr, bool fold_first = false) {
+  AppendArgs a = make_append_args(d, k_new, v_new, n_new, seq_lens, block_table, A_V, P_K, U_K,
+                                  K_cache, Z_cache, E_cache);
   if (!a.status) return BASISKV_ERR_CUDA;
   int rc;
   if (w_app) {  // prefill chunk: one tensor-core product per KV head
@@ -273,7 +290,7 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
               int max_seq_len, const int32_t* block_table, const basiskv_bf16* P_K,
               const basiskv_bf16* U_K, const basiskv_bf16* Z_cache, const basiskv_bf16* E_cache,
               int top_k, float* scores, int32_t* sel, uint8_t* ws, const WsLayout& L,
-              cudaStream_t st, bool pdl, int len_offset = 0) {
+              cudaStream_t st, bool pdl, int len_offset = 0, bool do_fold = true) {
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   const int wz = z_box_cols(d->r_v), we = e_box_cols(d->r_k);
@@ -281,9 +298,12 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   if (!cache_map(&tmZ, Z_cache, d, d->r_v, wz) || !cache_map(&tmE, E_cache, d, d->r_k, we))
     return BASISKV_ERR_CUDA;
   float* qt = reinterpret_cast<float*>(ws + L.qt);
-  FoldQArgs f{q, P_K, U_K, qt, d->B, d->Hq, d->Hkv, d->d, d->r_v, d->r_k};
-  int rc = launch_status(launch_fold_query(f, st, pdl));
-  if (rc) return rc;
+  int rc = BASISKV_OK;
+  if (do_fold) {
+    FoldQArgs f{q, P_K, U_K, qt, d->B, d->Hq, d->Hkv, d->d, d->r_v, d->r_k};
+    rc = launch_status(launch_fold_query(f, st, pdl));
+    if (rc) return rc;
+  }
   RouteArgs r{};
   r.qt = qt;
   r.seq_lens = seq_lens;
@@ -311,7 +331,7 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
                const int32_t* block_table, const basiskv_bf16* K_cache,
                const basiskv_bf16* Z_cache, const int32_t* sel, int top_k, float* a_lat,
                uint16_t* a_bf16, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl,
-               int len_offset = 0) {
+               int len_offset = 0, int* cnt = nullptr) {
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   const int wz = z_box_cols(d->r_v);
@@ -339,6 +359,13 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
   a.len_offset = len_offset;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d->d));
   a.status = status;
+  // Fused merge of the splits when its shared-memory scratch stays small.
+  if (cnt && (size_t)2 * L.nsplit * a.G * 4 <= 4096) {
+    a.cnt = cnt;
+    a.a_lat = a_lat;
+    a.a_bf16 = a_bf16;
+    return launch_status(launch_attend(a, tmK, tmZ, wz, st, pdl));
+  }
   int rc = launch_status(launch_attend(a, tmK, tmZ, wz, st, pdl));
   if (rc) return rc;
   CombineArgs c{a.partial, seq_lens, a_lat, a_bf16, d->B, d->Hq, d->Hkv, a.G, d->r_v,
@@ -348,7 +375,7 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
 
 int run_outproj(const basiskv_dims* d, const uint16_t* a_bf16, const basiskv_bf16* W_fold,
                 basiskv_bf16* y, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl,
-                int32_t* bump_lens = nullptr) {
+                int32_t* bump_lens = nullptr, int* cnt = nullptr) {
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   const int K = d->Hq * d->r_v;
@@ -371,6 +398,7 @@ int run_outproj(const basiskv_dims* d, const uint16_t* a_bf16, const basiskv_bf1
   o.bump_lens = bump_lens;
   o.bump_n = 1;
   o.bump_cap = d->max_pages_per_seq * d->page_size;
+  o.cnt = cnt;
   return launch_status(launch_outproj(o, tmW, tmA, st, pdl));
 }
 
@@ -575,19 +603,29 @@ int basiskv_decode(const basiskv_dims* dims, const basiskv_bf16* q, const basisk
   // only at the end of the step (by the out-projection launch), and the
   // stages in between read seq_lens[b] + 1.
   const int off = append ? 1 : 0;
-  if (append) {
-    rc = run_append(dims, k_new, v_new, 1, seq_lens, block_table, A_V, P_K, U_K, K_cache, Z_cache,
-                    E_cache, st, pdl, /*bump=*/false);
+  // Launch 1: the query fold and the token append side by side; it also
+  // zeroes the arrival counters of the fused merge and reduction below.
+  int* cnt = reinterpret_cast<int*>(ws + L.counters);
+  {
+    AppendArgs a = make_append_args(dims, append ? k_new : nullptr, v_new, 1, seq_lens,
+                                    block_table, A_V, P_K, U_K, K_cache, Z_cache, E_cache);
+    if (!a.status) return BASISKV_ERR_CUDA;
+    FoldQArgs f{q, P_K, U_K, reinterpret_cast<float*>(ws + L.qt), dims->B, dims->Hq, dims->Hkv,
+                dims->d, dims->r_v, dims->r_k};
+    rc = launch_status(
+        launch_decode_prologue(f, a, cnt, L.n_att_cnt + L.n_op_cnt, st, pdl));
     if (rc) return rc;
   }
   rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache, top_k,
-                 reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl, off);
+                 reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl, off,
+                 /*do_fold=*/false);
   if (rc) return rc;
   uint16_t* a16 = reinterpret_cast<uint16_t*>(ws + L.a_bf16);
   rc = run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel_buf, top_k, nullptr, a16,
-                  ws, L, st, pdl, off);
+                  ws, L, st, pdl, off, cnt);
   if (rc) return rc;
-  return run_outproj(dims, a16, W_fold, y, ws, L, st, pdl, append ? seq_lens : nullptr);
+  return run_outproj(dims, a16, W_fold, y, ws, L, st, pdl, append ? seq_lens : nullptr,
+                     cnt + L.n_att_cnt);
 }
 
 int basiskv_read_device_status(void* stream, uint32_t* flags) {

@@ -48,6 +48,7 @@ struct AttendGeom {
   int stage_bytes;
   int stages;
   int ps_off, red_off;  // scratch after the ring, double-buffered by item parity
+  int comb_off;         // fused merge: split weights and masses [2][nsplit][G] + a flag
   int smem_bytes;
 };
 
@@ -79,7 +80,8 @@ __global__ void __launch_bounds__(kAttThreads, kAttCtasPerSm)
                   AttendArgs a, AttendGeom geo) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1k(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + geo.smem_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + geo.smem_bytes +
+                                               (a.cnt ? ((2 * a.nsplit * G * 4 + 15) & ~15) : 0));
   uint64_t* empty = full + geo.stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + geo.stages);
   float* psb = reinterpret_cast<float*>(smem + geo.ps_off);    // [2][G][64] weights
@@ -201,20 +203,114 @@ __global__ void __launch_bounds__(kAttThreads, kAttCtasPerSm)
   const uint32_t zmask = geo.zmask;
   int it = 0;
   const int count = (int)(i_end - i_begin);
+  // Fused merge (a.cnt set): at the end of each run of consecutive items of
+  // one group, the CTA adds how many of the group's splits it wrote to the
+  // group's arrival counter; the CTA that completes the count merges the
+  // splits into a_lat / a_bf16.  One atomic per run instead of per item.
+  float* wsp = reinterpret_cast<float*>(smem + geo.comb_off);  // [nitems][G] weights
+  float* lsp = wsp + a.nsplit * G;                             // [nitems][G] masses
+  volatile int* flag = reinterpret_cast<volatile int*>(lsp + a.nsplit * G);
+  int seg_first = 0;  // first split of the current run
+  int n = 0, bg = 0, j = 0;
+  bool ready = false;
+  auto arrive = [&](int T) {
+    if (!a.cnt || (n + 1 < count && j + 1 < a.nsplit)) return;  // not the end of a run
+    const int Pb = T > 0 ? (T + S - 1) >> logS : 0;
+    const int nitems = (min(a.top_k, Pb) + geo.ppi - 1) / geo.ppi;
+    const int mine = min(j + 1, nitems) - seg_first;
+    named_bar_sync(1, kAttConsumers);  // the run's partial results are written
+    if (tid == 0) {
+      int last = 0;
+      if (ready && mine > 0) {
+        __threadfence();
+        last = atomicAdd(&a.cnt[bg], mine) + mine == nitems;
+      }
+      *flag = last;
+    }
+    named_bar_sync(1, kAttConsumers);
+    if (!*flag) return;
+    __threadfence();
+    const float* part = a.partial + (size_t)bg * a.nsplit * G * (r_v + 2);
+    // split statistics, all (split, head) pairs at once
+    for (int i = tid; i < nitems * G; i += kAttConsumers) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(part + (size_t)i * (r_v + 2)));
+      wsp[i] = ml.x;
+      lsp[i] = ml.y;
+    }
+    named_bar_sync(1, kAttConsumers);
+    // weights 2^(m_j - M) / L: warp w merges heads w, w + 4, ...
+    for (int h = warp; h < G; h += kAttConsumerWarps) {
+      float M = -INFINITY;
+      for (int it2 = lane; it2 < nitems; it2 += 32) M = fmaxf(M, wsp[it2 * G + h]);
+      M = warp_max(M);
+      float L = 0.f;
+      for (int it2 = lane; it2 < nitems; it2 += 32) {
+        const float w = exp2f(wsp[it2 * G + h] - M);
+        wsp[it2 * G + h] = w;
+        L += lsp[it2 * G + h] * w;
+      }
+      L = warp_sum(L);
+      const float invL = L > 0.f ? 1.f / L : 0.f;
+      for (int it2 = lane; it2 < nitems; it2 += 32) wsp[it2 * G + h] *= invL;
+    }
+    named_bar_sync(1, kAttConsumers);
+    // outputs, two latent channels per thread, sixteen splits in flight
+    const int b = bg / a.Hkv, g = bg - b * a.Hkv;
+    const size_t istride = (size_t)G * (r_v + 2);
+    for (int o2 = tid; o2 < G * r_v / 2; o2 += kAttConsumers) {
+      const int h = (2 * o2) / r_v, c = 2 * o2 - h * r_v;
+      const float* pc = part + (size_t)h * (r_v + 2) + 2 + c;
+      float vx = 0.f, vy = 0.f;
+      for (int i0 = 0; i0 < nitems; i0 += 16) {
+        float2 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          v[u] = i0 + u < nitems ? __ldcg(reinterpret_cast<const float2*>(pc + (i0 + u) * istride))
+                                 : make_float2(0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float w = i0 + u < nitems ? wsp[(i0 + u) * G + h] : 0.f;
+          vx = fmaf(v[u].x, w, vx);
+          vy = fmaf(v[u].y, w, vy);
+        }
+      }
+      const size_t oi = ((size_t)b * a.Hq + g * G + h) * r_v + c;
+      if (a.a_lat) {
+        a.a_lat[oi] = vx;
+        a.a_lat[oi + 1] = vy;
+      }
+      if (a.a_bf16)
+        *reinterpret_cast<uint32_t*>(a.a_bf16 + oi) =
+            (uint32_t)f_to_bf16(vx) | ((uint32_t)f_to_bf16(vy) << 16);
+    }
+    if (tid == 0) a.cnt[bg] = 0;  // ready for the next call
+    named_bar_sync(1, kAttConsumers);  // wsp is reused by the next merge
+  };
   ItemCursor cur;
   cur.init(i_begin, a.nsplit, a.Hkv);
-  for (int n = 0; n < count; ++n, cur.next(a.nsplit, a.Hkv)) {
-    const int bg = cur.bg, j = cur.j;
+  for (n = 0; n < count; ++n, cur.next(a.nsplit, a.Hkv)) {
+    bg = cur.bg;
+    j = cur.j;
+    if (n == 0 || j == 0) seg_first = j;
     const int s = it % geo.stages;
     const int my = it++;
     // On a timeout every later wait fails at once; the item is skipped but
     // the barrier sequence below is kept, so all consumer warps stay in step.
-    const bool ready = mbar_wait_or_abort(&full[s], (my / geo.stages) & 1, a.status, abort_flag);
+    ready = mbar_wait_or_abort(&full[s], (my / geo.stages) & 1, a.status, abort_flag);
     const uint8_t* st = smem + (size_t)s * geo.stage_bytes;
     const int* meta = reinterpret_cast<const int*>(st + geo.meta_off);
     if (ready && meta[0] < 0) {  // empty split: nothing to attend, nothing to write
+      const int T_empty = meta[31];  // read before the stage is handed back
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
+      if (a.cnt && j == 0) {  // an empty sequence: its fused merge output is zero
+        const size_t o0 = ((size_t)(bg / a.Hkv) * a.Hq + (bg % a.Hkv) * G) * r_v;
+        for (int o = tid; o < G * r_v; o += kAttConsumers) {
+          if (a.a_lat) a.a_lat[o0 + o] = 0.f;
+          if (a.a_bf16) a.a_bf16[o0 + o] = 0;
+        }
+      }
+      arrive(T_empty);
       continue;
     }
     float* red = redb + (my & 1) * 2 * kAttConsumerWarps * G;  // scratch by item parity
@@ -362,6 +458,7 @@ __global__ void __launch_bounds__(kAttThreads, kAttCtasPerSm)
       out[tid * (r_v + 2)] = m;
       out[tid * (r_v + 2) + 1] = l;
     }
+    arrive(T);
   }
 }
 
@@ -431,6 +528,11 @@ __global__ void combine_kernel(CombineArgs a) {
 
 int round1k(int x) { return (x + 1023) / 1024 * 1024; }
 
+// Shared-memory bytes of the fused merge (0 when it is off).
+size_t attend_merge_bytes(const AttendArgs& a) {
+  return a.cnt ? ((size_t)2 * a.nsplit * a.G * 4 + 15) / 16 * 16 : 0;
+}
+
 AttendGeom attend_geometry(int G, int d, int r_v, int S, int wz) {
   AttendGeom g{};
   g.ppi = kAttTokens / S;
@@ -454,14 +556,16 @@ AttendGeom attend_geometry(int G, int d, int r_v, int S, int wz) {
   if (g.stages > 6) g.stages = 6;
   g.ps_off = g.stages * g.stage_bytes;
   g.red_off = g.ps_off + 2 * G * kAttTokens * 4;
-  g.smem_bytes = (g.red_off + 2 * 2 * kAttConsumerWarps * G * 4 + 15) / 16 * 16;
+  g.comb_off = g.red_off + 2 * 2 * kAttConsumerWarps * G * 4;
+  g.smem_bytes = (g.comb_off + 16 + 15) / 16 * 16;  // + merge scratch, added at launch
   return g;
 }
 
 template <int G, int D>
 cudaError_t launch_attend_g(const AttendArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmZ,
                             const AttendGeom& geo, cudaStream_t st, bool pdl) {
-  const size_t smem = (size_t)geo.smem_bytes + 2 * geo.stages * 8 + 16 + 1024;
+  const size_t smem = (size_t)geo.smem_bytes + attend_merge_bytes(a) + 2 * geo.stages * 8 + 16 +
+                      1024;
   cudaError_t e = cudaFuncSetAttribute(attend_kernel<G, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

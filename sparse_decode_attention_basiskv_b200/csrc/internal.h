@@ -70,6 +70,11 @@ struct FoldQArgs {
   int B, Hq, Hkv, d, r_v, r_k;
 };
 cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl);
+// First launch of a fused decode step: the query fold and (when a.k_new is
+// set) the one-token append run side by side; n_counters ints at `counters`
+// are zeroed.
+cudaError_t launch_decode_prologue(const FoldQArgs& f, const AppendArgs& a, int* counters,
+                                   int n_counters, cudaStream_t st, bool pdl);
 
 struct RouteArgs {
   const float* qt;  // [B][Hq][r_v + r_k]
@@ -104,6 +109,12 @@ struct AttendArgs {
   int len_offset;
   float scale_log2;  // log2(e) / sqrt(d)
   unsigned int* status;
+  // Fused merge of the splits (when cnt is set): per (sequence, KV head) an
+  // arrival counter, zeroed before the launch; the CTA that writes a group's
+  // last split merges them into a_lat / a_bf16.
+  int* cnt;
+  float* a_lat;
+  uint16_t* a_bf16;
 };
 int attend_pages_per_split(int S);
 cudaError_t launch_attend(const AttendArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmZ,
@@ -130,6 +141,10 @@ struct OutprojArgs {
   // earlier kernel of the step has finished reading the lengths.
   int32_t* bump_lens;
   int bump_n, bump_cap;
+  // Fused K-split reduction (when cnt is set and ksplit > 1): per M tile an
+  // arrival counter, zeroed before the launch; the tile's last CTA sums the
+  // partials and writes y.
+  int* cnt;
 };
 // Chooses the K split for a given problem.
 int outproj_ksplit(int H, int K, int B);

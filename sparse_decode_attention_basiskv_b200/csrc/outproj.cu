@@ -189,6 +189,54 @@ __global__ void __launch_bounds__(kOpThreads, 1)
       }
     }
   }
+  if (a.ksplit > 1 && a.cnt) {
+    // arrival: the last CTA of this M tile sums the K-split partials into y
+    __shared__ int last;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last = atomicAdd(&a.cnt[blockIdx.x], 1) == a.ksplit - 1;
+    __syncthreads();
+    if (last) {
+      __threadfence();
+      // four rows of one batch column per float4; up to three groups per
+      // thread, every load of a split issued before any sum needs it
+      const int ngrp = kOpBM / 4 * a.B;
+      const size_t kstride = (size_t)a.B * a.H;
+      for (int i0 = tid; i0 < ngrp; i0 += 3 * kOpThreads) {
+        float4 acc[3];
+        const float* src[3];
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+          const int i = min(i0 + u * kOpThreads, ngrp - 1);
+          const int n = i / (kOpBM / 4), r4 = (i - n * (kOpBM / 4)) * 4;
+          src[u] = a.partial + (size_t)n * a.H + m0 + r4;
+          acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll 4
+        for (int k = 0; k < a.ksplit; ++k) {  // splits summed in order, as the reduce kernel does
+          float4 v[3];
+#pragma unroll
+          for (int u = 0; u < 3; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(src[u] + k * kstride));
+#pragma unroll
+          for (int u = 0; u < 3; ++u) {
+            acc[u].x += v[u].x;
+            acc[u].y += v[u].y;
+            acc[u].z += v[u].z;
+            acc[u].w += v[u].w;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+          if (i0 + u * kOpThreads >= ngrp) break;
+          uint16_t* dst = a.y + (src[u] - a.partial);
+          *reinterpret_cast<uint2*>(dst) =
+              make_uint2((uint32_t)f_to_bf16(acc[u].x) | ((uint32_t)f_to_bf16(acc[u].y) << 16),
+                         (uint32_t)f_to_bf16(acc[u].z) | ((uint32_t)f_to_bf16(acc[u].w) << 16));
+        }
+      }
+      if (tid == 0) a.cnt[blockIdx.x] = 0;  // ready for the next call
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -253,7 +301,7 @@ cudaError_t launch_outproj_bn(const OutprojArgs& a, const CUtensorMap& tmW,
   if (e != cudaSuccess) return e;
   dim3 grid(a.H / kOpBM, a.ksplit);
   e = launch_k(outproj_kernel<BN>, grid, dim3(kOpThreads), smem, st, pdl, tmW, tmA, a);
-  if (e != cudaSuccess || a.ksplit == 1) return e;
+  if (e != cudaSuccess || a.ksplit == 1 || a.cnt) return e;
   const size_t n = (size_t)a.B * a.H;
   return launch_k(ksplit_reduce_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, pdl,
                   (const float*)a.partial, a.y, a.ksplit, n);

@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "launch.cuh"
+#include "step_blocks.cuh"
 
 namespace basiskv {
 
@@ -28,63 +29,9 @@ namespace {
 // ----------------------------------------------------------- query folding
 // qt[b][h][j]       = sum_i P_K[g][j][i] q[b][h][i]          j < r_v
 // qt[b][h][r_v + c] = sum_i q[b][h][i] U_K[g][i][c]           c < r_k
-constexpr int kFoldThreads = 128;  // 32 outputs x 4 quarters of the head dim
-
-// CTA = (sequence, KV head, 32 consecutive outputs j).  Warp w sums the
-// products over the w-th quarter of the head dimension for every head of
-// the group; the four partial sums meet in shared memory.  All loads of a
-// thread are independent, so the kernel costs about one memory round trip.
 __global__ void __launch_bounds__(kFoldThreads) fold_query_kernel(FoldQArgs a) {
-  const int bg = blockIdx.x, b = bg / a.Hkv, g = bg % a.Hkv;
-  const int tid = threadIdx.x, lane = tid & 31, quarter = tid >> 5;
-  const int G = a.Hq / a.Hkv, rq = a.r_v + a.r_k, d = a.d;
-  const int j = blockIdx.y * 32 + lane;
-  const int i0 = quarter * (d / 4), n = d / 4;
   extern __shared__ float fsm[];
-  float* qs = fsm;               // [G][d]
-  float* part = fsm + G * d;     // [4][G][32]
-  pdl_wait();
-  for (int i = tid; i < G * d; i += kFoldThreads)
-    qs[i] = bf16_to_f(a.q[((size_t)b * a.Hq + g * G) * d + i]);
-  __syncthreads();
-  float acc[8];
-#pragma unroll
-  for (int h = 0; h < 8; ++h) acc[h] = 0.f;
-  if (j < a.r_v) {  // row j of P_K, this quarter: n contiguous bf16 (16-byte aligned)
-    const uint4* row = reinterpret_cast<const uint4*>(a.P_K + ((size_t)g * a.r_v + j) * d + i0);
-    for (int c = 0; c < n / 8; ++c) {
-      const uint4 w = row[c];
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float p0 = bf16lo(ws[e]), p1 = bf16hi(ws[e]);
-        const int ii = i0 + c * 8 + 2 * e;
-#pragma unroll
-        for (int h = 0; h < 8; ++h)
-          if (h < G) acc[h] = fmaf(p1, qs[h * d + ii + 1], fmaf(p0, qs[h * d + ii], acc[h]));
-      }
-    }
-  } else if (j < rq) {  // column j - r_v of U_K, this quarter (coalesced across lanes)
-    const uint16_t* col = a.U_K + (size_t)g * d * a.r_k + (j - a.r_v);
-    for (int i = i0; i < i0 + n; ++i) {
-      const float u = bf16_to_f(col[(size_t)i * a.r_k]);
-#pragma unroll
-      for (int h = 0; h < 8; ++h)
-        if (h < G) acc[h] = fmaf(u, qs[h * d + i], acc[h]);
-    }
-  }
-#pragma unroll
-  for (int h = 0; h < 8; ++h)
-    if (h < G) part[(quarter * G + h) * 32 + lane] = acc[h];
-  __syncthreads();
-  for (int o = tid; o < G * 32; o += kFoldThreads) {
-    const int h = o / 32, jj = blockIdx.y * 32 + (o % 32);
-    if (jj < rq) {
-      const float v = part[(0 * G + h) * 32 + o % 32] + part[(1 * G + h) * 32 + o % 32] +
-                      part[(2 * G + h) * 32 + o % 32] + part[(3 * G + h) * 32 + o % 32];
-      a.qt[((size_t)b * a.Hq + g * G + h) * rq + jj] = v;
-    }
-  }
+  fold_query_block(a, blockIdx.x, blockIdx.y, fsm);
 }
 
 // ------------------------------------------------------------ page scoring
@@ -711,7 +658,7 @@ cudaError_t launch_route_rs(const RouteArgs& a, const CUtensorMap& tmZ, const CU
 
 cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl) {
   const int G = a.Hq / a.Hkv;
-  const size_t smem = (size_t)(G * a.d + 4 * G * 32) * sizeof(float);
+  const size_t smem = fold_block_smem(G, a.d);
   dim3 grid(a.B * a.Hkv, (a.r_v + a.r_k + 31) / 32);
   return launch_k(fold_query_kernel, grid, dim3(kFoldThreads), smem, st, pdl, a);
 }

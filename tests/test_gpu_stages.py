@@ -146,6 +146,27 @@ def test_ragged_lengths_and_degenerate_pages():
     assert sel[0, 0, 0].item() == 0 and (sel[0, 0, 1:] == -1).all()  # one page
 
 
+def test_empty_sequence_gives_zero_output():
+    """A sequence of length 0 (no append) has no token to attend: its latent
+    output, hence its y row, is zero, also after an earlier step left other
+    values in the workspace; the other sequence is unaffected."""
+    wl = synth.with_sizes(synth.LLAMA8B_T4K, B=2, T=600, top_k=16)
+    pb, layer = gpu_layer(wl, seq_lens=[37, 600])
+    layer.decode(pb.q, max_seq_len=600)
+    layer.seq_lens[0] = 0
+    y = torch.full((wl.B, wl.hidden), float("nan"), dtype=torch.bfloat16, device="cuda")
+    layer.decode(pb.q, max_seq_len=600, y=y)
+    status_clean()
+    assert (y[0] == 0).all()
+    f = factors_np(pb)
+    W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
+    c = {k: np64(v[1]) for k, v in pb.cache.items()}
+    out = O.decode_sequence(np64(pb.q[1]), c["K"], c["Z"], c["E"], 600, wl.page_size,
+                            wl.top_k, f["P_K"], f["U_K"], W)
+    if not out["near_tie"].any():
+        assert_within(np64(y[1]), out["y"], Y_REL, Y_ABS)
+
+
 def test_dense_when_top_k_covers_context():
     """top_k >= P: every page is attended, so the result is plain attention."""
     wl = synth.with_sizes(synth.TINY, top_k=40)  # 32 pages
