@@ -306,6 +306,8 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   }
   RouteArgs r{};
   r.qt = qt;
+  r.Z = Z_cache;
+  r.E = E_cache;
   r.seq_lens = seq_lens;
   r.block_table = block_table;
   r.scores = scores;

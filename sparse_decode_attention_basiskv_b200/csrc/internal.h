@@ -78,6 +78,8 @@ cudaError_t launch_decode_prologue(const FoldQArgs& f, const AppendArgs& a, int*
 
 struct RouteArgs {
   const float* qt;  // [B][Hq][r_v + r_k]
+  const uint16_t* Z;  // Z cache [num_phys][Hkv][S][r_v] (plain-load kernel)
+  const uint16_t* E;  // E cache [num_phys][Hkv][S][r_k]
   const int32_t* seq_lens;
   const int32_t* block_table;
   float* scores;  // [B][Hkv][max_pages]
