@@ -181,7 +181,10 @@ WsLayout ws_layout(const basiskv_dims* d, int top_k) {
   w.ppi = attend_pages_per_split(d->page_size);
   w.nsplit = (top_k + w.ppi - 1) / w.ppi;
   w.partial = off;
-  off += align256((size_t)d->B * d->Hkv * w.nsplit * G * (d->r_v + 2) * 4);
+  size_t slots = (size_t)d->B * d->Hkv * w.nsplit;
+  if (attend_mma_supported(G, d->d, d->r_v, d->page_size))
+    slots = (size_t)attend_mma_slots(d->B, d->Hkv);
+  off += align256(slots * G * (d->r_v + 2) * 4);
   w.a_f32 = off;
   off += align256((size_t)d->B * d->Hq * d->r_v * 4);
   w.a_bf16 = off;
@@ -342,6 +345,8 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
     return BASISKV_ERR_CUDA;
   AttendArgs a{};
   a.q = q;
+  a.K = K_cache;
+  a.Z = Z_cache;
   a.seq_lens = seq_lens;
   a.block_table = block_table;
   a.sel = sel;
@@ -361,6 +366,17 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
   a.len_offset = len_offset;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d->d));
   a.status = status;
+  if (attend_mma_supported(a.G, a.d, a.r_v, a.S)) {
+    if (!cnt) {  // a standalone call: the arrival counters start from zero here
+      cnt = reinterpret_cast<int*>(ws + L.counters);
+      if (cudaMemsetAsync(cnt, 0, (size_t)L.n_att_cnt * 4, st) != cudaSuccess)
+        return BASISKV_ERR_LAUNCH_FAILED;
+    }
+    a.cnt = cnt;
+    a.a_lat = a_lat;
+    a.a_bf16 = a_bf16;
+    return launch_status(launch_attend_mma(a, st, pdl));
+  }
   // Fused merge of the splits when its shared-memory scratch stays small.
   if (cnt && (size_t)2 * L.nsplit * a.G * 4 <= 4096) {
     a.cnt = cnt;

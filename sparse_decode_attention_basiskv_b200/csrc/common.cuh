@@ -227,6 +227,15 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, u
                : "memory");
 }
 
+// Transpose of an 8x8 b16 matrix held one row fragment per lane (lane l:
+// row l/4, columns 2(l%4) and 2(l%4)+1); returns the same fragment of the
+// transpose.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
+
 // Splits two fp32 values into bf16 pairs hi (rounded) and lo (the rounded
 // remainder): x = hi + lo to about 16 significant bits.
 __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {

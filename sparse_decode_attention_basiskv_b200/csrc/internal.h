@@ -103,6 +103,8 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
 // ------------------------------------------------------------------ attend
 struct AttendArgs {
   const uint16_t* q;
+  const uint16_t* K;  // exact-Key cache [num_phys][Hkv][S][d] (plain-load kernel)
+  const uint16_t* Z;  // Value-latent cache [num_phys][Hkv][S][r_v]
   const int32_t* seq_lens;
   const int32_t* block_table;
   const int32_t* sel;
@@ -119,6 +121,12 @@ struct AttendArgs {
   uint16_t* a_bf16;
 };
 int attend_pages_per_split(int S);
+// Plain-load tensor-core attention with its own merge (needs a.cnt zeroed,
+// a.partial of attend_mma_slots(B, Hkv) * G * (r_v + 2) floats); returns
+// cudaErrorNotSupported for shapes it does not cover.
+bool attend_mma_supported(int G, int d, int r_v, int S);
+int attend_mma_slots(int B, int Hkv);
+cudaError_t launch_attend_mma(const AttendArgs& a, cudaStream_t st, bool pdl);
 cudaError_t launch_attend(const AttendArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmZ,
                           int wz, cudaStream_t st, bool pdl);
 
