@@ -163,7 +163,7 @@ int check_len_topk(const basiskv_dims* d, int top_k, int max_seq_len) {
 }
 
 struct WsLayout {
-  size_t qt, scores, sel, partial, a_f32, a_bf16, op_part, w_app, counters, total;
+  size_t qt, scores, sel, selp, partial, a_f32, a_bf16, op_part, w_app, counters, total;
   int n_att_cnt, n_op_cnt;
   int nsplit, ppi;
 };
@@ -177,6 +177,8 @@ WsLayout ws_layout(const basiskv_dims* d, int top_k) {
   w.scores = off;
   off += align256((size_t)d->B * d->Hkv * d->max_pages_per_seq * 4);
   w.sel = off;
+  off += align256((size_t)d->B * d->Hkv * top_k * 4);
+  w.selp = off;  // physical pages of the selection
   off += align256((size_t)d->B * d->Hkv * top_k * 4);
   w.ppi = attend_pages_per_split(d->page_size);
   w.nsplit = (top_k + w.ppi - 1) / w.ppi;
@@ -328,7 +330,8 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   rc = launch_status(launch_route_scores(r, tmZ, tmE, wz, we, st, pdl));
   if (rc) return rc;
   SelectArgs s{scores, seq_lens, sel, d->B, d->Hkv, d->page_size, d->max_pages_per_seq, top_k,
-               max_seq_len, len_offset};
+               max_seq_len, len_offset, block_table,
+               reinterpret_cast<int32_t*>(ws + L.selp)};
   return launch_status(launch_select(s, st, pdl));
 }
 
@@ -336,7 +339,7 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
                const int32_t* block_table, const basiskv_bf16* K_cache,
                const basiskv_bf16* Z_cache, const int32_t* sel, int top_k, float* a_lat,
                uint16_t* a_bf16, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl,
-               int len_offset = 0, int* cnt = nullptr) {
+               int len_offset = 0, int* cnt = nullptr, const int32_t* sel_phys = nullptr) {
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   const int wz = z_box_cols(d->r_v);
@@ -350,6 +353,7 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
   a.seq_lens = seq_lens;
   a.block_table = block_table;
   a.sel = sel;
+  a.sel_phys = sel_phys;
   a.partial = reinterpret_cast<float*>(ws + L.partial);
   a.B = d->B;
   a.Hq = d->Hq;
@@ -640,7 +644,7 @@ int basiskv_decode(const basiskv_dims* dims, const basiskv_bf16* q, const basisk
   if (rc) return rc;
   uint16_t* a16 = reinterpret_cast<uint16_t*>(ws + L.a_bf16);
   rc = run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel_buf, top_k, nullptr, a16,
-                  ws, L, st, pdl, off, cnt);
+                  ws, L, st, pdl, off, cnt, reinterpret_cast<const int32_t*>(ws + L.selp));
   if (rc) return rc;
   return run_outproj(dims, a16, W_fold, y, ws, L, st, pdl, append ? seq_lens : nullptr,
                      cnt + L.n_att_cnt);

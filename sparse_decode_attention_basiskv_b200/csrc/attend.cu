@@ -221,15 +221,11 @@ __global__ void __launch_bounds__(kAttThreads, kAttCtasPerSm)
     named_bar_sync(1, kAttConsumers);  // the run's partial results are written
     if (tid == 0) {
       int last = 0;
-      if (ready && mine > 0) {
-        __threadfence();
-        last = atomicAdd(&a.cnt[bg], mine) + mine == nitems;
-      }
+      if (ready && mine > 0) last = arrive_acq_rel(&a.cnt[bg], mine) + mine == nitems;
       *flag = last;
     }
     named_bar_sync(1, kAttConsumers);
     if (!*flag) return;
-    __threadfence();
     const float* part = a.partial + (size_t)bg * a.nsplit * G * (r_v + 2);
     // split statistics, all (split, head) pairs at once
     for (int i = tid; i < nitems * G; i += kAttConsumers) {
@@ -558,6 +554,7 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
   extern __shared__ float am_smem[];
   float* wacc = am_smem;                        // [warp][G][RV] latent sums of the run
   float* wml = am_smem + kAmWarps * G * RV;     // [warp][16]: m of heads 0-7, then l
+  uint4* qs = reinterpret_cast<uint4*>(wml + kAmWarps * 16);  // [NKC][lane] query fragments
   __shared__ int s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, lr = lane >> 2, lc = lane & 3;
   const int S = a.S, TP = S >> 4;
@@ -583,12 +580,15 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
     const int nsel = min(a.top_k, (T + S - 1) / S);
     const long valid_end = bg0 + (long)nsel * TP;  // units past it have no page
 
-    uint4 qf[NKC];  // B fragments: lane (r, c) holds head r, columns 32k + 8c .. +7
-#pragma unroll
-    for (int k = 0; k < NKC; ++k)
-      qf[k] = lr < G ? __ldg(reinterpret_cast<const uint4*>(
-                           a.q + ((size_t)b * a.Hq + g * G + lr) * D + 32 * k + 8 * lc))
-                     : make_uint4(0u, 0u, 0u, 0u);
+    // the group's queries as B fragments, shared by the CTA's warps: entry
+    // [k][lane (r, c)] holds head r, columns 32k + 8c .. +7 (zero past G)
+    for (int i = tid; i < NKC * 32; i += kAmThreads) {
+      const int k = i >> 5, r = (i & 31) >> 2, cc = i & 3;
+      qs[i] = r < G ? __ldg(reinterpret_cast<const uint4*>(
+                          a.q + ((size_t)b * a.Hq + g * G + r) * D + 32 * k + 8 * cc))
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2c, 2c + 1
     float acc[NZC][2][4];
 #pragma unroll
@@ -596,36 +596,90 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
 #pragma unroll
       for (int e = 0; e < 2; ++e) acc[c][e][0] = acc[c][e][1] = acc[c][e][2] = acc[c][e][3] = 0.f;
 
-    for (long u = seg + warp; u < seg_end && u < valid_end; u += kAmWarps) {
-      const int ui = (int)(u - bg0), k = ui / TP, tau = ui - k * TP;
-      const int lp = __ldg(a.sel + (size_t)bg * a.top_k + k);
-      if (lp < 0) continue;
-      int pp = lp < a.max_pages ? __ldg(a.block_table + (size_t)b * a.max_pages + lp) : -1;
-      if (pp < 0 || pp >= a.num_phys) {
-        if (lane == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
-        pp = 0;  // keep going; the output is flagged garbage
+    // Page ids of the warp's units in this run, fetched 32 at a time (lane i:
+    // unit seg + warp + 8 (n0 + i)) with the physical page from the
+    // selection's companion list when there is one (one round trip), else
+    // through the block table.
+    const long u_first = seg + warp;
+    const long u_stop = seg_end < valid_end ? seg_end : valid_end;
+    const int count =
+        u_first < u_stop ? (int)((u_stop - u_first + kAmWarps - 1) / kAmWarps) : 0;
+    int lp_l = -1, pp_l = -1, n0 = 0;
+    auto fetch_ids = [&](int base) {
+      const long uu = u_first + (long)kAmWarps * (base + lane);
+      lp_l = -1;
+      pp_l = -1;
+      if (uu < u_stop) {
+        const size_t si = (size_t)bg * a.top_k + (int)(uu - bg0) / TP;
+        lp_l = __ldg(a.sel + si);
+        if (a.sel_phys)
+          pp_l = __ldg(a.sel_phys + si);
+        else if (lp_l >= 0 && lp_l < a.max_pages)
+          pp_l = __ldg(a.block_table + (size_t)b * a.max_pages + lp_l);
       }
-      const size_t row = ((size_t)pp * a.Hkv + g) * S + 16 * tau + lr;
-      uint4 kx[NKC][2], zx[NZC][2];
+    };
+    // ids of unit nn (warp-uniform); a missing entry becomes a fully masked
+    // unit on page 0, a bad page is flagged and read as page 0
+    auto unit_ids = [&](int nn, int& lp, int& pp) {
+      if (nn - n0 >= 32) {
+        n0 = nn;
+        fetch_ids(n0);
+      }
+      lp = __shfl_sync(0xffffffffu, lp_l, nn - n0);
+      pp = __shfl_sync(0xffffffffu, pp_l, nn - n0);
+      if (lp < 0) {
+        pp = 0;
+      } else if (pp < 0 || pp >= a.num_phys) {
+        if (lane == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
+        pp = 0;
+      }
+    };
+    auto unit_row = [&](int nn, int pp) -> size_t {
+      const int tau = (int)(u_first + (long)kAmWarps * nn - bg0) % TP;
+      return ((size_t)pp * a.Hkv + g) * S + 16 * tau + lr;
+    };
+    uint4 kx[NKC][2], zx[NZC][2];
+    auto load_k = [&](size_t row) {
 #pragma unroll
       for (int c = 0; c < NKC; ++c) {
         kx[c][0] = ldg_stream(a.K + row * D + 32 * c + 8 * lc);
         kx[c][1] = ldg_stream(a.K + (row + 8) * D + 32 * c + 8 * lc);
       }
+    };
+    auto load_z = [&](size_t row) {
 #pragma unroll
       for (int c = 0; c < NZC; ++c) {
         zx[c][0] = ldg_stream(a.Z + row * RV + 32 * c + 8 * lc);
         zx[c][1] = ldg_stream(a.Z + (row + 8) * RV + 32 * c + 8 * lc);
       }
+    };
+    int lp_c = -1, pp_c = 0;
+    if (count > 0) {
+      fetch_ids(0);
+      unit_ids(0, lp_c, pp_c);
+      const size_t row0 = unit_row(0, pp_c);
+      load_k(row0);
+      load_z(row0);
+    }
+    // Unit n computes while unit n + 1 loads: its Keys are requested as soon
+    // as QK has consumed the current ones, its latents after PV.
+    for (int n = 0; n < count; ++n) {
+      const int tau = (int)(u_first + (long)kAmWarps * n - bg0) % TP;
+      const bool more = n + 1 < count;
+      int lp_n = -1, pp_n = 0;
+      if (more) unit_ids(n + 1, lp_n, pp_n);
+      const size_t row_n = more ? unit_row(n + 1, pp_n) : 0;
       // s = [tokens r, r + 8] x [heads 2c, 2c + 1]
       float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < NKC; ++c) {
-        mma_bf16_16816(s, kx[c][0].x, kx[c][1].x, kx[c][0].y, kx[c][1].y, qf[c].x, qf[c].y);
-        mma_bf16_16816(s, kx[c][0].z, kx[c][1].z, kx[c][0].w, kx[c][1].w, qf[c].z, qf[c].w);
+        const uint4 qf = qs[c * 32 + lane];
+        mma_bf16_16816(s, kx[c][0].x, kx[c][1].x, kx[c][0].y, kx[c][1].y, qf.x, qf.y);
+        mma_bf16_16816(s, kx[c][0].z, kx[c][1].z, kx[c][0].w, kx[c][1].w, qf.z, qf.w);
       }
-      const int pos = lp * S + 16 * tau + lr;
-      const bool v0 = pos < T, v1 = pos + 8 < T;
+      if (more) load_k(row_n);
+      const int pos = lp_c * S + 16 * tau + lr;
+      const bool v0 = lp_c >= 0 && pos < T, v1 = lp_c >= 0 && pos + 8 < T;
       const float x00 = v0 ? s[0] * a.scale_log2 : -INFINITY;
       const float x01 = v0 ? s[1] * a.scale_log2 : -INFINITY;
       const float x10 = v1 ? s[2] * a.scale_log2 : -INFINITY;
@@ -680,7 +734,11 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
           mma_bf16_16816(acc[c][e], t0[2 * e], t0[2 * e + 1], t1[2 * e], t1[2 * e + 1], bl0, bl1);
         }
       }
+      if (more) load_z(row_n);
+      lp_c = lp_n;
+      pp_c = pp_n;
     }
+    (void)pp_c;
 
     // ---- the run's warps meet: per-warp state to shared memory
 #pragma unroll
@@ -747,25 +805,27 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
     __syncthreads();  // slot written; the shared state is free again
     if (has) {
       const int c0 = cta_of(bg0), c1 = cta_of(valid_end - 1);
-      if (tid == 0) {
-        __threadfence();
-        s_last = atomicAdd(&a.cnt[bg], 1) + 1 == c1 - c0 + 1;
-      }
+      if (tid == 0) s_last = arrive_acq_rel(&a.cnt[bg], 1) + 1 == c1 - c0 + 1;
       __syncthreads();
       if (s_last) {  // every run of the group is written: merge them
-        __threadfence();
         for (int o = tid; o < G * RV; o += kAmThreads) {
           const int h = o / RV, j = o - h * RV;
-          float M = -INFINITY;
-          for (int c = c0; c <= c1; ++c)
-            M = fmaxf(M, __ldcg(a.partial + (size_t)(c + bg) * G * RS + h * RS));
-          float L = 0.f, A = 0.f;
+          // one pass with a running maximum: every slot's loads are independent
+          float M = -INFINITY, L = 0.f, A = 0.f;
+#pragma unroll 4
           for (int c = c0; c <= c1; ++c) {
             const float* sl = a.partial + (size_t)(c + bg) * G * RS + h * RS;
-            const float mc = __ldcg(sl);
-            const float f = mc == -INFINITY ? 0.f : exp2f(mc - M);
-            L = fmaf(__ldcg(sl + 1), f, L);
-            A = fmaf(__ldcg(sl + 2 + j), f, A);
+            const float mc = __ldcg(sl), lcv = __ldcg(sl + 1), ac = __ldcg(sl + 2 + j);
+            if (mc == -INFINITY) continue;
+            if (mc > M) {
+              const float r = exp2f(M - mc);  // 0 while M is -inf
+              L *= r;
+              A *= r;
+              M = mc;
+            }
+            const float f = exp2f(mc - M);
+            L = fmaf(lcv, f, L);
+            A = fmaf(ac, f, A);
           }
           const float v = L > 0.f ? A / L : 0.f;
           const size_t oi = ((size_t)b * a.Hq + g * G + h) * RV + j;
@@ -786,7 +846,7 @@ cudaError_t launch_attend_mma_t(const AttendArgs& a, cudaStream_t st, bool pdl) 
   if (grid > kAmMaxCtas) grid = kAmMaxCtas;
   if (grid > units) grid = units;  // every CTA gets at least one unit
   if (grid < 1) return cudaSuccess;
-  const size_t smem = (size_t)kAmWarps * (G * RV + 16) * sizeof(float);
+  const size_t smem = (size_t)kAmWarps * (G * RV + 16) * sizeof(float) + (D / 32) * 32 * 16;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(attend_mma_kernel<G, D, RV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -256,6 +256,19 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return r;
 }
 
+// Arrival on a gpu-scope counter: atomic add with release semantics for the
+// calling thread's prior writes and those of its block ordered before it by
+// a barrier, and acquire semantics for what earlier arrivers released.
+// Returns the old value.
+__device__ __forceinline__ int arrive_acq_rel(int* counter, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(counter), "r"(v)
+               : "memory");
+  return old;
+}
+
 // ------------------------------------------------------------- PDL control
 __device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");

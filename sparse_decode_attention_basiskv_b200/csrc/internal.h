@@ -97,6 +97,10 @@ struct SelectArgs {
   int32_t* sel;  // [B][Hkv][top_k]
   int B, Hkv, S, max_pages, top_k, max_seq_len;
   int len_offset;
+  // Optional: the physical page of each selected entry (block-table lookup
+  // done here, so the attention kernel reads page ids in one round trip).
+  const int32_t* block_table;
+  int32_t* sel_phys;  // [B][Hkv][top_k] or null
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
 
@@ -108,6 +112,7 @@ struct AttendArgs {
   const int32_t* seq_lens;
   const int32_t* block_table;
   const int32_t* sel;
+  const int32_t* sel_phys;  // physical pages of sel (null: look them up)
   float* partial;  // [B*Hkv][nsplit][G][r_v + 2]
   int B, Hq, Hkv, G, d, r_v, S, max_pages, num_phys, top_k, nsplit, pages_per_split;
   int len_offset;

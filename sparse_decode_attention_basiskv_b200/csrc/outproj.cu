@@ -192,12 +192,10 @@ __global__ void __launch_bounds__(kOpThreads, 1)
   if (a.ksplit > 1 && a.cnt) {
     // arrival: the last CTA of this M tile sums the K-split partials into y
     __shared__ int last;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last = atomicAdd(&a.cnt[blockIdx.x], 1) == a.ksplit - 1;
+    __syncthreads();  // this CTA's partials are written
+    if (tid == 0) last = arrive_acq_rel(&a.cnt[blockIdx.x], 1) == a.ksplit - 1;
     __syncthreads();
     if (last) {
-      __threadfence();
       // four rows of one batch column per float4; up to three groups per
       // thread, every load of a split issued before any sum needs it
       const int ngrp = kOpBM / 4 * a.B;

@@ -450,6 +450,195 @@ __global__ void __launch_bounds__(kRsThreads, kRsCtasPerSm)
   }
 }
 
+// -------------------------------------------------------- page selection
+// Per (sequence, KV head): sink page 0 and newest page P-1 always; the other
+// top_k - 2 slots go to the best remaining pages by (score desc, index asc),
+// found exactly with an MSB-first radix select over order-preserving 32-bit
+// keys; ties at the threshold are taken in index order.  Output ascending.
+constexpr int kSelThreads = 512;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f == 0.f) f = 0.f;  // -0 ranks as +0
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+struct SelShared {
+  int hist[2][256];  // radix histograms, alternating between passes
+  int sh[32];        // scan scratch
+  uint32_t digit;
+  int rem;
+};
+
+// Exclusive prefix sum over a block of NT threads; *total receives the sum.
+template <int NT>
+__device__ int block_excl_scan(int v, int* sh, int* total) {
+  constexpr int W = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sh[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < W ? sh[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    sh[lane] = w;
+  }
+  __syncthreads();
+  const int res = (warp ? sh[warp - 1] : 0) + x - v;
+  *total = sh[W - 1];
+  __syncthreads();
+  return res;
+}
+
+// Selection of one (sequence, KV head) by a block of NT threads.  keys and
+// tbl: shared arrays of at least ceil(max_seq_len / S) entries.
+template <int NT>
+__device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32_t* keys, int* tbl,
+                                          SelShared& ss) {
+  const int b = bg / a.Hkv, tid = threadIdx.x;
+  int T = a.seq_lens[b] + a.len_offset;
+  T = T < 0 ? 0 : (T > a.max_seq_len ? a.max_seq_len : T);
+  const int P = (T + a.S - 1) / a.S;
+  int32_t* out = a.sel + (size_t)bg * a.top_k;
+  int32_t* outp = a.sel_phys ? a.sel_phys + (size_t)bg * a.top_k : nullptr;
+  const int32_t* bt = a.block_table + (size_t)b * a.max_pages;
+  if (a.top_k >= P) {
+    for (int i = tid; i < a.top_k; i += NT) {
+      out[i] = i < P ? i : -1;
+      if (outp) outp[i] = i < P ? bt[i] : -1;
+    }
+    return;
+  }
+  const int n = P - 2, need = a.top_k - 2;
+  const float* sc = a.scores + (size_t)bg * a.max_pages + 1;
+  // Scores (and the block-table row of the sequence) in batches of eight
+  // independent loads a thread: one memory round trip per batch.
+  for (int base = 0; base < P; base += 8 * NT) {
+    float v[8];
+    int t[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * NT + tid;
+      v[u] = i < n ? __ldcg(sc + i) : 0.f;
+      t[u] = (outp && i < P) ? bt[i] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * NT + tid;
+      if (i < n) keys[i] = order_key(v[u]);
+      if (outp && i < P) tbl[i] = t[u];
+    }
+  }
+  for (int i = tid; i < 512; i += NT) (&ss.hist[0][0])[i] = 0;
+  __syncthreads();
+
+  // MSB-first radix select of the need-th largest key: two barriers a pass
+  // (the scanning warp clears the other histogram for the next pass).
+  uint32_t prefix = 0, pmask = 0;
+  int rem = need;
+  if (need > 0) {
+    int cur = 0;
+    for (int shift = 24; shift >= 0; shift -= 8, cur ^= 1) {
+      int* hist = ss.hist[cur];
+      // The leading digits of one context's scores are mostly the same (sign
+      // and exponent): lanes sharing lane 0's digit add through one atomic,
+      // the others individually, so same-address atomics do not serialise.
+      for (int base = 0; base < n; base += NT) {
+        const int i = base + tid;
+        int bin = -1;
+        if (i < n) {
+          const uint32_t k = keys[i];
+          if ((k & pmask) == prefix) bin = (int)((k >> shift) & 255);
+        }
+        const int b0 = __shfl_sync(0xffffffffu, bin, 0);
+        const unsigned same = __ballot_sync(0xffffffffu, bin == b0);
+        if (bin >= 0) {
+          if (bin != b0)
+            atomicAdd(&hist[bin], 1);
+          else if ((tid & 31) == __ffs(same) - 1)
+            atomicAdd(&hist[bin], __popc(same));
+        }
+      }
+      __syncthreads();
+      if (tid < 32) {  // lane l covers digits 255-8l .. 248-8l, high to low
+        int local = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) local += hist[255 - 8 * tid - j];
+        int cum = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, cum, o);
+          if (tid >= o) cum += y;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, cum >= rem);
+        const int L = __ffs(hit) - 1;
+        if (tid == L) {
+          int start = cum - local;
+          for (int j = 0; j < 8; ++j) {
+            const int dg = 255 - 8 * L - j;
+            if (start + hist[dg] >= rem) {
+              ss.digit = (uint32_t)dg;
+              ss.rem = rem - start;
+              break;
+            }
+            start += hist[dg];
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss.hist[cur ^ 1][8 * tid + j] = 0;
+      }
+      __syncthreads();
+      prefix |= ss.digit << shift;
+      pmask |= 0xffu << shift;
+      rem = ss.rem;
+    }
+  }
+  const uint32_t thr = prefix;
+  // Contiguous candidate chunk per thread, so prefix sums follow index order.
+  // One scan of packed counts (keys above the threshold << 16 | keys equal to
+  // it): the first `rem` equal keys in index order are taken.
+  const int E = (n + NT - 1) / NT;
+  const int i0 = min(tid * E, n), i1 = min(i0 + E, n);
+  int n_gt = 0, n_eq = 0;
+  if (need > 0)
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t k = keys[i];
+      n_gt += k > thr;
+      n_eq += k == thr;
+    }
+  int total;
+  const int before = block_excl_scan<NT>((n_gt << 16) | n_eq, ss.sh, &total);
+  if (need > 0) {
+    int r = before & 0xffff;
+    int pos = 1 + (before >> 16) + min(r, rem);
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t k = keys[i];
+      if ((k > thr) || (k == thr && r < rem)) {
+        if (outp) outp[pos] = tbl[i + 1];
+        out[pos++] = i + 1;
+      }
+      r += k == thr;
+    }
+  }
+  if (tid == 0) {
+    out[0] = 0;
+    out[a.top_k - 1] = P - 1;
+    if (outp) {
+      outp[0] = tbl[0];
+      outp[a.top_k - 1] = tbl[P - 1];
+    }
+  }
+}
+
 // -------------------------------------- page scoring, plain loads + MMA
 // The same scores without TMA or a staging ring: one warp scores one page
 // at a time straight from plain 16-byte global loads (PW pages per batch,
@@ -523,6 +712,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <int G, int RV, int RK, int S, int PW>
 __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RV, RK, S>()))
     route_mma_kernel(RouteArgs a) {
+  extern __shared__ uint4 rm_frags[];
   constexpr int NZ = RV / 32, NC = (RV + RK) / 32, NT = S / 8, RQ = RV + RK;
   constexpr int SETS = G == 8 ? 2 : 1;
   const int lane = threadIdx.x & 31, lr = lane >> 2, lc = lane & 3;
@@ -589,7 +779,6 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RV, RK, S>()))
   // A fragments of the current group, per warp in shared memory:
   // [set][chunk][k-step][lane] -> (a0, a1, a2, a3).  Each lane writes and
   // reads only its own entries.
-  extern __shared__ uint4 rm_frags[];
   uint4* qa = rm_frags + (size_t)(threadIdx.x >> 5) * (SETS * NC * 2 * 32) + lane;
   int frag_bg = -1;
   auto load_frags = [&](int bb, int gg) {
@@ -697,142 +886,12 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RV, RK, S>()))
   }
 }
 
-// -------------------------------------------------------- page selection
-// Per (sequence, KV head): sink page 0 and newest page P-1 always; the other
-// top_k - 2 slots go to the best remaining pages by (score desc, index asc),
-// found exactly with an MSB-first radix select over order-preserving 32-bit
-// keys; ties at the threshold are taken in index order.  Output ascending.
-constexpr int kSelThreads = 512;
-constexpr int kSelWarps = kSelThreads / 32;
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-  if (f == 0.f) f = 0.f;  // -0 ranks as +0
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-// Exclusive prefix sum over the block; *total receives the sum of all v.
-__device__ int block_excl_scan(int v, int* sh, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sh[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < kSelWarps ? sh[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    sh[lane] = w;
-  }
-  __syncthreads();
-  const int res = (warp ? sh[warp - 1] : 0) + x - v;
-  *total = sh[kSelWarps - 1];
-  __syncthreads();
-  return res;
-}
-
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   extern __shared__ uint32_t keys[];
-  __shared__ int hist[256];
-  __shared__ int sh[32];
-  __shared__ uint32_t s_digit;
-  __shared__ int s_rem;
+  __shared__ SelShared ss;
   pdl_wait();
-  const int bg = blockIdx.x, b = bg / a.Hkv, tid = threadIdx.x;
-  int T = a.seq_lens[b] + a.len_offset;
-  T = T < 0 ? 0 : (T > a.max_seq_len ? a.max_seq_len : T);
-  const int P = (T + a.S - 1) / a.S;
-  int32_t* out = a.sel + (size_t)bg * a.top_k;
-  if (a.top_k >= P) {
-    for (int i = tid; i < a.top_k; i += kSelThreads) out[i] = i < P ? i : -1;
-    return;
-  }
-  const int n = P - 2, need = a.top_k - 2;
-  const float* sc = a.scores + (size_t)bg * a.max_pages + 1;
-  for (int i = tid; i < n; i += kSelThreads) keys[i] = order_key(sc[i]);
-  __syncthreads();
-
-  uint32_t prefix = 0, pmask = 0;
-  int rem = need;
-  if (need > 0) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      if (tid < 256) hist[tid] = 0;
-      __syncthreads();
-      for (int i = tid; i < n; i += kSelThreads) {
-        const uint32_t k = keys[i];
-        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255], 1);
-      }
-      __syncthreads();
-      if (tid < 32) {  // lane l covers digits 255-8l .. 248-8l, high to low
-        int local = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) local += hist[255 - 8 * tid - j];
-        int cum = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, cum, o);
-          if (tid >= o) cum += y;
-        }
-        const unsigned hit = __ballot_sync(0xffffffffu, cum >= rem);
-        const int L = __ffs(hit) - 1;
-        if (tid == L) {
-          int start = cum - local;
-          for (int j = 0; j < 8; ++j) {
-            const int dg = 255 - 8 * L - j;
-            if (start + hist[dg] >= rem) {
-              s_digit = (uint32_t)dg;
-              s_rem = rem - start;
-              break;
-            }
-            start += hist[dg];
-          }
-        }
-      }
-      __syncthreads();
-      prefix |= s_digit << shift;
-      pmask |= 0xffu << shift;
-      rem = s_rem;
-      __syncthreads();
-    }
-  }
-  const uint32_t thr = prefix;
-  // Contiguous candidate chunk per thread, so prefix sums follow index order.
-  const int E = (n + kSelThreads - 1) / kSelThreads;
-  const int i0 = min(tid * E, n), i1 = min(i0 + E, n);
-  int total;
-  int n_eq = 0;
-  if (need > 0)
-    for (int i = i0; i < i1; ++i) n_eq += keys[i] == thr;
-  int eq_rank = block_excl_scan(n_eq, sh, &total);
-  int n_take = 0;
-  if (need > 0) {
-    int r = eq_rank;
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t k = keys[i];
-      n_take += (k > thr) || (k == thr && r < rem);
-      r += k == thr;
-    }
-  }
-  int pos = 1 + block_excl_scan(n_take, sh, &total);
-  if (need > 0) {
-    int r = eq_rank;
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t k = keys[i];
-      if ((k > thr) || (k == thr && r < rem)) out[pos++] = i + 1;
-      r += k == thr;
-    }
-  }
-  if (tid == 0) {
-    out[0] = 0;
-    out[a.top_k - 1] = P - 1;
-  }
+  int* tbl = reinterpret_cast<int*>(keys + (a.max_seq_len + a.S - 1) / a.S);
+  select_group<kSelThreads>(a, blockIdx.x, keys, tbl, ss);
 }
 
 RouteGeom route_geometry(int G, int r_v, int r_k, int S, int wz, int we) {
@@ -974,7 +1033,7 @@ cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
   const int P_max = (a.max_seq_len + a.S - 1) / a.S;
-  const size_t smem = (size_t)(P_max > 2 ? P_max : 2) * sizeof(uint32_t);
+  const size_t smem = (size_t)(P_max > 2 ? P_max : 2) * sizeof(uint32_t) * (a.sel_phys ? 2 : 1);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
