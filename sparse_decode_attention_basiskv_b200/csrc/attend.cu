@@ -575,41 +575,18 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
     const long bg0 = (long)bg * upb;
     const long seg_end = c_end < bg0 + upb ? c_end : bg0 + upb;
     const int b = bg / a.Hkv, g = bg - b * a.Hkv;
-    int T = a.seq_lens[b] + a.len_offset;
-    T = T < 0 ? 0 : T;
-    const int nsel = min(a.top_k, (T + S - 1) / S);
-    const long valid_end = bg0 + (long)nsel * TP;  // units past it have no page
-
-    // the group's queries as B fragments, shared by the CTA's warps: entry
-    // [k][lane (r, c)] holds head r, columns 32k + 8c .. +7 (zero past G)
-    for (int i = tid; i < NKC * 32; i += kAmThreads) {
-      const int k = i >> 5, r = (i & 31) >> 2, cc = i & 3;
-      qs[i] = r < G ? __ldg(reinterpret_cast<const uint4*>(
-                          a.q + ((size_t)b * a.Hq + g * G + r) * D + 32 * k + 8 * cc))
-                    : make_uint4(0u, 0u, 0u, 0u);
-    }
-    __syncthreads();
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2c, 2c + 1
-    float acc[NZC][2][4];
-#pragma unroll
-    for (int c = 0; c < NZC; ++c)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) acc[c][e][0] = acc[c][e][1] = acc[c][e][2] = acc[c][e][3] = 0.f;
-
+    const long u_first = seg + warp;
     // Page ids of the warp's units in this run, fetched 32 at a time (lane i:
     // unit seg + warp + 8 (n0 + i)) with the physical page from the
-    // selection's companion list when there is one (one round trip), else
-    // through the block table.
-    const long u_first = seg + warp;
-    const long u_stop = seg_end < valid_end ? seg_end : valid_end;
-    const int count =
-        u_first < u_stop ? (int)((u_stop - u_first + kAmWarps - 1) / kAmWarps) : 0;
+    // selection's companion list when there is one, else through the block
+    // table.  The first batch goes out with the length and the queries (one
+    // round trip); entries past the selection are fetched but never used.
     int lp_l = -1, pp_l = -1, n0 = 0;
     auto fetch_ids = [&](int base) {
       const long uu = u_first + (long)kAmWarps * (base + lane);
       lp_l = -1;
       pp_l = -1;
-      if (uu < u_stop) {
+      if (uu < seg_end) {
         const size_t si = (size_t)bg * a.top_k + (int)(uu - bg0) / TP;
         lp_l = __ldg(a.sel + si);
         if (a.sel_phys)
@@ -618,6 +595,30 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
           pp_l = __ldg(a.block_table + (size_t)b * a.max_pages + lp_l);
       }
     };
+    int T = a.seq_lens[b] + a.len_offset;
+    fetch_ids(0);
+    // the group's queries as B fragments, shared by the CTA's warps: entry
+    // [k][lane (r, c)] holds head r, columns 32k + 8c .. +7 (zero past G)
+    for (int i = tid; i < NKC * 32; i += kAmThreads) {
+      const int k = i >> 5, r = (i & 31) >> 2, cc = i & 3;
+      qs[i] = r < G ? __ldg(reinterpret_cast<const uint4*>(
+                          a.q + ((size_t)b * a.Hq + g * G + r) * D + 32 * k + 8 * cc))
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+    T = T < 0 ? 0 : T;
+    const int nsel = min(a.top_k, (T + S - 1) / S);
+    const long valid_end = bg0 + (long)nsel * TP;  // units past it have no page
+    __syncthreads();
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2c, 2c + 1
+    float acc[NZC][2][4];
+#pragma unroll
+    for (int c = 0; c < NZC; ++c)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) acc[c][e][0] = acc[c][e][1] = acc[c][e][2] = acc[c][e][3] = 0.f;
+
+    const long u_stop = seg_end < valid_end ? seg_end : valid_end;
+    const int count =
+        u_first < u_stop ? (int)((u_stop - u_first + kAmWarps - 1) / kAmWarps) : 0;
     // ids of unit nn (warp-uniform); a missing entry becomes a fully masked
     // unit on page 0, a bad page is flagged and read as page 0
     auto unit_ids = [&](int nn, int& lp, int& pp) {
@@ -655,7 +656,6 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
     };
     int lp_c = -1, pp_c = 0;
     if (count > 0) {
-      fetch_ids(0);
       unit_ids(0, lp_c, pp_c);
       const size_t row0 = unit_row(0, pp_c);
       load_k(row0);

@@ -505,12 +505,25 @@ template <int NT>
 __device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32_t* keys, int* tbl,
                                           SelShared& ss) {
   const int b = bg / a.Hkv, tid = threadIdx.x;
-  int T = a.seq_lens[b] + a.len_offset;
-  T = T < 0 ? 0 : (T > a.max_seq_len ? a.max_seq_len : T);
-  const int P = (T + a.S - 1) / a.S;
+  const int P_max = (a.max_seq_len + a.S - 1) / a.S;
   int32_t* out = a.sel + (size_t)bg * a.top_k;
   int32_t* outp = a.sel_phys ? a.sel_phys + (size_t)bg * a.top_k : nullptr;
   const int32_t* bt = a.block_table + (size_t)b * a.max_pages;
+  const float* sc = a.scores + (size_t)bg * a.max_pages + 1;
+  // The length, the first batch of scores and the block-table row are
+  // requested together (up to the longest possible context; what lies past
+  // this sequence's pages is dropped): one memory round trip, not two.
+  int T = a.seq_lens[b] + a.len_offset;
+  float v[8];
+  int t[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int i = u * NT + tid;
+    v[u] = i < P_max - 1 ? __ldcg(sc + i) : 0.f;
+    t[u] = (outp && i < P_max) ? bt[i] : 0;
+  }
+  T = T < 0 ? 0 : (T > a.max_seq_len ? a.max_seq_len : T);
+  const int P = (T + a.S - 1) / a.S;
   if (a.top_k >= P) {
     for (int i = tid; i < a.top_k; i += NT) {
       out[i] = i < P ? i : -1;
@@ -519,17 +532,14 @@ __device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32
     return;
   }
   const int n = P - 2, need = a.top_k - 2;
-  const float* sc = a.scores + (size_t)bg * a.max_pages + 1;
-  // Scores (and the block-table row of the sequence) in batches of eight
-  // independent loads a thread: one memory round trip per batch.
-  for (int base = 0; base < P; base += 8 * NT) {
-    float v[8];
-    int t[8];
+  for (int base = 0; base < P; base += 8 * NT) {  // batches of eight loads a thread
+    if (base > 0) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = base + u * NT + tid;
-      v[u] = i < n ? __ldcg(sc + i) : 0.f;
-      t[u] = (outp && i < P) ? bt[i] : 0;
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * NT + tid;
+        v[u] = i < n ? __ldcg(sc + i) : 0.f;
+        t[u] = (outp && i < P) ? bt[i] : 0;
+      }
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
