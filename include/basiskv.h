@@ -176,7 +176,9 @@ BASISKV_API int basiskv_append(const basiskv_dims* dims, const basiskv_bf16* k_n
  *                (used to size the grid; <= max_pages_per_seq*S)
  *   page_scores  fp32 [B][Hkv][max_pages_per_seq] or NULL; entries p >= P_b
  *                are not written
- *   sel          int32 [B][Hkv][top_k] */
+ *   sel          int32 [B][Hkv][top_k], or NULL to compute the page scores
+ *                only (page_scores must then be given)
+ * Both outputs NULL is BASISKV_ERR_INVALID_ARG. */
 BASISKV_API int basiskv_route(const basiskv_dims* dims, const basiskv_bf16* q,
                   const int32_t* seq_lens, int max_seq_len,
                   const int32_t* block_table, const basiskv_bf16* P_K,

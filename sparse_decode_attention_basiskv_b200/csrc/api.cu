@@ -328,7 +328,7 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   r.len_offset = len_offset;
   r.status = status;
   rc = launch_status(launch_route_scores(r, tmZ, tmE, wz, we, st, pdl));
-  if (rc) return rc;
+  if (rc || !sel) return rc;  // no selection requested: scores only
   SelectArgs s{scores, seq_lens, sel, d->B, d->Hkv, d->page_size, d->max_pages_per_seq, top_k,
                max_seq_len, len_offset, block_table,
                reinterpret_cast<int32_t*>(ws + L.selp)};
@@ -532,7 +532,8 @@ int basiskv_route(const basiskv_dims* dims, const basiskv_bf16* q, const int32_t
   BKV_REQUIRE(U_K);
   BKV_REQUIRE(Z_cache);
   BKV_REQUIRE(E_cache);
-  BKV_REQUIRE4(sel);
+  if (!sel && !page_scores) return BASISKV_ERR_INVALID_ARG;  // nothing to write
+  if (sel && !aligned4(sel)) return BASISKV_ERR_INVALID_ARG;
   if (page_scores && !aligned4(page_scores)) return BASISKV_ERR_INVALID_ARG;
   WsLayout L;
   rc = check_ws(dims, top_k, workspace, workspace_bytes, &L);

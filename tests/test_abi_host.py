@@ -84,7 +84,8 @@ def test_route_rejects_bad_args(lib):
 
     assert call(1, None) == bkv.ERR_INVALID_ARG          # q null
     assert call(1, FAKE + 2) == bkv.ERR_INVALID_ARG      # q misaligned
-    assert call(11, None) == bkv.ERR_INVALID_ARG         # sel null
+    assert call(11, None) == bkv.ERR_INVALID_ARG         # sel and page scores both null
+    assert call(11, FAKE + 2) == bkv.ERR_INVALID_ARG     # sel misaligned
     assert call(9, 1) == bkv.ERR_INVALID_ARG             # top_k < 2
     assert call(3, 0) == bkv.ERR_INVALID_ARG             # empty context bound
     assert call(3, 64 * 16 + 1) == bkv.ERR_INVALID_ARG   # past the block-table row

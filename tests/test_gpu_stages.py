@@ -21,6 +21,12 @@ SMALL = {
     "llama_b16_t2k": synth.with_sizes(synth.LLAMA8B_T32K_B16, T=2000, top_k=32),
     # the Qwen3-32B layer shape (G 8, page 32) at a short context
     "qwen_b2_t3k": synth.with_sizes(synth.QWEN32B_T64K_B8, B=2, T=3000, prefill_tokens=0),
+    # shapes outside the plain-load kernels' lists: page 8 (TMA-ring scoring
+    # and attention kernels with their split merge) and r_k 64 (generic scoring)
+    "llama_p8_b2_t1500": synth.with_sizes(synth.LLAMA8B_T4K, B=2, T=1500, page_size=8,
+                                          top_k=48),
+    "llama_rk64_b2_t1500": synth.with_sizes(synth.LLAMA8B_T4K, B=2, T=1500, r_v=64, r_k=64,
+                                            top_k=32),
 }
 
 
@@ -181,6 +187,25 @@ def test_dense_when_top_k_covers_context():
     out = O.decode_sequence(np64(pb.q[0]), c["K"], c["Z"], c["E"], wl.T, 16, 40, f["P_K"],
                             f["U_K"], W)
     assert_within(np64(y[0]), out["y"], Y_REL, Y_ABS)
+
+
+def test_route_scores_only_matches_full_call():
+    """basiskv_route with sel = NULL computes the same page scores (bit for
+    bit) as the full call, and writes no selection."""
+    wl = synth.with_sizes(synth.LLAMA8B_T4K, B=2, T=1000, top_k=16)
+    pb, layer = gpu_layer(wl)
+    d = layer.dims
+    sc1 = torch.zeros(2, 8, d.max_pages_per_seq, device="cuda")
+    sc2 = torch.zeros_like(sc1)
+    sel = torch.empty(2, 8, 16, dtype=torch.int32, device="cuda")
+    bkv.basiskv_route(d, pb.q, layer.seq_lens, wl.T, layer.block_table, layer.P_K, layer.U_K,
+                      layer.Z, layer.E, 16, sc1, sel, layer.workspace)
+    bkv.basiskv_route(d, pb.q, layer.seq_lens, wl.T, layer.block_table, layer.P_K, layer.U_K,
+                      layer.Z, layer.E, 16, sc2, None, layer.workspace)
+    torch.cuda.synchronize()
+    status_clean()
+    P = -(-wl.T // wl.page_size)
+    assert torch.equal(sc1[:, :, :P], sc2[:, :, :P])
 
 
 def test_block_table_permutation_invariance():
