@@ -21,29 +21,36 @@ __global__ void __launch_bounds__(kAppendThreads) append_small_kernel(AppendArgs
   extern __shared__ __align__(16) uint16_t fac[];  // A_V | P_K | U_K of head g
   __shared__ float vs[kAppendThreads], ks[kAppendThreads], zs[kAppendThreads],
       rs[kAppendThreads];
-  append_block(a, blockIdx.x, blockIdx.y, blockIdx.z, fac, vs, ks, zs, rs);
+  append_block(a, blockIdx.x, blockIdx.y, blockIdx.z, fac, vs, ks, zs, rs, threadIdx.x, 0);
 }
 
-// The first launch of a fused decode step: blocks [0, n_fold) fold the
-// queries, the next B*Hkv blocks append the step's token (one per sequence
-// and KV head), and block 0 also zeroes the step's arrival counters.  The
-// two jobs are independent, so one launch runs them side by side.
-__global__ void __launch_bounds__(kAppendThreads)
-    decode_prologue_kernel(FoldQArgs f, AppendArgs a, int n_fold, int fold_ny, int* counters,
+// The first launch of a fused decode step, one block per (sequence, KV
+// head): 128-thread group i < n_fold folds the group's queries for outputs
+// 32i .. 32i + 31, and (when the step appends) the last group appends the
+// step's token; each group synchronises on its own named barrier, so the
+// fold and the append run side by side in one wave.  Block 0 also zeroes
+// the step's arrival counters.
+constexpr int kPrologueMaxThreads = 7 * 128;  // up to 6 fold groups + the append group
+
+__global__ void __launch_bounds__(kPrologueMaxThreads)
+    decode_prologue_kernel(FoldQArgs f, AppendArgs a, int n_fold, int* counters,
                            int n_counters) {
-  extern __shared__ __align__(16) uint16_t dyn[];
+  extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ float vs[kAppendThreads], ks[kAppendThreads], zs[kAppendThreads],
       rs[kAppendThreads];
-  const int bid = blockIdx.x;
-  if (bid == 0 && counters) {
+  const int bg = blockIdx.x, grp = threadIdx.x / kFoldThreads, gtid = threadIdx.x % kFoldThreads;
+  if (bg == 0 && counters) {
     pdl_wait();
     for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
   }
-  if (bid < n_fold) {
-    fold_query_block(f, bid / fold_ny, bid % fold_ny, reinterpret_cast<float*>(dyn));
+  const size_t fold_bytes = fold_block_smem(f.Hq / f.Hkv, f.d);
+  if (grp < n_fold) {
+    fold_query_block(f, bg, grp, reinterpret_cast<float*>(dyn + grp * fold_bytes), gtid,
+                     1 + grp);
   } else {
-    const int r = bid - n_fold;  // (sequence, KV head)
-    append_block(a, r % a.Hkv, 0, r / a.Hkv, dyn, vs, ks, zs, rs);
+    append_block(a, bg % a.Hkv, 0, bg / a.Hkv,
+                 reinterpret_cast<uint16_t*>(dyn + n_fold * fold_bytes), vs, ks, zs, rs, gtid,
+                 1 + grp);
   }
 }
 
@@ -84,22 +91,19 @@ cudaError_t launch_bump_lengths(const AppendArgs& a, cudaStream_t st, bool pdl) 
 
 cudaError_t launch_decode_prologue(const FoldQArgs& f, const AppendArgs& a, int* counters,
                                    int n_counters, cudaStream_t st, bool pdl) {
-  const int G = f.Hq / f.Hkv;
-  const int fold_ny = (f.r_v + f.r_k + 31) / 32;
-  const int n_fold = f.B * f.Hkv * fold_ny;
-  const int n_app = a.k_new ? a.B * a.Hkv : 0;
-  size_t smem = fold_block_smem(G, f.d);
-  if (n_app) {
-    const size_t s2 = append_block_smem(a.d, a.r_v, a.r_k);
-    if (s2 > smem) smem = s2;
-  }
+  const int n_fold = (f.r_v + f.r_k + 31) / 32;
+  const bool app = a.k_new != nullptr;
+  const int threads = (n_fold + (app ? 1 : 0)) * kFoldThreads;
+  if (threads > kPrologueMaxThreads) return cudaErrorInvalidConfiguration;
+  size_t smem = (size_t)n_fold * fold_block_smem(f.Hq / f.Hkv, f.d);
+  if (app) smem += append_block_smem(a.d, a.r_v, a.r_k);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(decode_prologue_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_k(decode_prologue_kernel, dim3(n_fold + n_app), dim3(kAppendThreads), smem, st,
-                  pdl, f, a, n_fold, fold_ny, counters, n_counters);
+  return launch_k(decode_prologue_kernel, dim3(f.B * f.Hkv), dim3(threads), smem, st, pdl, f, a,
+                  n_fold, counters, n_counters);
 }
 
 }  // namespace basiskv

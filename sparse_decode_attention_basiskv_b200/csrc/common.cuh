@@ -269,6 +269,21 @@ __device__ __forceinline__ int arrive_acq_rel(int* counter, int v) {
   return old;
 }
 
+// Asynchronous 16-byte global -> shared copy (no register staging); complete
+// after cp_async_wait_all() in the issuing thread, visible to the block after
+// a barrier that follows it.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // ------------------------------------------------------------- PDL control
 __device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");

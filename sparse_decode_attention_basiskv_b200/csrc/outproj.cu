@@ -129,9 +129,12 @@ __global__ void __launch_bounds__(kOpThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();
-  if (a.bump_lens && blockIdx.x == 0 && blockIdx.y == 0) {
-    for (int b = tid; b < a.B; b += kOpThreads) {
+  // Only the producer (before the latent tiles) and the length update wait
+  // for the earlier kernels: W' is a weight no kernel of the step writes, so
+  // the first stages of it are requested while the attention finishes.
+  if (a.bump_lens && blockIdx.x == 0 && blockIdx.y == 0 && warp == 2) {
+    pdl_wait();
+    for (int b = lane; b < a.B; b += 32) {
       const int len = a.bump_lens[b];
       if (len >= 0 && len + a.bump_n <= a.bump_cap) a.bump_lens[b] = len + a.bump_n;
     }
@@ -139,7 +142,15 @@ __global__ void __launch_bounds__(kOpThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {  // ---------------------------------------- TMA producer
-      for (int kb = kb0, it = 0; kb < kb1; ++kb, ++it) {
+      const int pre = kb1 - kb0 < kOpStages ? kb1 - kb0 : kOpStages;
+      for (int it = 0; it < pre; ++it) {  // stages start empty
+        mbar_arrive_expect_tx(&full[it], kOpATile + kBTile);
+        tma_load_2d(a_tiles + it * kOpATile, &tmW, (kb0 + it) * kOpBK, m0, &full[it]);
+      }
+      pdl_wait();
+      for (int it = 0; it < pre; ++it)
+        tma_load_2d(b_tiles + it * kBTile, &tmA, (kb0 + it) * kOpBK, 0, &full[it]);
+      for (int kb = kb0 + pre, it = pre; kb < kb1; ++kb, ++it) {
         const int s = it % kOpStages;
         if (!mbar_wait(&empty[s], ((it / kOpStages) & 1) ^ 1, a.status)) break;
         mbar_arrive_expect_tx(&full[s], kOpATile + kBTile);

@@ -31,7 +31,7 @@ namespace {
 // qt[b][h][r_v + c] = sum_i q[b][h][i] U_K[g][i][c]           c < r_k
 __global__ void __launch_bounds__(kFoldThreads) fold_query_kernel(FoldQArgs a) {
   extern __shared__ float fsm[];
-  fold_query_block(a, blockIdx.x, blockIdx.y, fsm);
+  fold_query_block(a, blockIdx.x, blockIdx.y, fsm, threadIdx.x, 0);
 }
 
 // ------------------------------------------------------------ page scoring

@@ -11,12 +11,13 @@ namespace basiskv {
 constexpr int kAppendThreads = 128;  // >= max(d, r_v, r_k) of every supported shape
 constexpr int kFoldThreads = 128;    // 32 outputs x 4 quarters of the head dim
 
-// Copies n bf16 values (n % 8 == 0, both pointers 16-byte aligned) with
-// independent 16-byte loads spread over the block.
-__device__ __forceinline__ void stage_bf16(uint16_t* dst, const uint16_t* src, int n) {
-  const uint4* s4 = reinterpret_cast<const uint4*>(src);
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-  for (int i = threadIdx.x; i < n / 8; i += blockDim.x) d4[i] = s4[i];
+// Starts copying n bf16 values (n % 8 == 0, both pointers 16-byte aligned)
+// into shared memory with asynchronous 16-byte copies spread over the block:
+// every copy is in flight at once (one memory round trip in all).  Complete
+// after cp_async_wait_all() and a barrier.
+__device__ __forceinline__ void stage_bf16_async(uint16_t* dst, const uint16_t* src, int n,
+                                                 int tid, int nthreads) {
+  for (int i = tid; i < n / 8; i += nthreads) cp_async16(dst + 8 * i, src + 8 * i);
 }
 
 // Appends token j of sequence b for KV head g:
@@ -24,30 +25,35 @@ __device__ __forceinline__ void stage_bf16(uint16_t* dst, const uint16_t* src, i
 // The head's three factors (at most 128x128 + 128x128 + 128x64 bf16 = 80 KB)
 // are first staged in `fac` (shared) with independent 16-byte loads, so the
 // dot products read shared memory instead of waiting on one global load per
-// step.  vs, ks, zs, rs: shared scratch of kAppendThreads floats each.
+// step.  vs, ks, zs, rs: shared scratch of kAppendThreads floats each.  Run
+// by kAppendThreads threads (tid = 0..kAppendThreads-1) that synchronise on
+// named barrier bar (0 when they are the whole block).
 __device__ __forceinline__ void append_block(const AppendArgs& a, int g, int j, int b,
                                              uint16_t* fac, float* vs, float* ks, float* zs,
-                                             float* rs) {
-  const int tid = threadIdx.x;
+                                             float* rs, int tid, int bar) {
   const int d = a.d, r_v = a.r_v, r_k = a.r_k;
   uint16_t* A = fac;
   uint16_t* Pk = fac + d * r_v;
   uint16_t* U = Pk + r_v * d;
-  // Factors are inputs no predecessor writes: stage them before the wait.
-  stage_bf16(A, a.A_V + (size_t)g * d * r_v, d * r_v);
-  stage_bf16(Pk, a.P_K + (size_t)g * r_v * d, r_v * d);
-  stage_bf16(U, a.U_K + (size_t)g * d * r_k, d * r_k);
+  // Factors are inputs no predecessor writes: their copies start before the
+  // wait and land while the length and the page are looked up.
+  stage_bf16_async(A, a.A_V + (size_t)g * d * r_v, d * r_v, tid, kAppendThreads);
+  stage_bf16_async(Pk, a.P_K + (size_t)g * r_v * d, r_v * d, tid, kAppendThreads);
+  stage_bf16_async(U, a.U_K + (size_t)g * d * r_k, d * r_k, tid, kAppendThreads);
+  cp_async_commit();
   pdl_wait();
   const int len = a.seq_lens[b];
   const int cap = a.max_pages * a.S;
   if (len < 0 || len + a.n_new > cap) {
     if (tid == 0 && g == 0 && j == 0) raise_status(a.status, BASISKV_DEV_OVERFLOW);
+    cp_async_wait_all();  // no copy outlives the block
     return;
   }
   const int pos = len + j;
   const int pp = a.block_table[(size_t)b * a.max_pages + pos / a.S];
   if (pp < 0 || pp >= a.num_phys) {
     if (tid == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
+    cp_async_wait_all();
     return;
   }
   const size_t slot = ((size_t)pp * a.Hkv + g) * a.S + pos % a.S;
@@ -58,7 +64,8 @@ __device__ __forceinline__ void append_block(const AppendArgs& a, int g, int j, 
     vs[tid] = bf16_to_f(a.v_new[tok + tid]);
     a.K_cache[slot * d + tid] = kb;
   }
-  __syncthreads();
+  cp_async_wait_all();
+  named_bar_sync(bar, kAppendThreads);
   if (tid < r_v) {  // z_j = sum_i v_i A_V[i][j]
     float acc = 0.f;
 #pragma unroll 8
@@ -66,14 +73,14 @@ __device__ __forceinline__ void append_block(const AppendArgs& a, int g, int j, 
     zs[tid] = acc;
     a.Z_cache[slot * r_v + tid] = f_to_bf16(acc);
   }
-  __syncthreads();
+  named_bar_sync(bar, kAppendThreads);
   if (tid < d) {  // residual_i = k_i - sum_j z_j P_K[j][i]   (z unrounded)
     float acc = ks[tid];
 #pragma unroll 8
     for (int jj = 0; jj < r_v; ++jj) acc = fmaf(-zs[jj], bf16_to_f(Pk[jj * d + tid]), acc);
     rs[tid] = acc;
   }
-  __syncthreads();
+  named_bar_sync(bar, kAppendThreads);
   if (tid < r_k) {  // e_c = sum_i residual_i U_K[i][c]
     float acc = 0.f;
 #pragma unroll 8
@@ -88,11 +95,12 @@ __device__ __forceinline__ void append_block(const AppendArgs& a, int g, int j, 
 // Warp w sums the products over the w-th quarter of the head dimension for
 // every head of the group; the four partial sums meet in shared memory
 // (fsm: G*d + 4*G*32 floats).  All loads of a thread are independent, so the
-// block costs about one memory round trip.
+// block costs about one memory round trip.  Run by kFoldThreads threads
+// (tid = 0..kFoldThreads-1, whole warps) on named barrier bar.
 __device__ __forceinline__ void fold_query_block(const FoldQArgs& a, int bg, int yblk,
-                                                 float* fsm) {
+                                                 float* fsm, int tid, int bar) {
   const int b = bg / a.Hkv, g = bg % a.Hkv;
-  const int tid = threadIdx.x, lane = tid & 31, quarter = tid >> 5;
+  const int lane = tid & 31, quarter = tid >> 5;
   const int G = a.Hq / a.Hkv, rq = a.r_v + a.r_k, d = a.d;
   const int j = yblk * 32 + lane;
   const int i0 = quarter * (d / 4), n = d / 4;
@@ -101,12 +109,13 @@ __device__ __forceinline__ void fold_query_block(const FoldQArgs& a, int bg, int
   pdl_wait();
   for (int i = tid; i < G * d; i += kFoldThreads)
     qs[i] = bf16_to_f(a.q[((size_t)b * a.Hq + g * G) * d + i]);
-  __syncthreads();
+  named_bar_sync(bar, kFoldThreads);
   float acc[8];
 #pragma unroll
   for (int h = 0; h < 8; ++h) acc[h] = 0.f;
   if (j < a.r_v) {  // row j of P_K, this quarter: n contiguous bf16 (16-byte aligned)
     const uint4* row = reinterpret_cast<const uint4*>(a.P_K + ((size_t)g * a.r_v + j) * d + i0);
+#pragma unroll 4
     for (int c = 0; c < n / 8; ++c) {
       const uint4 w = row[c];
       const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -121,6 +130,7 @@ __device__ __forceinline__ void fold_query_block(const FoldQArgs& a, int bg, int
     }
   } else if (j < rq) {  // column j - r_v of U_K, this quarter (coalesced across lanes)
     const uint16_t* col = a.U_K + (size_t)g * d * a.r_k + (j - a.r_v);
+#pragma unroll 8
     for (int i = i0; i < i0 + n; ++i) {
       const float u = bf16_to_f(col[(size_t)i * a.r_k]);
 #pragma unroll
@@ -131,7 +141,7 @@ __device__ __forceinline__ void fold_query_block(const FoldQArgs& a, int bg, int
 #pragma unroll
   for (int h = 0; h < 8; ++h)
     if (h < G) part[(quarter * G + h) * 32 + lane] = acc[h];
-  __syncthreads();
+  named_bar_sync(bar, kFoldThreads);
   for (int o = tid; o < G * 32; o += kFoldThreads) {
     const int h = o / 32, jj = yblk * 32 + (o % 32);
     if (jj < rq) {
@@ -142,9 +152,12 @@ __device__ __forceinline__ void fold_query_block(const FoldQArgs& a, int bg, int
   }
 }
 
-inline size_t append_block_smem(int d, int r_v, int r_k) {
+__host__ __device__ inline size_t append_block_smem(int d, int r_v, int r_k) {
   return (size_t)(2 * d * r_v + d * r_k) * sizeof(uint16_t);
 }
-inline size_t fold_block_smem(int G, int d) { return (size_t)(G * d + 4 * G * 32) * sizeof(float); }
+__host__ __device__ inline size_t fold_block_smem(int G, int d) {
+  return (size_t)(G * d + 4 * G * 32) * sizeof(float);
+}
+static_assert(kAppendThreads == kFoldThreads, "the prologue's groups share one size");
 
 }  // namespace basiskv
