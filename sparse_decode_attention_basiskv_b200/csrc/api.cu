@@ -269,7 +269,9 @@ int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_b
   if (w_app) {  // prefill chunk: one tensor-core product per KV head
     if (fold_first) {
       FoldAppArgs f{A_V, P_K, U_K, w_app, d->Hkv, d->d, d->r_v, d->r_k};
-      rc = launch_status(launch_fold_append(f, st, pdl));
+      // no programmatic early start: this kernel reads its inputs without a
+      // grid-dependency wait
+      rc = launch_status(launch_fold_append(f, st, false));
       if (rc) return rc;
     }
     const int N = d->r_v + d->r_k;
@@ -295,7 +297,8 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
               int max_seq_len, const int32_t* block_table, const basiskv_bf16* P_K,
               const basiskv_bf16* U_K, const basiskv_bf16* Z_cache, const basiskv_bf16* E_cache,
               int top_k, float* scores, int32_t* sel, uint8_t* ws, const WsLayout& L,
-              cudaStream_t st, bool pdl, int len_offset = 0, bool do_fold = true) {
+              cudaStream_t st, bool pdl, int len_offset = 0, bool do_fold = true,
+              const AppendArgs* with_append = nullptr) {
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   const int wz = z_box_cols(d->r_v), we = e_box_cols(d->r_k);
@@ -332,6 +335,7 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   SelectArgs s{scores, seq_lens, sel, d->B, d->Hkv, d->page_size, d->max_pages_per_seq, top_k,
                max_seq_len, len_offset, block_table,
                reinterpret_cast<int32_t*>(ws + L.selp)};
+  if (with_append) return launch_status(launch_select_append(s, *with_append, st, pdl));
   return launch_status(launch_select(s, st, pdl));
 }
 
@@ -626,22 +630,27 @@ int basiskv_decode(const basiskv_dims* dims, const basiskv_bf16* q, const basisk
   // only at the end of the step (by the out-projection launch), and the
   // stages in between read seq_lens[b] + 1.
   const int off = append ? 1 : 0;
-  // Launch 1: the query fold and the token append side by side; it also
-  // zeroes the arrival counters of the fused merge and reduction below.
+  // Launch 1: the query fold; it also zeroes the arrival counters of the
+  // fused merge and reduction below.  The token append runs in the selection
+  // launch (launch 3): the scoring reads the newest page before the new token
+  // is in it, which only changes that page's score, and the newest page is
+  // selected whatever its score.
   int* cnt = reinterpret_cast<int*>(ws + L.counters);
-  {
-    AppendArgs a = make_append_args(dims, append ? k_new : nullptr, v_new, 1, seq_lens,
+  AppendArgs app = make_append_args(dims, append ? k_new : nullptr, v_new, 1, seq_lens,
                                     block_table, A_V, P_K, U_K, K_cache, Z_cache, E_cache);
-    if (!a.status) return BASISKV_ERR_CUDA;
+  if (!app.status) return BASISKV_ERR_CUDA;
+  {
+    AppendArgs none = app;
+    none.k_new = nullptr;
     FoldQArgs f{q, P_K, U_K, reinterpret_cast<float*>(ws + L.qt), dims->B, dims->Hq, dims->Hkv,
                 dims->d, dims->r_v, dims->r_k};
     rc = launch_status(
-        launch_decode_prologue(f, a, cnt, L.n_att_cnt + L.n_op_cnt, st, pdl));
+        launch_decode_prologue(f, none, cnt, L.n_att_cnt + L.n_op_cnt, st, pdl));
     if (rc) return rc;
   }
   rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache, top_k,
                  reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl, off,
-                 /*do_fold=*/false);
+                 /*do_fold=*/false, append ? &app : nullptr);
   if (rc) return rc;
   uint16_t* a16 = reinterpret_cast<uint16_t*>(ws + L.a_bf16);
   rc = run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel_buf, top_k, nullptr, a16,

@@ -103,6 +103,10 @@ struct SelectArgs {
   int32_t* sel_phys;  // [B][Hkv][top_k] or null
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
+// The selection together with a one-token append (a.n_new == 1), whose
+// result no stage before the attention reads.
+cudaError_t launch_select_append(const SelectArgs& s, const AppendArgs& a, cudaStream_t st,
+                                 bool pdl);
 
 // ------------------------------------------------------------------ attend
 struct AttendArgs {

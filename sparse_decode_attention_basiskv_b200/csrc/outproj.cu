@@ -24,9 +24,15 @@ namespace {
 
 constexpr int kOpThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
 constexpr int kOpBM = 128, kOpBK = 64;
-// Ring depth: 6 stages of (16 KB + BN*128 B) fit in shared memory up to BN = 128.
+// Ring depth: as many stages of (16 KB + BN*128 B) as fit in 200 KB, at most
+// 8 (a decode-size K slice is 8 stages deep, so the whole slice of W' can be
+// in flight before the latents are ready).
 template <int BN>
-constexpr int op_stages() { return BN >= 256 ? 4 : 6; }
+constexpr int op_stages() {
+  return (200 * 1024) / (kOpBM * kOpBK * 2 + BN * kOpBK * 2) < 8
+             ? (200 * 1024) / (kOpBM * kOpBK * 2 + BN * kOpBK * 2)
+             : 8;
+}
 constexpr int kOpATile = kOpBM * kOpBK * 2;  // 16 KB
 
 // tcgen05 instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B,

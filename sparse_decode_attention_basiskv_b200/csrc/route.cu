@@ -1041,6 +1041,46 @@ cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
   }
 }
 
+namespace {
+// Selection blocks [0, B*Hkv) and, after them, one block per (sequence, KV
+// head) that appends the step's token (its first 128 threads; the append's
+// result is first read by the attention kernel, so it runs in the shadow of
+// the selection instead of before the scoring).
+__global__ void __launch_bounds__(kSelThreads)
+    select_append_kernel(SelectArgs s, AppendArgs a) {
+  extern __shared__ __align__(16) uint8_t sa_dyn[];
+  __shared__ SelShared ss;
+  __shared__ float vs[kAppendThreads], ks[kAppendThreads], zs[kAppendThreads],
+      rs[kAppendThreads];
+  const int nsel = s.B * s.Hkv;
+  if ((int)blockIdx.x < nsel) {
+    pdl_wait();
+    uint32_t* keys = reinterpret_cast<uint32_t*>(sa_dyn);
+    select_group<kSelThreads>(s, blockIdx.x, keys,
+                              reinterpret_cast<int*>(keys + (s.max_seq_len + s.S - 1) / s.S), ss);
+  } else if (threadIdx.x < kAppendThreads) {
+    const int r = blockIdx.x - nsel;  // (sequence, KV head)
+    append_block(a, r % a.Hkv, 0, r / a.Hkv, reinterpret_cast<uint16_t*>(sa_dyn), vs, ks, zs, rs,
+                 threadIdx.x, 1);
+  }
+}
+}  // namespace
+
+cudaError_t launch_select_append(const SelectArgs& s, const AppendArgs& a, cudaStream_t st,
+                                 bool pdl) {
+  const int P_max = (s.max_seq_len + s.S - 1) / s.S;
+  size_t smem = (size_t)(P_max > 2 ? P_max : 2) * sizeof(uint32_t) * (s.sel_phys ? 2 : 1);
+  const size_t app = append_block_smem(a.d, a.r_v, a.r_k);
+  if (app > smem) smem = app;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(select_append_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_k(select_append_kernel, dim3(2 * s.B * s.Hkv), dim3(kSelThreads), smem, st, pdl,
+                  s, a);
+}
+
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl) {
   const int P_max = (a.max_seq_len + a.S - 1) / a.S;
   const size_t smem = (size_t)(P_max > 2 ? P_max : 2) * sizeof(uint32_t) * (a.sel_phys ? 2 : 1);

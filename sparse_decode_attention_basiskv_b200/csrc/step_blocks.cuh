@@ -23,7 +23,7 @@ __device__ __forceinline__ void stage_bf16_async(uint16_t* dst, const uint16_t* 
 // Appends token j of sequence b for KV head g:
 //   z = v A_V,g;  e = (k - z P_K,g) U_K,g (z unrounded);  K <- k.
 // The head's three factors (at most 128x128 + 128x128 + 128x64 bf16 = 80 KB)
-// are first staged in `fac` (shared) with independent 16-byte loads, so the
+// are first staged in `fac` (shared) with asynchronous 16-byte copies, so the
 // dot products read shared memory instead of waiting on one global load per
 // step.  vs, ks, zs, rs: shared scratch of kAppendThreads floats each.  Run
 // by kAppendThreads threads (tid = 0..kAppendThreads-1) that synchronise on
@@ -35,58 +35,81 @@ __device__ __forceinline__ void append_block(const AppendArgs& a, int g, int j, 
   uint16_t* A = fac;
   uint16_t* Pk = fac + d * r_v;
   uint16_t* U = Pk + r_v * d;
-  // Factors are inputs no predecessor writes: their copies start before the
-  // wait and land while the length and the page are looked up.
+  // Every input is read after the wait (a kernel just before this one may
+  // have written any of them), but all first reads go out together: the
+  // factor copies, the length, and the token itself, whose position in the
+  // cache is not needed until the final stores.
+  pdl_wait();
   stage_bf16_async(A, a.A_V + (size_t)g * d * r_v, d * r_v, tid, kAppendThreads);
   stage_bf16_async(Pk, a.P_K + (size_t)g * r_v * d, r_v * d, tid, kAppendThreads);
   stage_bf16_async(U, a.U_K + (size_t)g * d * r_k, d * r_k, tid, kAppendThreads);
   cp_async_commit();
-  pdl_wait();
-  const int len = a.seq_lens[b];
-  const int cap = a.max_pages * a.S;
-  if (len < 0 || len + a.n_new > cap) {
-    if (tid == 0 && g == 0 && j == 0) raise_status(a.status, BASISKV_DEV_OVERFLOW);
-    cp_async_wait_all();  // no copy outlives the block
-    return;
-  }
-  const int pos = len + j;
-  const int pp = a.block_table[(size_t)b * a.max_pages + pos / a.S];
-  if (pp < 0 || pp >= a.num_phys) {
-    if (tid == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
-    cp_async_wait_all();
-    return;
-  }
-  const size_t slot = ((size_t)pp * a.Hkv + g) * a.S + pos % a.S;
   const size_t tok = (((size_t)b * a.n_new + j) * a.Hkv + g) * d;
+  uint16_t kb = 0;
   if (tid < d) {
-    const uint16_t kb = a.k_new[tok + tid];
+    kb = a.k_new[tok + tid];
     ks[tid] = bf16_to_f(kb);
     vs[tid] = bf16_to_f(a.v_new[tok + tid]);
-    a.K_cache[slot * d + tid] = kb;
   }
+  const int len = a.seq_lens[b];
+  const int cap = a.max_pages * a.S;
+  const bool fits = len >= 0 && len + a.n_new <= cap;
+  const int pos = len + j;
+  // block-table entry requested now, used at the end
+  const int pp = fits ? a.block_table[(size_t)b * a.max_pages + pos / a.S] : -1;
   cp_async_wait_all();
   named_bar_sync(bar, kAppendThreads);
+  float zv = 0.f, ev = 0.f;
+  // Each dot product keeps four independent partial sums (d and r_v are
+  // multiples of 32), so its chain of dependent FMAs is a quarter as long.
   if (tid < r_v) {  // z_j = sum_i v_i A_V[i][j]
-    float acc = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < d; ++i) acc = fmaf(vs[i], bf16_to_f(A[i * r_v + tid]), acc);
-    zs[tid] = acc;
-    a.Z_cache[slot * r_v + tid] = f_to_bf16(acc);
+    float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+#pragma unroll 4
+    for (int i = 0; i < d; i += 4) {
+      c0 = fmaf(vs[i], bf16_to_f(A[i * r_v + tid]), c0);
+      c1 = fmaf(vs[i + 1], bf16_to_f(A[(i + 1) * r_v + tid]), c1);
+      c2 = fmaf(vs[i + 2], bf16_to_f(A[(i + 2) * r_v + tid]), c2);
+      c3 = fmaf(vs[i + 3], bf16_to_f(A[(i + 3) * r_v + tid]), c3);
+    }
+    zv = (c0 + c1) + (c2 + c3);
+    zs[tid] = zv;
   }
   named_bar_sync(bar, kAppendThreads);
   if (tid < d) {  // residual_i = k_i - sum_j z_j P_K[j][i]   (z unrounded)
-    float acc = ks[tid];
-#pragma unroll 8
-    for (int jj = 0; jj < r_v; ++jj) acc = fmaf(-zs[jj], bf16_to_f(Pk[jj * d + tid]), acc);
-    rs[tid] = acc;
+    float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+#pragma unroll 4
+    for (int jj = 0; jj < r_v; jj += 4) {
+      c0 = fmaf(zs[jj], bf16_to_f(Pk[jj * d + tid]), c0);
+      c1 = fmaf(zs[jj + 1], bf16_to_f(Pk[(jj + 1) * d + tid]), c1);
+      c2 = fmaf(zs[jj + 2], bf16_to_f(Pk[(jj + 2) * d + tid]), c2);
+      c3 = fmaf(zs[jj + 3], bf16_to_f(Pk[(jj + 3) * d + tid]), c3);
+    }
+    rs[tid] = ks[tid] - ((c0 + c1) + (c2 + c3));
   }
   named_bar_sync(bar, kAppendThreads);
   if (tid < r_k) {  // e_c = sum_i residual_i U_K[i][c]
-    float acc = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < d; ++i) acc = fmaf(rs[i], bf16_to_f(U[i * r_k + tid]), acc);
-    a.E_cache[slot * r_k + tid] = f_to_bf16(acc);
+    float c0 = 0.f, c1 = 0.f, c2 = 0.f, c3 = 0.f;
+#pragma unroll 4
+    for (int i = 0; i < d; i += 4) {
+      c0 = fmaf(rs[i], bf16_to_f(U[i * r_k + tid]), c0);
+      c1 = fmaf(rs[i + 1], bf16_to_f(U[(i + 1) * r_k + tid]), c1);
+      c2 = fmaf(rs[i + 2], bf16_to_f(U[(i + 2) * r_k + tid]), c2);
+      c3 = fmaf(rs[i + 3], bf16_to_f(U[(i + 3) * r_k + tid]), c3);
+    }
+    ev = (c0 + c1) + (c2 + c3);
   }
+  if (!fits) {
+    if (tid == 0 && g == 0 && j == 0) raise_status(a.status, BASISKV_DEV_OVERFLOW);
+    return;
+  }
+  if (pp < 0 || pp >= a.num_phys) {
+    if (tid == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
+    return;
+  }
+  const size_t slot = ((size_t)pp * a.Hkv + g) * a.S + pos % a.S;
+  if (tid < d) a.K_cache[slot * d + tid] = kb;
+  if (tid < r_v) a.Z_cache[slot * r_v + tid] = f_to_bf16(zv);
+  if (tid < r_k) a.E_cache[slot * r_k + tid] = f_to_bf16(ev);
 }
 
 // Folds the queries of (sequence, KV head) bg for outputs 32*yblk .. +31:
@@ -107,35 +130,62 @@ __device__ __forceinline__ void fold_query_block(const FoldQArgs& a, int bg, int
   float* qs = fsm;            // [G][d]
   float* part = fsm + G * d;  // [4][G][32]
   pdl_wait();
-  for (int i = tid; i < G * d; i += kFoldThreads)
-    qs[i] = bf16_to_f(a.q[((size_t)b * a.Hq + g * G) * d + i]);
+  // This thread's factor values go out first, all at once (they do not
+  // depend on the queries): a row quarter of P_K (n/8 <= 4 chunks of 16
+  // bytes) or a column quarter of U_K (n <= 32 values).
+  const bool is_p = j < a.r_v, is_u = !is_p && j < rq;
+  uint4 prow[4];
+  float ucol[32];
+  if (is_p) {
+    const uint4* row = reinterpret_cast<const uint4*>(a.P_K + ((size_t)g * a.r_v + j) * d + i0);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) prow[c] = c < n / 8 ? row[c] : make_uint4(0u, 0u, 0u, 0u);
+  } else if (is_u) {
+    const uint16_t* col = a.U_K + (size_t)g * d * a.r_k + (j - a.r_v) + (size_t)i0 * a.r_k;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) ucol[k] = k < n ? bf16_to_f(col[(size_t)k * a.r_k]) : 0.f;
+  }
+  {  // the group's queries: 16-byte loads, all in flight together (G*d/8 <= 128)
+    const uint4* q8 = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + g * G) * d);
+    for (int i = tid; i < G * d / 8; i += kFoldThreads) {
+      const uint4 w = q8[i];
+      float4* dst = reinterpret_cast<float4*>(qs + 8 * i);
+      dst[0] = make_float4(bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y));
+      dst[1] = make_float4(bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w));
+    }
+  }
   named_bar_sync(bar, kFoldThreads);
   float acc[8];
 #pragma unroll
   for (int h = 0; h < 8; ++h) acc[h] = 0.f;
-  if (j < a.r_v) {  // row j of P_K, this quarter: n contiguous bf16 (16-byte aligned)
-    const uint4* row = reinterpret_cast<const uint4*>(a.P_K + ((size_t)g * a.r_v + j) * d + i0);
-#pragma unroll 4
-    for (int c = 0; c < n / 8; ++c) {
-      const uint4 w = row[c];
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  if (is_p) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c >= n / 8) break;
+      const uint32_t ws[4] = {prow[c].x, prow[c].y, prow[c].z, prow[c].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float p0 = bf16lo(ws[e]), p1 = bf16hi(ws[e]);
         const int ii = i0 + c * 8 + 2 * e;
 #pragma unroll
         for (int h = 0; h < 8; ++h)
-          if (h < G) acc[h] = fmaf(p1, qs[h * d + ii + 1], fmaf(p0, qs[h * d + ii], acc[h]));
+          if (h < G) {
+            const float2 qv = *reinterpret_cast<const float2*>(qs + h * d + ii);
+            acc[h] = fmaf(p1, qv.y, fmaf(p0, qv.x, acc[h]));
+          }
       }
     }
-  } else if (j < rq) {  // column j - r_v of U_K, this quarter (coalesced across lanes)
-    const uint16_t* col = a.U_K + (size_t)g * d * a.r_k + (j - a.r_v);
-#pragma unroll 8
-    for (int i = i0; i < i0 + n; ++i) {
-      const float u = bf16_to_f(col[(size_t)i * a.r_k]);
+  } else if (is_u) {
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+      if (k >= n) break;
 #pragma unroll
       for (int h = 0; h < 8; ++h)
-        if (h < G) acc[h] = fmaf(u, qs[h * d + i], acc[h]);
+        if (h < G) {
+          const float4 qv = *reinterpret_cast<const float4*>(qs + h * d + i0 + k);
+          acc[h] = fmaf(ucol[k + 3], qv.w,
+                        fmaf(ucol[k + 2], qv.z, fmaf(ucol[k + 1], qv.y, fmaf(ucol[k], qv.x, acc[h]))));
+        }
     }
   }
 #pragma unroll
