@@ -375,6 +375,7 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d->d));
   a.status = status;
   if (attend_mma_supported(a.G, a.d, a.r_v, a.S)) {
+    a.early_inputs = cnt != nullptr;  // inside the fused step: follows the selection launch
     if (!cnt) {  // a standalone call: the arrival counters start from zero here
       cnt = reinterpret_cast<int*>(ws + L.counters);
       if (cudaMemsetAsync(cnt, 0, (size_t)L.n_att_cnt * 4, st) != cudaSuccess)

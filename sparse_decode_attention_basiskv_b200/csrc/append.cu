@@ -39,6 +39,9 @@ __global__ void __launch_bounds__(kPrologueMaxThreads)
   __shared__ float vs[kAppendThreads], ks[kAppendThreads], zs[kAppendThreads],
       rs[kAppendThreads];
   const int bg = blockIdx.x, grp = threadIdx.x / kFoldThreads, gtid = threadIdx.x % kFoldThreads;
+  // One wave of blocks: the scoring grid may take the rest of the SMs and
+  // start on its page loads while the fold finishes.
+  pdl_launch_dependents();
   if (bg == 0 && counters) {
     pdl_wait();
     for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;

@@ -567,7 +567,7 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
     const long c = ((x + 1) * C - 1) / total;
     return (int)(c < C - 1 ? c : C - 1);
   };
-  pdl_wait();
+  if (!a.early_inputs) pdl_wait();
 
   long seg = total * blockIdx.x / C;
   while (seg < c_end) {
@@ -596,7 +596,6 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
       }
     };
     int T = a.seq_lens[b] + a.len_offset;
-    fetch_ids(0);
     // the group's queries as B fragments, shared by the CTA's warps: entry
     // [k][lane (r, c)] holds head r, columns 32k + 8c .. +7 (zero past G)
     for (int i = tid; i < NKC * 32; i += kAmThreads) {
@@ -605,6 +604,8 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
                           a.q + ((size_t)b * a.Hq + g * G + r) * D + 32 * k + 8 * cc))
                     : make_uint4(0u, 0u, 0u, 0u);
     }
+    pdl_wait();  // the selection is the previous launch's output
+    fetch_ids(0);
     T = T < 0 ? 0 : T;
     const int nsel = min(a.top_k, (T + S - 1) / S);
     const long valid_end = bg0 + (long)nsel * TP;  // units past it have no page

@@ -128,6 +128,10 @@ struct AttendArgs {
   int* cnt;
   float* a_lat;
   uint16_t* a_bf16;
+  // Set when this launch follows another kernel of the same call (never a
+  // caller's kernel): the queries and lengths are then read before the
+  // grid-dependency wait.
+  int early_inputs;
 };
 int attend_pages_per_split(int S);
 // Plain-load tensor-core attention with its own merge (needs a.cnt zeroed,

@@ -728,7 +728,10 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RV, RK, S>()))
   const int lane = threadIdx.x & 31, lr = lane >> 2, lc = lane & 3;
   const long wid = (long)blockIdx.x * kRmWarps + (threadIdx.x >> 5);
   const long nw = (long)gridDim.x * kRmWarps;
-  pdl_wait();
+  // The grid-dependency wait comes only before the folded queries are read:
+  // the lengths, the block table and the caches are not written by the fold
+  // launch this kernel follows, so the first pages are requested while it
+  // finishes.
 
   // Work: pages (sequence, KV head, logical page) in that order; warp wid
   // takes a contiguous range.  Pages past a sequence's length are skipped.
@@ -792,6 +795,7 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RV, RK, S>()))
   uint4* qa = rm_frags + (size_t)(threadIdx.x >> 5) * (SETS * NC * 2 * 32) + lane;
   int frag_bg = -1;
   auto load_frags = [&](int bb, int gg) {
+    pdl_wait();
     const float* qs = a.qt + ((size_t)bb * a.Hkv + gg) * G * RQ;
 #pragma unroll
     for (int set = 0; set < SETS; ++set) {
@@ -1053,6 +1057,7 @@ __global__ void __launch_bounds__(kSelThreads)
   __shared__ float vs[kAppendThreads], ks[kAppendThreads], zs[kAppendThreads],
       rs[kAppendThreads];
   const int nsel = s.B * s.Hkv;
+  pdl_launch_dependents();  // one wave: the attention CTAs may take the free SMs
   if ((int)blockIdx.x < nsel) {
     pdl_wait();
     uint32_t* keys = reinterpret_cast<uint32_t*>(sa_dyn);
