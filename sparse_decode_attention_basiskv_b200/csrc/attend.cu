@@ -555,6 +555,9 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
   float* wacc = am_smem;                        // [warp][G][RV] latent sums of the run
   float* wml = am_smem + kAmWarps * G * RV;     // [warp][16]: m of heads 0-7, then l
   uint4* qs = reinterpret_cast<uint4*>(wml + kAmWarps * 16);  // [NKC][lane] query fragments
+  // per-warp ring of two units' Value-latent chunks, [slot][chunk][half][lane]:
+  // each lane copies (cp.async) and later reads only its own 16-byte entries
+  uint4* zring = qs + NKC * 32 + (size_t)(threadIdx.x >> 5) * (2 * NZC * 2 * 32);
   __shared__ int s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, lr = lane >> 2, lc = lane & 3;
   const int S = a.S, TP = S >> 4;
@@ -648,11 +651,13 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
         kx[c][1] = ldg_stream(a.K + (row + 8) * D + 32 * c + 8 * lc);
       }
     };
-    auto load_z = [&](size_t row) {
+    auto load_z = [&](size_t row, int slot) {  // asynchronous, into the warp's ring
 #pragma unroll
       for (int c = 0; c < NZC; ++c) {
-        zx[c][0] = ldg_stream(a.Z + row * RV + 32 * c + 8 * lc);
-        zx[c][1] = ldg_stream(a.Z + (row + 8) * RV + 32 * c + 8 * lc);
+        cp_async16(zring + ((slot * NZC + c) * 2 + 0) * 32 + lane,
+                   a.Z + row * RV + 32 * c + 8 * lc);
+        cp_async16(zring + ((slot * NZC + c) * 2 + 1) * 32 + lane,
+                   a.Z + (row + 8) * RV + 32 * c + 8 * lc);
       }
     };
     int lp_c = -1, pp_c = 0;
@@ -660,16 +665,20 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
       unit_ids(0, lp_c, pp_c);
       const size_t row0 = unit_row(0, pp_c);
       load_k(row0);
-      load_z(row0);
+      load_z(row0, 0);
     }
-    // Unit n computes while unit n + 1 loads: its Keys are requested as soon
-    // as QK has consumed the current ones, its latents after PV.
+    cp_async_commit();
+    // Unit n computes while unit n + 1 loads: its latents are requested
+    // (into shared memory) before unit n starts, its Keys (into registers) as
+    // soon as QK has consumed the current ones.
     for (int n = 0; n < count; ++n) {
       const int tau = (int)(u_first + (long)kAmWarps * n - bg0) % TP;
       const bool more = n + 1 < count;
       int lp_n = -1, pp_n = 0;
       if (more) unit_ids(n + 1, lp_n, pp_n);
       const size_t row_n = more ? unit_row(n + 1, pp_n) : 0;
+      if (more) load_z(row_n, (n + 1) & 1);
+      cp_async_commit();
       // s = [tokens r, r + 8] x [heads 2c, 2c + 1]
       float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -715,6 +724,12 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
       split_bf16x2(p10, p11, wh1, wl1);
       const uint32_t bh0 = movmatrix_trans(wh0), bh1 = movmatrix_trans(wh1);
       const uint32_t bl0 = movmatrix_trans(wl0), bl1 = movmatrix_trans(wl1);
+      cp_async_wait_prior();  // unit n's latents have landed
+#pragma unroll
+      for (int c = 0; c < NZC; ++c) {
+        zx[c][0] = zring[(((n & 1) * NZC + c) * 2 + 0) * 32 + lane];
+        zx[c][1] = zring[(((n & 1) * NZC + c) * 2 + 1) * 32 + lane];
+      }
       // latent rows past the length hold stale data (0 * NaN would poison the sum)
       if (!v0)
 #pragma unroll
@@ -735,10 +750,10 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
           mma_bf16_16816(acc[c][e], t0[2 * e], t0[2 * e + 1], t1[2 * e], t1[2 * e + 1], bl0, bl1);
         }
       }
-      if (more) load_z(row_n);
       lp_c = lp_n;
       pp_c = pp_n;
     }
+    cp_async_wait_all();  // the ring is refilled by the next run
     (void)pp_c;
 
     // ---- the run's warps meet: per-warp state to shared memory
@@ -847,7 +862,8 @@ cudaError_t launch_attend_mma_t(const AttendArgs& a, cudaStream_t st, bool pdl) 
   if (grid > kAmMaxCtas) grid = kAmMaxCtas;
   if (grid > units) grid = units;  // every CTA gets at least one unit
   if (grid < 1) return cudaSuccess;
-  const size_t smem = (size_t)kAmWarps * (G * RV + 16) * sizeof(float) + (D / 32) * 32 * 16;
+  const size_t smem = (size_t)kAmWarps * (G * RV + 16) * sizeof(float) + (D / 32) * 32 * 16 +
+                      (size_t)kAmWarps * 2 * (RV / 32) * 2 * 32 * 16;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(attend_mma_kernel<G, D, RV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

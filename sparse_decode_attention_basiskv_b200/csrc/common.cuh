@@ -283,6 +283,10 @@ __device__ __forceinline__ void cp_async_commit() {
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
+// Waits until at most one committed group of the calling thread is pending.
+__device__ __forceinline__ void cp_async_wait_prior() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
 
 // ------------------------------------------------------------- PDL control
 __device__ __forceinline__ void pdl_wait() {
