@@ -23,7 +23,8 @@ formulas below are the plainest reading of those statements:
   route    khat_t = z_t P_K + e_t U_K^T ;
            score(page) = max over the page's live tokens and over the query
            heads h of the group of  q_h . khat_t
-  select   keep the sink page 0 and the newest page P-1, then the best
+  select   keep the sink page 0 and the newest page P-1 (more generally
+           the first n_sink and the last n_recent pages), then the best
            remaining pages by (score desc, page index asc), k pages in all,
            listed ascending and padded with -1
   attend   s_t = q_h . K_t / sqrt(d) over the selected pages' live tokens;
@@ -81,13 +82,21 @@ def predicted_keys(z: np.ndarray, e: np.ndarray, P_K: np.ndarray,
 
 
 def page_scores(q_group: np.ndarray, z: np.ndarray, e: np.ndarray,
-                P_K: np.ndarray, U_K: np.ndarray, T: int, S: int) -> np.ndarray:
+                P_K: np.ndarray, U_K: np.ndarray, T: int, S: int,
+                r_b: int | None = None, r_q: int | None = None) -> np.ndarray:
     """Routing score of every page of one (sequence, KV head) group.
 
     q_group [G][d] are the group's query heads; z [>=T][r_v], e [>=T][r_k]
     the cached latents in logical order (only t < T is read).  Page p holds
-    tokens [p*S, min((p+1)*S, T)).  Returns float64 [P], P = ceil(T/S)."""
-    khat = predicted_keys(z[:T], e[:T], P_K, U_K)
+    tokens [p*S, min((p+1)*S, T)).  Returns float64 [P], P = ceil(T/S).
+
+    A narrower router (Table 4: routing reads r_b of the r_V latent
+    dimensions and the residual code; Table 9's B16R16 router) reads only
+    z[:, :r_b] and e[:, :r_q]: its predicted key is
+    z[:, :r_b] P_K[:r_b] + e[:, :r_q] U_K[:, :r_q]^T.  None = full width."""
+    r_b = z.shape[1] if r_b is None else r_b
+    r_q = e.shape[1] if r_q is None else r_q
+    khat = predicted_keys(z[:T, :r_b], e[:T, :r_q], P_K[:r_b], U_K[:, :r_q])
     logits = q_group @ khat.T  # [G][T]
     P = -(-T // S)
     out = np.empty(P)
@@ -100,15 +109,19 @@ def page_scores(q_group: np.ndarray, z: np.ndarray, e: np.ndarray,
 # (2b) page selection — sink + newest always kept; top-k pages (the pages'
 #      Table 9 caption uses a routed budget plus a recent window).
 # --------------------------------------------------------------------------
-def select_pages(scores, top_k: int) -> tuple:
+def select_pages(scores, top_k: int, n_sink: int = 1, n_recent: int = 1) -> tuple:
     """Choose top_k pages of one group.
 
     scores: the group's P page scores; they are rounded to float32 here
-    because the choice is taken in the kernel's precision.  Returns
-    (sel, near_tie): sel is an int32 array of length top_k, ascending, padded
-    with -1; near_tie is True when the last chosen and the first rejected
-    non-forced page have float32 scores within 1e-4 relative of each other
-    (a slot whose order rounding may decide)."""
+    because the choice is taken in the kernel's precision.  The first
+    n_sink pages and the last n_recent pages are always kept (the default
+    keeps the sink page 0 and the newest page; Table 9's budget is a routed
+    part plus a recent window); the other top_k - n_sink - n_recent slots go
+    to the best remaining pages.  Returns (sel, near_tie): sel is an int32
+    array of length top_k, ascending, padded with -1; near_tie is True when
+    the last chosen and the first rejected non-forced page have float32
+    scores within 1e-4 relative of each other (a slot whose order rounding
+    may decide)."""
     s = np.asarray(scores, dtype=np.float32).astype(np.float64)
     s[s == 0.0] = 0.0  # -0 and +0 compare equal and rank by index
     P = len(s)
@@ -116,9 +129,10 @@ def select_pages(scores, top_k: int) -> tuple:
     if top_k >= P:
         sel[:P] = np.arange(P)
         return sel, False
-    forced = [0, P - 1]
+    assert n_sink + n_recent <= top_k
+    forced = list(range(n_sink)) + list(range(P - n_recent, P))
     need = top_k - len(forced)
-    cand = np.arange(1, P - 1)
+    cand = np.arange(n_sink, P - n_recent)
     order = cand[np.lexsort((cand, -s[cand]))]  # score desc, then index asc
     chosen = order[:need]
     near_tie = False
@@ -184,15 +198,18 @@ def outproj(a: np.ndarray, W_fold: np.ndarray) -> np.ndarray:
 def decode_sequence(q: np.ndarray, K: np.ndarray, Z: np.ndarray, E: np.ndarray,
                     T: int, S: int, top_k: int, P_K: np.ndarray,
                     U_K: np.ndarray, W_fold: np.ndarray,
-                    k_new=None, v_new=None, A_V=None) -> dict:
+                    k_new=None, v_new=None, A_V=None, r_b=None, r_q=None,
+                    n_sink: int = 1, n_recent: int = 1) -> dict:
     """Decode step for one sequence.
 
     q [Hq][d]; K [Hkv][cap][d], Z [Hkv][cap][r_v], E [Hkv][cap][r_k] logical
     caches holding T tokens; factors per KV head (A_V [Hkv][d][r_v],
     P_K [Hkv][r_v][d], U_K [Hkv][d][r_k]); W_fold [Hq][r_v][hidden].
     With k_new / v_new ([Hkv][d]) the token is appended first and the step
-    attends over T + 1 tokens.  Returns a dict with the appended state, the
-    scores, the selection, near-tie flags, a and y."""
+    attends over T + 1 tokens.  r_b, r_q, n_sink, n_recent: the router's
+    widths and the kept pages (page_scores, select_pages).  Returns a dict
+    with the appended state, the scores, the selection, near-tie flags, a
+    and y."""
     Hkv = K.shape[0]
     Hq = q.shape[0]
     G = Hq // Hkv
@@ -213,8 +230,8 @@ def decode_sequence(q: np.ndarray, K: np.ndarray, Z: np.ndarray, E: np.ndarray,
     scores, sels, ties, a = [], [], [], np.zeros((Hq, Z.shape[2]))
     for g in range(Hkv):
         qg = q[g * G:(g + 1) * G]
-        sc = page_scores(qg, Z[g], E[g], P_K[g], U_K[g], T, S)
-        sel, tie = select_pages(sc, top_k)
+        sc = page_scores(qg, Z[g], E[g], P_K[g], U_K[g], T, S, r_b, r_q)
+        sel, tie = select_pages(sc, top_k, n_sink, n_recent)
         a[g * G:(g + 1) * G], _ = attend(qg, K[g], Z[g], sel, T, S)
         scores.append(sc)
         sels.append(sel)

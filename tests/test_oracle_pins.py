@@ -53,6 +53,34 @@ def test_select_matches_brute_force(P):
             assert got == valid[0]
 
 
+@pytest.mark.parametrize("P", range(1, 10))
+def test_select_sink_and_recent_windows_brute_force(P):
+    """The first n_sink and last n_recent pages are forced; the rest of the
+    budget goes to the unique dominating set of the middle pages."""
+    rng = np.random.default_rng(100 + P)
+    for trial in range(15):
+        s = rng.integers(-2, 3, size=P).astype(np.float64)
+        for n_sink, n_recent in [(0, 1), (1, 2), (2, 1), (2, 3), (0, 3)]:
+            for k in range(n_sink + n_recent, P + 2):
+                if k < 1:
+                    continue
+                sel, _ = O.select_pages(s, k, n_sink, n_recent)
+                got = [int(p) for p in sel if p >= 0]
+                if k >= P:
+                    assert got == list(range(P))
+                    continue
+                forced = set(range(n_sink)) | set(range(P - n_recent, P))
+                cand = [p for p in range(P) if p not in forced]
+                need = k - len(forced)
+                valid = []
+                for chosen in itertools.combinations(cand, need):
+                    rest = [u for u in cand if u not in chosen]
+                    if all(_dominates(s, c, u) for c in chosen for u in rest):
+                        valid.append(sorted(forced | set(chosen)))
+                assert len(valid) == 1
+                assert got == valid[0]
+
+
 def test_select_near_tie_flag():
     s = np.array([0.0, 5.0, 3.0, 3.0000001, 1.0, 0.0])
     _, tie = O.select_pages(s, 4)  # last chosen 3.0000001 vs rejected 3.0
@@ -102,6 +130,38 @@ def test_identity_factors_closed_form():
 
 
 # ---------------------------------------------------------------- routing
+@pytest.mark.parametrize("r_b,r_q", [(4, 3), (8, 0), (0, 5), (8, 5)])
+def test_narrow_router_equals_zeroed_factors(r_b, r_q):
+    """A router reading z[:, :r_b] and e[:, :r_q] scores exactly like the
+    full router with P_K rows >= r_b and U_K columns >= r_q set to zero."""
+    rng = np.random.default_rng(7 + r_b * 10 + r_q)
+    d, r_v, r_k, G, T, S = 16, 8, 5, 3, 45, 8
+    P_K = rng.standard_normal((r_v, d))
+    U_K = _orth(rng, d, r_k)
+    z = rng.standard_normal((T, r_v))
+    e = rng.standard_normal((T, r_k))
+    q = rng.standard_normal((G, d))
+    narrow = O.page_scores(q, z, e, P_K, U_K, T, S, r_b, r_q)
+    Pz, Uz = P_K.copy(), U_K.copy()
+    Pz[r_b:] = 0.0
+    Uz[:, r_q:] = 0.0
+    np.testing.assert_allclose(narrow, O.page_scores(q, z, e, Pz, Uz, T, S), atol=1e-12)
+    full = O.page_scores(q, z, e, P_K, U_K, T, S, r_v, r_k)
+    np.testing.assert_array_equal(full, O.page_scores(q, z, e, P_K, U_K, T, S))
+
+
+def test_narrow_router_ignores_unread_dimensions():
+    """Latent dims >= r_b and residual dims >= r_q carry all the signal: the
+    narrow router's scores are exactly zero."""
+    rng = np.random.default_rng(8)
+    d, r_v, r_k, T, S = 16, 8, 6, 30, 8
+    z = np.zeros((T, r_v))
+    z[:, 4:] = rng.standard_normal((T, 4))
+    e = np.zeros((T, r_k))
+    e[:, 2:] = rng.standard_normal((T, 4))
+    sc = O.page_scores(rng.standard_normal((2, d)), z, e, rng.standard_normal((r_v, d)),
+                       _orth(rng, d, r_k), T, S, 4, 2)
+    np.testing.assert_array_equal(sc, np.zeros_like(sc))
 @pytest.mark.parametrize("T,S", [(37, 8), (32, 8), (5, 16), (64, 16)])
 def test_page_scores_closed_form(T, S):
     """khat_t = c_t u and q_h = alpha_h u  =>  score(p) = max_{t,h} alpha_h c_t.
