@@ -54,7 +54,8 @@ def algorithmic_bytes(wl, T: int, append: bool = True) -> dict:
     S = wl.page_size
     P = -(-T // S)
     sel = min(wl.top_k, P)
-    route = wl.B * wl.Hkv * T * (wl.r_v + wl.r_k) * 2
+    r = wl.router  # the router reads z[:, :r_b] and e[:, :r_q]
+    route = wl.B * wl.Hkv * T * (r["r_b"] + r["r_q"]) * 2
     attend = wl.B * wl.Hkv * sel * S * (wl.d + wl.r_v) * 2
     outproj = wl.Hq * wl.r_v * wl.hidden * 2
     small = (wl.B * wl.Hq * wl.d * 2                      # q (fold + attend)
@@ -162,8 +163,10 @@ def oracle_group_step(wl, s) -> None:
     E = c["E"].copy()
     K = c["K"].copy()
     Z[T], E[T], K[T] = O.to_bf16(z[0]), O.to_bf16(e[0]), s["k"]
-    sc = O.page_scores(s["q"], Z, E, f["P_K"][0], f["U_K"][0], T + 1, wl.page_size)
-    sel, _ = O.select_pages(sc, wl.top_k)
+    r = wl.router
+    sc = O.page_scores(s["q"], Z, E, f["P_K"][0], f["U_K"][0], T + 1, wl.page_size, r["r_b"],
+                       r["r_q"])
+    sel, _ = O.select_pages(sc, wl.top_k, r["n_sink"], r["n_recent"])
     a, _ = O.attend(s["q"], K, Z, sel, T + 1, wl.page_size)
     W = O.fold_outproj(f["B_V"][:1], f["W_O"][:wl.G * wl.d], wl.G)
     O.outproj(a, W)
@@ -311,7 +314,7 @@ def run_gpu(args) -> None:
     r1.record(stream)
     torch.cuda.synchronize()
     route_ms = r0.elapsed_time(r1) / reps
-    route_bytes = wl.B * wl.Hkv * T_r * (wl.r_v + wl.r_k) * 2
+    route_bytes = wl.B * wl.Hkv * T_r * (wl.router["r_b"] + wl.router["r_q"]) * 2
     peak, peak_kind = measured_peak()
     achieved = route_bytes / (route_ms / 1e3) / 1e9
     traffic = None
@@ -322,7 +325,7 @@ def run_gpu(args) -> None:
         # DRAM traffic of one launch, captured with ncu on a smaller batch of the
         # same kernel (B = 4) and scaled by the units processed: traffic grows in
         # proportion to the pages streamed.
-        if tr.get("kernel_source_sha") == _route_source_sha():
+        if tr.get("kernel_source_sha") == _route_source_sha() and WL is synth.LLAMA8B_T32K_B16:
             traffic = tr["traffic_over_algorithmic"] * route_bytes
 
     # ------------------------------------ end to end through the public API
@@ -413,7 +416,13 @@ def main():
                     help="override the batch (smaller cases for profiling)")
     ap.add_argument("--context", type=int, default=0,
                     help="override the context length (smaller cases for profiling)")
+    ap.add_argument("--router", default="full", choices=["full", "b16r16"],
+                    help="full: the default router (all latent and residual dims, sink + "
+                         "newest page); b16r16: the pages' narrow router and budget")
     args = ap.parse_args()
+    global WL
+    if args.router == "b16r16":
+        WL = synth.LLAMA8B_T32K_B16_B16R16
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -43,6 +43,11 @@
  *   K_cache [num_phys_pages][Hkv][S][d]    exact Keys        (Table 4 "Exact Key")
  *   Z_cache [num_phys_pages][Hkv][S][r_v]  Value latents z   (Table 4 "Compressed Value")
  *   E_cache [num_phys_pages][Hkv][S][r_k]  Key residuals e   (Table 4 "Residual code")
+ *   With a narrow router (route_r_v < r_v or route_r_k < r_k, below), each
+ *   Z (E) tile stores its rows' first route_r_v (route_r_k) columns first,
+ *   [S][route_r_v] then [S][r_v - route_r_v], so the router reads one
+ *   contiguous block per tile (HBM fetches whole lines: a strided subset of
+ *   each row would cost the full row).
  *   block_table int32 [B][max_pages_per_seq]: logical page -> physical page.
  *   Token t of sequence b lives in physical page block_table[b][t / S], row
  *   t % S.
@@ -58,7 +63,9 @@
  *
  * Supported shapes: d in {64, 128}; r_v in {32, 64, 96, 128}; r_k in
  * {16, 32, 64}; G in {1, 2, 4, 8}; S in {8, 16, 32}; H a multiple of 128;
- * top_k >= 2.  Other shapes return BASISKV_ERR_UNSUPPORTED_SHAPE.
+ * top_k >= 2.  A router narrower than (r_v, r_k) is supported for G in
+ * {4, 8}, r_k = 32 and S in {16, 32} (widths 16 or 32 each).  Other shapes
+ * return BASISKV_ERR_UNSUPPORTED_SHAPE.
  */
 #ifndef BASISKV_H_
 #define BASISKV_H_
@@ -89,6 +96,22 @@ typedef struct basiskv_dims {
   int32_t page_size;         /* S, tokens per page */
   int32_t max_pages_per_seq; /* length of one block-table row */
   int32_t num_phys_pages;    /* pages held by each physical cache */
+  /* Router and budget (zero-initialised = the default router):
+   *   route_r_v     latent dims the router reads, z[:, :route_r_v] with
+   *                 P_K[:route_r_v] (Table 4: routing reads r_b of r_V);
+   *                 0 = all r_v, else a multiple of 16 <= r_v
+   *   route_r_k     residual dims the router reads, e[:, :route_r_k] with
+   *                 U_K[:, :route_r_k]; 0 = all r_k, else a multiple of 16
+   *                 <= r_k
+   *   sink_pages    leading pages always selected; 0 = 1 (the sink page),
+   *                 negative = none
+   *   recent_pages  trailing pages always selected (a recent window, Table
+   *                 9's budget); 0 = 1 (the newest page), else >= 1
+   * top_k counts the forced pages; top_k >= sink + recent. */
+  int32_t route_r_v;
+  int32_t route_r_k;
+  int32_t sink_pages;
+  int32_t recent_pages;
 } basiskv_dims;
 
 enum basiskv_status {

@@ -127,6 +127,12 @@ bool pdl_enabled() {
   return on;
 }
 
+// Effective router widths and kept pages (zero fields select the defaults).
+int route_rv(const basiskv_dims* d) { return d->route_r_v ? d->route_r_v : d->r_v; }
+int route_rk(const basiskv_dims* d) { return d->route_r_k ? d->route_r_k : d->r_k; }
+int sink_pages(const basiskv_dims* d) { return d->sink_pages == 0 ? 1 : (d->sink_pages < 0 ? 0 : d->sink_pages); }
+int recent_pages(const basiskv_dims* d) { return d->recent_pages == 0 ? 1 : d->recent_pages; }
+
 int check_dims(const basiskv_dims* d) {
   if (!d) return BASISKV_ERR_INVALID_ARG;
   if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->max_pages_per_seq < 1 ||
@@ -149,16 +155,24 @@ int check_dims(const basiskv_dims* d) {
     return BASISKV_ERR_UNSUPPORTED_SHAPE;
   if ((long long)d->max_pages_per_seq * d->page_size >= (1ll << 30))
     return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  // router widths and kept pages
+  if (d->route_r_v < 0 || d->route_r_v > d->r_v || d->route_r_v % 16) return BASISKV_ERR_INVALID_ARG;
+  if (d->route_r_k < 0 || d->route_r_k > d->r_k || d->route_r_k % 16) return BASISKV_ERR_INVALID_ARG;
+  if (d->recent_pages < 0) return BASISKV_ERR_INVALID_ARG;
+  if ((route_rv(d) < d->r_v || route_rk(d) < d->r_k) &&
+      !route_narrow_supported(G, d->r_v, d->r_k, route_rv(d), route_rk(d), d->page_size))
+    return BASISKV_ERR_UNSUPPORTED_SHAPE;
   return BASISKV_OK;
 }
 
 int check_len_topk(const basiskv_dims* d, int top_k, int max_seq_len) {
-  if (top_k < 2) return BASISKV_ERR_INVALID_ARG;
+  if (top_k < 2 || top_k < sink_pages(d) + recent_pages(d)) return BASISKV_ERR_INVALID_ARG;
   if (max_seq_len < 1 || (long long)max_seq_len > (long long)d->max_pages_per_seq * d->page_size)
     return BASISKV_ERR_INVALID_ARG;
-  // Page selection keeps one 32-bit key per page in shared memory.
+  // Page selection keeps a 32-bit key and a block-table entry per page in
+  // shared memory.
   const long long P = (max_seq_len + d->page_size - 1) / d->page_size;
-  if (P * 4 > 200 * 1024) return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  if (P * 8 > 200 * 1024) return BASISKV_ERR_UNSUPPORTED_SHAPE;
   return BASISKV_OK;
 }
 
@@ -254,6 +268,8 @@ AppendArgs make_append_args(const basiskv_dims* d, const basiskv_bf16* k_new,
   a.max_pages = d->max_pages_per_seq;
   a.num_phys = d->num_phys_pages;
   a.status = device_status_ptr();
+  a.zsplit = route_rv(d);
+  a.esplit = route_rk(d);
   return a;
 }
 
@@ -330,11 +346,13 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   r.max_seq_len = max_seq_len;
   r.len_offset = len_offset;
   r.status = status;
+  r.rb = route_rv(d);
+  r.rq = route_rk(d);
   rc = launch_status(launch_route_scores(r, tmZ, tmE, wz, we, st, pdl));
   if (rc || !sel) return rc;  // no selection requested: scores only
   SelectArgs s{scores, seq_lens, sel, d->B, d->Hkv, d->page_size, d->max_pages_per_seq, top_k,
                max_seq_len, len_offset, block_table,
-               reinterpret_cast<int32_t*>(ws + L.selp)};
+               reinterpret_cast<int32_t*>(ws + L.selp), sink_pages(d), recent_pages(d)};
   if (with_append) return launch_status(launch_select_append(s, *with_append, st, pdl));
   return launch_status(launch_select(s, st, pdl));
 }
@@ -358,6 +376,7 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
   a.block_table = block_table;
   a.sel = sel;
   a.sel_phys = sel_phys;
+  a.zsplit = route_rv(d);
   a.partial = reinterpret_cast<float*>(ws + L.partial);
   a.B = d->B;
   a.Hq = d->Hq;

@@ -560,7 +560,7 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
   uint4* zring = qs + NKC * 32 + (size_t)(threadIdx.x >> 5) * (2 * NZC * 2 * 32);
   __shared__ int s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, lr = lane >> 2, lc = lane & 3;
-  const int S = a.S, TP = S >> 4;
+  const int S = a.S, TP = S >> 4, logS = 31 - __clz(S);
   const int upb = a.top_k * TP;  // units per (sequence, KV head)
   const long total = (long)a.B * a.Hkv * upb;
   const int C = gridDim.x;
@@ -652,12 +652,17 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm) attend_mma_kernel(At
       }
     };
     auto load_z = [&](size_t row, int slot) {  // asynchronous, into the warp's ring
+      // tiles may store their first zsplit columns first (a narrow router's)
+      const size_t tile = row >> logS;
+      const int trow = (int)(row & (S - 1));
+      const uint16_t* zt = a.Z + tile * S * RV;
 #pragma unroll
       for (int c = 0; c < NZC; ++c) {
+        const int col = 32 * c + 8 * lc;
         cp_async16(zring + ((slot * NZC + c) * 2 + 0) * 32 + lane,
-                   a.Z + row * RV + 32 * c + 8 * lc);
+                   zt + split_off(trow, col, S, RV, a.zsplit));
         cp_async16(zring + ((slot * NZC + c) * 2 + 1) * 32 + lane,
-                   a.Z + (row + 8) * RV + 32 * c + 8 * lc);
+                   zt + split_off(trow + 8, col, S, RV, a.zsplit));
       }
     };
     int lp_c = -1, pp_c = 0;

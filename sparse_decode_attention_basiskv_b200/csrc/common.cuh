@@ -196,6 +196,14 @@ __device__ __forceinline__ uint16_t f_to_bf16(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
+// Element offset of (row t, column j) inside one (page, KV head) tile of S
+// rows of width W whose first F columns are stored first: [S][F] then
+// [S][W - F].  F == W is the plain [S][W] tile.  (A narrow router's columns
+// are kept contiguous this way.)
+__host__ __device__ __forceinline__ size_t split_off(int t, int j, int S, int W, int F) {
+  return j < F ? (size_t)t * F + j : (size_t)S * F + (size_t)t * (W - F) + (j - F);
+}
+
 // ------------------------------------------------- warp-level tensor cores
 // mma.m16n8k16 with bf16 operands and fp32 accumulation: d += A (16x16, row)
 // * B (16x8, col).  Lane l holds A rows l/4, l/4+8 (columns 2(l%4)+{0,1},
@@ -286,6 +294,14 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // Waits until at most one committed group of the calling thread is pending.
 __device__ __forceinline__ void cp_async_wait_prior() {
   asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
+// 8-byte form, written straight into the low half of dst (no register copy
+// that would wait for the load).
+__device__ __forceinline__ void ldg_stream8(uint4& dst, const void* p) {
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+               : "=r"(dst.x), "=r"(dst.y)
+               : "l"(p));
 }
 
 // ------------------------------------------------------------- PDL control

@@ -41,6 +41,7 @@ struct AppendArgs {
   uint16_t* E_cache;
   int B, Hkv, d, r_v, r_k, S, max_pages, num_phys;
   unsigned int* status;
+  int zsplit, esplit;  // Z / E tiles store their first zsplit / esplit columns first
 };
 cudaError_t launch_append_small(const AppendArgs& a, cudaStream_t st, bool pdl);
 
@@ -86,7 +87,11 @@ struct RouteArgs {
   int B, Hkv, G, r_v, r_k, S, max_pages, num_phys, max_seq_len;
   int len_offset;  // added to seq_lens[b] (tokens appended in this step, not yet counted)
   unsigned int* status;
+  int rb, rq;  // widths the router reads: z[:, :rb], e[:, :rq]
 };
+// Whether the plain-load scoring kernel has an instance for a router
+// narrower than the cached widths.
+bool route_narrow_supported(int G, int r_v, int r_k, int rb, int rq, int S);
 cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
                                 const CUtensorMap& tmE, int wz, int we, cudaStream_t st,
                                 bool pdl);
@@ -101,6 +106,7 @@ struct SelectArgs {
   // done here, so the attention kernel reads page ids in one round trip).
   const int32_t* block_table;
   int32_t* sel_phys;  // [B][Hkv][top_k] or null
+  int n_sink, n_recent;  // leading / trailing pages always kept
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
 // The selection together with a one-token append (a.n_new == 1), whose
@@ -132,6 +138,7 @@ struct AttendArgs {
   // caller's kernel): the queries and lengths are then read before the
   // grid-dependency wait.
   int early_inputs;
+  int zsplit;  // Z tiles store their first zsplit columns first
 };
 int attend_pages_per_split(int S);
 // Plain-load tensor-core attention with its own merge (needs a.cnt zeroed,

@@ -236,8 +236,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int i = 0; i < 8; ++i)
         pk[i] = (uint32_t)f_to_bf16(v[2 * i]) | ((uint32_t)f_to_bf16(v[2 * i + 1]) << 16);
       // columns c0..c0+15 are z (c < r_v) or e (c >= r_v); r_v, r_k are multiples of 16
-      uint16_t* dst = c0 < a.r_v ? a.Z_cache + slot * a.r_v + c0
-                                 : a.E_cache + slot * a.r_k + (c0 - a.r_v);
+      const size_t tile = slot / a.S;
+      const int trow = (int)(slot - tile * a.S);
+      uint16_t* dst =
+          c0 < a.r_v
+              ? a.Z_cache + tile * a.S * a.r_v + split_off(trow, c0, a.S, a.r_v, a.zsplit)
+              : a.E_cache + tile * a.S * a.r_k +
+                    split_off(trow, c0 - a.r_v, a.S, a.r_k, a.esplit);
       uint4* d4 = reinterpret_cast<uint4*>(dst);
       d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);

@@ -451,8 +451,9 @@ __global__ void __launch_bounds__(kRsThreads, kRsCtasPerSm)
 }
 
 // -------------------------------------------------------- page selection
-// Per (sequence, KV head): sink page 0 and newest page P-1 always; the other
-// top_k - 2 slots go to the best remaining pages by (score desc, index asc),
+// Per (sequence, KV head): the first n_sink and the last n_recent pages
+// always (by default the sink page 0 and the newest page P-1); the other
+// slots go to the best remaining pages by (score desc, index asc),
 // found exactly with an MSB-first radix select over order-preserving 32-bit
 // keys; ties at the threshold are taken in index order.  Output ascending.
 constexpr int kSelThreads = 512;
@@ -509,7 +510,8 @@ __device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32
   int32_t* out = a.sel + (size_t)bg * a.top_k;
   int32_t* outp = a.sel_phys ? a.sel_phys + (size_t)bg * a.top_k : nullptr;
   const int32_t* bt = a.block_table + (size_t)b * a.max_pages;
-  const float* sc = a.scores + (size_t)bg * a.max_pages + 1;
+  const int ns = a.n_sink, nr = a.n_recent;  // forced leading / trailing pages
+  const float* sc = a.scores + (size_t)bg * a.max_pages + ns;  // candidate i = page ns + i
   // The length, the first batch of scores and the block-table row are
   // requested together (up to the longest possible context; what lies past
   // this sequence's pages is dropped): one memory round trip, not two.
@@ -519,7 +521,7 @@ __device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int i = u * NT + tid;
-    v[u] = i < P_max - 1 ? __ldcg(sc + i) : 0.f;
+    v[u] = i < P_max - ns ? __ldcg(sc + i) : 0.f;
     t[u] = (outp && i < P_max) ? bt[i] : 0;
   }
   T = T < 0 ? 0 : (T > a.max_seq_len ? a.max_seq_len : T);
@@ -531,7 +533,7 @@ __device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32
     }
     return;
   }
-  const int n = P - 2, need = a.top_k - 2;
+  const int n = P - ns - nr, need = a.top_k - ns - nr;  // n >= 1: P > top_k >= ns + nr
   for (int base = 0; base < P; base += 8 * NT) {  // batches of eight loads a thread
     if (base > 0) {
 #pragma unroll
@@ -629,23 +631,21 @@ __device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32
   const int before = block_excl_scan<NT>((n_gt << 16) | n_eq, ss.sh, &total);
   if (need > 0) {
     int r = before & 0xffff;
-    int pos = 1 + (before >> 16) + min(r, rem);
+    int pos = ns + (before >> 16) + min(r, rem);
     for (int i = i0; i < i1; ++i) {
       const uint32_t k = keys[i];
       if ((k > thr) || (k == thr && r < rem)) {
-        if (outp) outp[pos] = tbl[i + 1];
-        out[pos++] = i + 1;
+        if (outp) outp[pos] = tbl[i + ns];
+        out[pos++] = i + ns;
       }
       r += k == thr;
     }
   }
-  if (tid == 0) {
-    out[0] = 0;
-    out[a.top_k - 1] = P - 1;
-    if (outp) {
-      outp[0] = tbl[0];
-      outp[a.top_k - 1] = tbl[P - 1];
-    }
+  for (int i = tid; i < ns + nr; i += NT) {  // the forced pages, first and last
+    const int slot = i < ns ? i : a.top_k - nr + (i - ns);
+    const int page = i < ns ? i : P - nr + (i - ns);
+    out[slot] = page;
+    if (outp) outp[slot] = tbl[page];
   }
 }
 
@@ -673,9 +673,11 @@ constexpr int kRmWarps = kRmThreads / 32;
 // and accumulators fit, else two.  Measured at the 32K-context, B = 16
 // Llama-8B shape: one page in flight per warp with 24 warps per SM beats two
 // pages per warp with 16 warps (136 vs 153 us for fold + scoring + select).
-template <int G, int RV, int RK, int S>
+template <int G, int RB, int RQ, int S>
 __host__ __device__ constexpr int rm_ctas_per_sm() {
-  return (S / 8) * ((RV + RK) / 32) * 4 + (S / 8) * (G == 8 ? 2 : 1) * 4 <= 40 ? 3 : 2;
+  return (S / 8) * ((RB + 31) / 32 + (RQ + 31) / 32) * 4 + (S / 8) * (G == 8 ? 2 : 1) * 4 <= 40
+             ? 3
+             : 2;
 }
 
 // A-operand row r of row set `set`: the head it holds (-1: a zero row) and
@@ -719,11 +721,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return (uint32_t)f_to_bf16(lo) | ((uint32_t)f_to_bf16(hi) << 16);
 }
 
-template <int G, int RV, int RK, int S, int PW>
-__global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RV, RK, S>()))
+// RV, RK: the cache rows' widths (pitches); RB <= RV, RQ <= RK: the columns
+// the router reads (multiples of 16).  A row's read columns form chunks of 32
+// (lane c loads columns 8c .. 8c+7, 16 bytes: two k-steps of the MMA) and at
+// most one 16-column tail chunk (lane c loads columns 4c .. 4c+3, 8 bytes:
+// one k-step), so every lane loads and every loaded byte is used.
+template <int G, int RV, int RK, int RB, int RQ, int S, int PW>
+__global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S>()))
     route_mma_kernel(RouteArgs a) {
   extern __shared__ uint4 rm_frags[];
-  constexpr int NZ = RV / 32, NC = (RV + RK) / 32, NT = S / 8, RQ = RV + RK;
+  constexpr int NZF = RB / 32, NZH = (RB % 32) / 16, NEF = RQ / 32, NEH = (RQ % 32) / 16;
+  constexpr int NCZ = NZF + NZH, NC = NCZ + NEF + NEH, NT = S / 8, RQ_ = RV + RK;
+  constexpr int ZP = RB, EP = RQ;  // row pitch of the columns read (== RV, RK when full)
   constexpr int SETS = G == 8 ? 2 : 1;
   const int lane = threadIdx.x & 31, lr = lane >> 2, lc = lane & 3;
   const long wid = (long)blockIdx.x * kRmWarps + (threadIdx.x >> 5);
@@ -796,7 +805,7 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RV, RK, S>()))
   int frag_bg = -1;
   auto load_frags = [&](int bb, int gg) {
     pdl_wait();
-    const float* qs = a.qt + ((size_t)bb * a.Hkv + gg) * G * RQ;
+    const float* qs = a.qt + ((size_t)bb * a.Hkv + gg) * G * RQ_;
 #pragma unroll
     for (int set = 0; set < SETS; ++set) {
       int h0, p0, h1, p1;
@@ -806,10 +815,16 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RV, RK, S>()))
       for (int c = 0; c < NC; ++c)
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-          const int col = 32 * c + 8 * lc + 4 * k;
+          const bool zc = c < NCZ;  // latent chunk, else residual chunk
+          const int cc = zc ? c : c - NCZ;
+          const bool half = zc ? (NZH && cc == NZF) : (NEH && cc == NEF);
+          const bool live = !(half && k == 1);  // a 16-column chunk has one k-step
+          const int col = (zc ? 0 : RV) + 32 * cc + (half ? 4 * lc : 8 * lc + 4 * k);
           const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4 v0 = h0 >= 0 ? *reinterpret_cast<const float4*>(qs + h0 * RQ + col) : z4;
-          const float4 v1 = h1 >= 0 ? *reinterpret_cast<const float4*>(qs + h1 * RQ + col) : z4;
+          const float4 v0 =
+              (h0 >= 0 && live) ? *reinterpret_cast<const float4*>(qs + h0 * RQ_ + col) : z4;
+          const float4 v1 =
+              (h1 >= 0 && live) ? *reinterpret_cast<const float4*>(qs + h1 * RQ_ + col) : z4;
           qa[((set * NC + c) * 2 + k) * 32] =
               make_uint4(pack_bf16x2(bf16_part(v0.x, p0), bf16_part(v0.y, p0)),
                          pack_bf16x2(bf16_part(v1.x, p1), bf16_part(v1.y, p1)),
@@ -838,15 +853,28 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RV, RK, S>()))
           if (lane == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
           pp = 0;  // the page's score is flagged garbage
         }
-        const size_t row = ((size_t)pp * a.Hkv + g) * S + lr;
-        const uint16_t* zr = a.Z + row * RV + 8 * lc;
-        const uint16_t* er = a.E + row * RK + 8 * lc;
+        // a narrow router's columns lead each tile: [S][RB] then the rest
+        const size_t tile = (size_t)pp * a.Hkv + g;
+        const uint16_t* zr = a.Z + tile * S * RV + lr * ZP + 8 * lc;
+        const uint16_t* er = a.E + tile * S * RK + lr * EP + 8 * lc;
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
 #pragma unroll
-          for (int c = 0; c < NZ; ++c) x[k][t][c] = ldg_stream(zr + t * 8 * RV + 32 * c);
+          for (int c = 0; c < NCZ; ++c) {
+            if (NZH && c == NZF) {
+              ldg_stream8(x[k][t][c], zr - 4 * lc + t * 8 * ZP + 32 * c);
+            } else {
+              x[k][t][c] = ldg_stream(zr + t * 8 * ZP + 32 * c);
+            }
+          }
 #pragma unroll
-          for (int c = NZ; c < NC; ++c) x[k][t][c] = ldg_stream(er + t * 8 * RK + 32 * (c - NZ));
+          for (int c = NCZ; c < NC; ++c) {
+            if (NEH && c - NCZ == NEF) {
+              ldg_stream8(x[k][t][c], er - 4 * lc + t * 8 * EP + 32 * (c - NCZ));
+            } else {
+              x[k][t][c] = ldg_stream(er + t * 8 * EP + 32 * (c - NCZ));
+            }
+          }
         }
         advance();
         skip();
@@ -874,7 +902,9 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RV, RK, S>()))
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
             mma_bf16_16816(acc[t][set], f0.x, f0.y, f0.z, f0.w, x[k][t][c].x, x[k][t][c].y);
-            mma_bf16_16816(acc[t][set], f1.x, f1.y, f1.z, f1.w, x[k][t][c].z, x[k][t][c].w);
+            const bool half = c < NCZ ? (NZH && c == NZF) : (NEH && c - NCZ == NEF);
+            if (!half)
+              mma_bf16_16816(acc[t][set], f1.x, f1.y, f1.z, f1.w, x[k][t][c].z, x[k][t][c].w);
           }
         }
       float best = -INFINITY;
@@ -974,26 +1004,58 @@ cudaError_t launch_route_rs(const RouteArgs& a, const CUtensorMap& tmZ, const CU
                   pdl, tmZ, tmE, a, geo);
 }
 
-template <int G, int RV, int RK, int S>
+// Pages a warp loads before scoring them: the full-width router keeps one
+// page (24 load registers at r_v 64) in flight with 24 warps per SM; a narrow
+// router's pages are a few registers each, so a warp batches more of them to
+// keep about as many bytes in flight.
+template <int RB, int RQ, int S>
+constexpr int rm_pages_per_batch() {
+  return (S / 8) * (4 * (RB / 32 + RQ / 32) + 2 * ((RB % 32) / 16 + (RQ % 32) / 16)) <= 8
+             ? 3
+             : ((S / 8) * (4 * (RB / 32 + RQ / 32) + 2 * ((RB % 32) / 16 + (RQ % 32) / 16)) <= 12
+                    ? 2
+                    : 1);
+}
+
+template <int G, int RV, int RK, int RB, int RQ, int S>
 cudaError_t launch_route_mma(const RouteArgs& a, cudaStream_t st, bool pdl) {
-  constexpr int PW = 1;
+  constexpr int PW = rm_pages_per_batch<RB, RQ, S>();
+  constexpr int NC = (RB + 31) / 32 + (RQ + 31) / 32;
   const int P_max = (a.max_seq_len + S - 1) / S;
   const long pages = (long)a.B * a.Hkv * P_max;
-  long grid = (long)num_sms() * rm_ctas_per_sm<G, RV, RK, S>();
+  long grid = (long)num_sms() * rm_ctas_per_sm<G, RB, RQ, S>();
   const long need = (pages + kRmWarps - 1) / kRmWarps;
   if (grid > need) grid = need;
   if (grid < 1) grid = 1;
-  const size_t smem = (size_t)kRmWarps * (G == 8 ? 2 : 1) * ((RV + RK) / 32) * 2 * 32 * 16;
+  const size_t smem = (size_t)kRmWarps * (G == 8 ? 2 : 1) * NC * 2 * 32 * 16;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(route_mma_kernel<G, RV, RK, S, PW>,
+    cudaError_t e = cudaFuncSetAttribute(route_mma_kernel<G, RV, RK, RB, RQ, S, PW>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_k(route_mma_kernel<G, RV, RK, S, PW>, dim3((unsigned)grid), dim3(kRmThreads),
-                  smem, st, pdl, a);
+  return launch_k(route_mma_kernel<G, RV, RK, RB, RQ, S, PW>, dim3((unsigned)grid),
+                  dim3(kRmThreads), smem, st, pdl, a);
 }
 
+// Narrow routers with an instance: (G, S) in {(4, 16), (8, 32)}, r_k 32,
+// r_v in {64, 96}, widths 16 or 32 each.
+#define BKV_RM_NARROW(X)                                                            \
+  X(4, 64, 32, 16, 16, 16) X(4, 64, 32, 16, 32, 16) X(4, 64, 32, 32, 16, 16)        \
+  X(4, 64, 32, 32, 32, 16) X(4, 96, 32, 16, 16, 16) X(4, 96, 32, 16, 32, 16)        \
+  X(4, 96, 32, 32, 16, 16) X(4, 96, 32, 32, 32, 16) X(8, 64, 32, 16, 16, 32)        \
+  X(8, 64, 32, 16, 32, 32) X(8, 64, 32, 32, 16, 32) X(8, 64, 32, 32, 32, 32)        \
+  X(8, 96, 32, 16, 16, 32) X(8, 96, 32, 16, 32, 32) X(8, 96, 32, 32, 16, 32)        \
+  X(8, 96, 32, 32, 32, 32)
+
 }  // namespace
+
+bool route_narrow_supported(int G, int r_v, int r_k, int rb, int rq, int S) {
+#define BKV_RMQ(GG, V, K, RB_, RQ_, SS) \
+  if (G == GG && r_v == V && r_k == K && rb == RB_ && rq == RQ_ && S == SS) return true;
+  BKV_RM_NARROW(BKV_RMQ)
+#undef BKV_RMQ
+  return false;
+}
 
 cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl) {
   const int G = a.Hq / a.Hkv;
@@ -1005,10 +1067,19 @@ cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl) {
 cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
                                 const CUtensorMap& tmE, int wz, int we, cudaStream_t st,
                                 bool pdl) {
+  if ((a.rb != a.r_v || a.rq != a.r_k) && !(a.Z && a.E)) return cudaErrorNotSupported;
   if (a.Z && a.E) {
+    if (a.rb != a.r_v || a.rq != a.r_k) {  // a narrow router
+#define BKV_RMN(GG, V, K, RB_, RQ_, SS)                                                    \
+  if (a.G == GG && a.r_v == V && a.r_k == K && a.rb == RB_ && a.rq == RQ_ && a.S == SS) \
+    return launch_route_mma<GG, V, K, RB_, RQ_, SS>(a, st, pdl);
+      BKV_RM_NARROW(BKV_RMN)
+#undef BKV_RMN
+      return cudaErrorNotSupported;
+    }
 #define BKV_RM(GG, V, K, SS)                                     \
   if (a.G == GG && a.r_v == V && a.r_k == K && a.S == SS) \
-    return launch_route_mma<GG, V, K, SS>(a, st, pdl);
+    return launch_route_mma<GG, V, K, V, K, SS>(a, st, pdl);
     BKV_RM(4, 64, 32, 16)
     BKV_RM(4, 96, 32, 16)
     BKV_RM(4, 128, 32, 16)

@@ -106,10 +106,13 @@ __device__ __forceinline__ void append_block(const AppendArgs& a, int g, int j, 
     if (tid == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
     return;
   }
-  const size_t slot = ((size_t)pp * a.Hkv + g) * a.S + pos % a.S;
-  if (tid < d) a.K_cache[slot * d + tid] = kb;
-  if (tid < r_v) a.Z_cache[slot * r_v + tid] = f_to_bf16(zv);
-  if (tid < r_k) a.E_cache[slot * r_k + tid] = f_to_bf16(ev);
+  const size_t tile = (size_t)pp * a.Hkv + g;
+  const int row = pos % a.S;
+  if (tid < d) a.K_cache[(tile * a.S + row) * d + tid] = kb;
+  if (tid < r_v)
+    a.Z_cache[tile * a.S * r_v + split_off(row, tid, a.S, r_v, a.zsplit)] = f_to_bf16(zv);
+  if (tid < r_k)
+    a.E_cache[tile * a.S * r_k + split_off(row, tid, a.S, r_k, a.esplit)] = f_to_bf16(ev);
 }
 
 // Folds the queries of (sequence, KV head) bg for outputs 32*yblk .. +31:

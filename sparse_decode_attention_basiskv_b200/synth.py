@@ -68,6 +68,11 @@ class Workload:
     prefill_tokens: int = 0  # tokens of one prefill chunk (sequence 0)
     layers: int = 1
     steps: int = 1
+    # router and budget (0 = the defaults: full widths, sink page, newest page)
+    route_r_v: int = 0
+    route_r_k: int = 0
+    sink_pages: int = 0
+    recent_pages: int = 0
 
     @property
     def G(self) -> int:
@@ -86,11 +91,25 @@ class Workload:
     def pages_capacity(self) -> int:
         return -(-self.capacity_tokens() // self.page_size)
 
+    @property
+    def router(self) -> dict:
+        """Effective router widths and forced pages."""
+        return {"r_b": self.route_r_v or self.r_v, "r_q": self.route_r_k or self.r_k,
+                "n_sink": 1 if self.sink_pages == 0 else max(self.sink_pages, 0),
+                "n_recent": self.recent_pages or 1}
+
+    def tile_lead(self) -> dict:
+        """Columns stored first in each cache tile (a narrow router's)."""
+        return {"Z": self.route_r_v or self.r_v, "E": self.route_r_k or self.r_k}
+
     def describe(self) -> dict:
-        return {k: getattr(self, k) for k in (
+        out = {k: getattr(self, k) for k in (
             "name", "B", "Hq", "Hkv", "d", "hidden", "T", "page_size", "r_v",
             "r_k", "top_k", "append_tokens", "prefill_tokens", "layers",
             "steps")}
+        if (self.route_r_v, self.route_r_k, self.sink_pages, self.recent_pages) != (0, 0, 0, 0):
+            out["router"] = self.router
+        return out
 
 
 # The five workloads.  Names say what they are; sizes follow the pages' model
@@ -105,6 +124,12 @@ LLAMA8B_T32K_B16 = Workload("llama8b_layer_b16_t32k_v64_append1", B=16, Hq=32,
                             Hkv=8, d=128, hidden=4096, T=32768, page_size=16,
                             r_v=64, r_k=32, top_k=128, n_planted=8, seed=2,
                             append_tokens=1)
+# The headline shape with the pages' narrow router and budget (Table 9's
+# B16R16 router: 16 latent + 16 residual dimensions read per token; 2048
+# routed tokens plus a 64-token recent window, no sink page), at page 16.
+LLAMA8B_T32K_B16_B16R16 = replace(
+    LLAMA8B_T32K_B16, name="llama8b_layer_b16_t32k_v64_router_b16r16_recent64", top_k=132,
+    route_r_v=16, route_r_k=16, sink_pages=-1, recent_pages=4)
 QWEN32B_T64K_B8 = Workload("qwen32b_layer_b8_t64k_v96_prefill4k", B=8, Hq=64,
                            Hkv=8, d=128, hidden=5120, T=65536, page_size=32,
                            r_v=96, r_k=32, top_k=64, n_planted=8, seed=3,
@@ -250,10 +275,34 @@ def block_table(wl: Workload, device="cpu") -> torch.Tensor:
     return perm.view(wl.B, pc).to(device)
 
 
+def split_tiles(tiles: torch.Tensor, lead: int) -> torch.Tensor:
+    """Tiles [..., S, r] stored with their first `lead` columns first: the
+    memory of each tile holds [S][lead] then [S][r - lead] (the layout the
+    C-ABI uses for a narrow router's columns).  lead == r: unchanged."""
+    S, r = tiles.shape[-2:]
+    if lead == r:
+        return tiles
+    flat = torch.cat([tiles[..., :lead].reshape(*tiles.shape[:-2], S * lead),
+                      tiles[..., lead:].reshape(*tiles.shape[:-2], S * (r - lead))], -1)
+    return flat.reshape(tiles.shape)
+
+
+def unsplit_tiles(tiles: torch.Tensor, lead: int) -> torch.Tensor:
+    """Inverse of split_tiles."""
+    S, r = tiles.shape[-2:]
+    if lead == r:
+        return tiles
+    flat = tiles.reshape(*tiles.shape[:-2], S * r)
+    a = flat[..., :S * lead].reshape(*tiles.shape[:-2], S, lead)
+    b = flat[..., S * lead:].reshape(*tiles.shape[:-2], S, r - lead)
+    return torch.cat([a, b], -1)
+
+
 def paginate(logical: torch.Tensor, table: torch.Tensor, page_size: int,
-             num_phys: int) -> torch.Tensor:
+             num_phys: int, lead: int = 0) -> torch.Tensor:
     """Scatter a logical cache [B][Hkv][cap][r] into the paged layout
-    [num_phys][Hkv][page_size][r] through the block table."""
+    [num_phys][Hkv][page_size][r] through the block table (each tile with
+    its first `lead` columns first when 0 < lead < r)."""
     B, Hkv, cap, r = logical.shape
     pc = table.shape[1]
     pad = pc * page_size - cap
@@ -261,6 +310,7 @@ def paginate(logical: torch.Tensor, table: torch.Tensor, page_size: int,
         logical = torch.cat([logical, torch.full((B, Hkv, pad, r), FILLER,
                             dtype=logical.dtype, device=logical.device)], 2)
     tiles = logical.view(B, Hkv, pc, page_size, r).permute(0, 2, 1, 3, 4)
+    tiles = split_tiles(tiles, lead or r)
     out = torch.full((num_phys, Hkv, page_size, r), FILLER, dtype=logical.dtype,
                      device=logical.device)
     out[table.long().reshape(-1).to(logical.device)] = tiles.reshape(B * pc, Hkv, page_size, r)
@@ -293,7 +343,8 @@ class Problem:
 
     def paged(self) -> dict:
         n = self.wl.B * self.wl.pages_capacity()
-        return {k: paginate(v, self.table.to(v.device), self.wl.page_size, n)
+        lead = self.wl.tile_lead()
+        return {k: paginate(v, self.table.to(v.device), self.wl.page_size, n, lead.get(k, 0))
                 for k, v in self.cache.items()}
 
 

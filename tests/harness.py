@@ -64,9 +64,10 @@ def oracle_route(pb, b: int, g: int, T: int, cache=None) -> tuple:
     f = factors_np(pb)
     c = pb.cache if cache is None else cache
     qg = np64(pb.q[b, g * wl.G:(g + 1) * wl.G])
+    r = wl.router
     sc = O.page_scores(qg, np64(c["Z"][b, g]), np64(c["E"][b, g]), f["P_K"][g], f["U_K"][g], T,
-                       wl.page_size)
-    sel, tie = O.select_pages(sc, wl.top_k)
+                       wl.page_size, r["r_b"], r["r_q"])
+    sel, tie = O.select_pages(sc, wl.top_k, r["n_sink"], r["n_recent"])
     return sc, sel, tie
 
 
@@ -84,3 +85,14 @@ def compare_selection(gpu_sel: np.ndarray, ref_sel: np.ndarray, tie: bool, stats
 def status_clean():
     flags = bkv.read_device_status()
     assert flags == 0, f"device status bits {flags:#x}"
+
+
+def cache_row(paged, wl, name: str, phys: int, g: int, rows):
+    """Rows of one (page, KV head) tile of a paged cache in logical column
+    order (undoing the narrow router's column split)."""
+    lead = wl.tile_lead().get(name, paged.shape[-1])
+    tiles = synth.unsplit_tiles(paged[phys, g], lead)
+    if tiles.dim() == 2:  # one tile
+        return tiles[rows]
+    return tiles[torch.arange(tiles.shape[0], device=tiles.device),
+                 torch.as_tensor(rows).to(tiles.device)]

@@ -72,6 +72,34 @@ def test_route_rejects_bad_dims(lib, field, value, status):
     assert rc == status
 
 
+@pytest.mark.parametrize("field,value,status", [
+    ("route_r_v", 8, bkv.ERR_INVALID_ARG),      # not a multiple of 16
+    ("route_r_v", 80, bkv.ERR_INVALID_ARG),     # wider than r_v
+    ("route_r_k", -16, bkv.ERR_INVALID_ARG),
+    ("recent_pages", -1, bkv.ERR_INVALID_ARG),
+])
+def test_router_fields_validated(lib, field, value, status):
+    d = _dims(**{field: value})
+    rc = lib.basiskv_route(ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, FAKE, FAKE, FAKE, 8,
+                           None, FAKE, FAKE, 1 << 30, None)
+    assert rc == status
+
+
+def test_narrow_router_shapes_and_budget(lib):
+    # no instance of the scoring kernel for a narrow router at G = 1
+    d = _dims(Hq=2, route_r_v=16)
+    assert lib.basiskv_route(ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, FAKE, FAKE, FAKE, 8,
+                             None, FAKE, FAKE, 1 << 30, None) == bkv.ERR_UNSUPPORTED_SHAPE
+    # the forced pages must fit in top_k
+    d = _dims(route_r_v=16, route_r_k=16, sink_pages=2, recent_pages=4)
+    assert lib.basiskv_route(ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, FAKE, FAKE, FAKE, 5,
+                             None, FAKE, FAKE, 1 << 30, None) == bkv.ERR_INVALID_ARG
+    # a supported narrow router passes validation (then fails on the tiny workspace)
+    d = _dims(route_r_v=16, route_r_k=16, sink_pages=-1, recent_pages=4)
+    assert lib.basiskv_route(ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, FAKE, FAKE, FAKE, 8,
+                             None, FAKE, FAKE, 64, None) == bkv.ERR_WORKSPACE_TOO_SMALL
+
+
 def test_route_rejects_bad_args(lib):
     d = _dims()
     args = [ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, FAKE, FAKE, FAKE, 8, None, FAKE, FAKE,

@@ -8,7 +8,7 @@ import torch
 from oracle import basiskv_oracle as O
 from sparse_decode_attention_basiskv_b200 import synth
 
-from harness import (Y_ABS, Y_REL, ZE_REL, assert_within, compare_selection, factors_np,
+from harness import (cache_row, Y_ABS, Y_REL, ZE_REL, assert_within, compare_selection, factors_np,
                      gpu_layer, np64, status_clean)
 
 pytestmark = pytest.mark.gpu
@@ -31,8 +31,10 @@ def _check_step(pb, layer, y, sel, samples, T_before, k_new=None, v_new=None):
             if k_new is not None:
                 slot = (layer.block_table[b, T_before // wl.page_size].item(), g,
                         T_before % wl.page_size)
-                assert_within(np64(layer.Z[slot]), out["z_new"][g], ZE_REL, what="z")
-                assert_within(np64(layer.E[slot]), out["e_new"][g], ZE_REL, what="e")
+                assert_within(np64(cache_row(layer.Z, wl, "Z", *slot)), out["z_new"][g], ZE_REL,
+                          what="z")
+                assert_within(np64(cache_row(layer.E, wl, "E", *slot)), out["e_new"][g], ZE_REL,
+                          what="e")
         if not out["near_tie"].any():
             assert_within(np64(y[b]), out["y"], Y_REL, Y_ABS, what=f"y b{b}")
     assert stats.get("clean_mismatch", 0) == 0, stats

@@ -9,7 +9,8 @@ import sparse_decode_attention_basiskv_b200 as bkv
 from oracle import basiskv_oracle as O
 from sparse_decode_attention_basiskv_b200 import synth
 
-from harness import (A_REL, S_REL, Y_ABS, Y_REL, ZE_REL, assert_within, compare_selection,
+from harness import (A_REL, S_REL, Y_ABS, Y_REL, ZE_REL, assert_within, cache_row,
+                     compare_selection,
                      factors_np, gpu_layer, np64, oracle_route, status_clean)
 
 pytestmark = pytest.mark.gpu
@@ -27,6 +28,13 @@ SMALL = {
                                           top_k=48),
     "llama_rk64_b2_t1500": synth.with_sizes(synth.LLAMA8B_T4K, B=2, T=1500, r_v=64, r_k=64,
                                             top_k=32),
+    # the pages' narrow router (16 latent + 16 residual dims) with a recent
+    # window of 4 pages and no sink page, at the headline shape
+    "llama_b16r16_b4_t2k": synth.with_sizes(synth.LLAMA8B_T32K_B16_B16R16, B=4, T=2000,
+                                            top_k=24),
+    # a narrow router with the default sink/newest pages, Qwen3-32B shape
+    "qwen_b32r16_b2_t3k": synth.with_sizes(synth.QWEN32B_T64K_B8, B=2, T=3000,
+                                           prefill_tokens=0, route_r_v=32, route_r_k=16),
 }
 
 
@@ -116,12 +124,14 @@ def test_decode_step_with_append(setup):
         c = {k: np64(v[b]) for k, v in pb.cache.items()}
         out = O.decode_sequence(np64(pb.q[b]), c["K"], c["Z"], c["E"], wl.T, wl.page_size,
                                 wl.top_k, f["P_K"], f["U_K"], W, k_new=np64(k_new[b]),
-                                v_new=np64(v_new[b]), A_V=f["A_V"])
+                                v_new=np64(v_new[b]), A_V=f["A_V"], **wl.router)
         # appended state, read back from the paged caches
         for g in range(wl.Hkv):
             slot = (layer.block_table[b, wl.T // wl.page_size].item(), g, wl.T % wl.page_size)
-            assert_within(np64(layer.Z[slot]), out["z_new"][g], ZE_REL, what="z")
-            assert_within(np64(layer.E[slot]), out["e_new"][g], ZE_REL, what="e")
+            assert_within(np64(cache_row(layer.Z, wl, "Z", *slot)), out["z_new"][g], ZE_REL,
+                          what="z")
+            assert_within(np64(cache_row(layer.E, wl, "E", *slot)), out["e_new"][g], ZE_REL,
+                          what="e")
             assert torch.equal(layer.K[slot], k_new[b, g])
             compare_selection(sel[b, g].cpu().numpy(), out["sel"][g], out["near_tie"][g], stats)
         if not out["near_tie"].any():
@@ -260,8 +270,8 @@ def test_prefill_chunk_append(prefolded):
         toks = np.arange(wl.T, wl.T + 4096)
         phys = layer.block_table[b, toks // wl.page_size].long().cpu()
         rows = torch.as_tensor(toks % wl.page_size)
-        assert_within(np64(layer.Z[phys, g, rows]), z_ref, ZE_REL, what="prefill z")
-        assert_within(np64(layer.E[phys, g, rows]), e_ref, ZE_REL, what="prefill e")
+        assert_within(np64(cache_row(layer.Z, wl, "Z", phys, g, rows)), z_ref, ZE_REL, what="prefill z")
+        assert_within(np64(cache_row(layer.E, wl, "E", phys, g, rows)), e_ref, ZE_REL, what="prefill e")
         assert torch.equal(layer.K[phys, g, rows], k[b, :, g])
 
 
