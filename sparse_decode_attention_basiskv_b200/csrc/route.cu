@@ -880,13 +880,9 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S>()))
         skip();
       }
     }
-#pragma unroll
-    for (int k = 0; k < PW; ++k) {
-      if (!uok[k]) continue;
-      if (ubg[k] != frag_bg) {
-        load_frags(ub[k], ug[k]);
-        frag_bg = ubg[k];
-      }
+    // This lane's maximum over page k's live tokens and the group's heads
+    // (the warp reduction follows).
+    auto page_best = [&](int k) -> float {
       float acc[NT][SETS][4];
 #pragma unroll
       for (int t = 0; t < NT; ++t)
@@ -924,8 +920,39 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S>()))
         if (tok < uT[k]) best = fmaxf(best, s0);
         if (tok + 1 < uT[k]) best = fmaxf(best, s1);
       }
-      best = warp_max(best);
-      if (lane == 0) a.scores[(size_t)ubg[k] * a.max_pages + ulp[k]] = best;
+      return best;
+    };
+    bool one_group = true;
+#pragma unroll
+    for (int k = 1; k < PW; ++k) one_group = one_group && (!uok[k] || ubg[k] == ubg[0]);
+    if (one_group) {  // the common case: the batch's pages are scored side by side
+      if (ubg[0] != frag_bg) {
+        load_frags(ub[0], ug[0]);
+        frag_bg = ubg[0];
+      }
+      float best[PW];
+#pragma unroll
+      for (int k = 0; k < PW; ++k) best[k] = uok[k] ? page_best(k) : -INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int k = 0; k < PW; ++k)
+          best[k] = fmaxf(best[k], __shfl_xor_sync(0xffffffffu, best[k], o));
+      if (lane == 0)
+#pragma unroll
+        for (int k = 0; k < PW; ++k)
+          if (uok[k]) a.scores[(size_t)ubg[k] * a.max_pages + ulp[k]] = best[k];
+    } else {  // the batch crosses a group boundary
+#pragma unroll
+      for (int k = 0; k < PW; ++k) {
+        if (!uok[k]) continue;
+        if (ubg[k] != frag_bg) {
+          load_frags(ub[k], ug[k]);
+          frag_bg = ubg[k];
+        }
+        const float best = warp_max(page_best(k));
+        if (lane == 0) a.scores[(size_t)ubg[k] * a.max_pages + ulp[k]] = best;
+      }
     }
   }
 }
