@@ -231,6 +231,20 @@ def run_reference(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------ replicas (N > 1)
+def replica_throughput(local_ms: float, total_bytes: float, dist=None, device="cpu") -> tuple:
+    """Whole-job timing of N independent replicas ("replicas only": the
+    single-GPU step has no exchange): the slowest rank's span, and the bytes
+    of all ranks over it in TB/s.  Returns (ms_max, TB/s)."""
+    t = torch.tensor([float(local_ms)], device=device)
+    world = 1
+    if dist is not None and dist.is_initialized():
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        world = dist.get_world_size()
+    ms_max = float(t.item())
+    return ms_max, world * total_bytes / (ms_max / 1e3) / 1e12
+
+
 # ---------------------------------------------------------------- GPU arm
 def run_gpu(args) -> None:
     import sparse_decode_attention_basiskv_b200 as bkv
@@ -284,13 +298,9 @@ def run_gpu(args) -> None:
     launches = bkv.launch_count() - launches0
     ms = ev0.elapsed_time(ev1)
     assert bkv.read_device_status() == 0
-    ms_t = torch.tensor([ms], device="cuda")
-    if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
     bytes_steps = [algorithmic_bytes(wl, T0 + i + 1) for i in range(W, W + K)]
     total_bytes = sum(b["total"] for b in bytes_steps)
-    value = world * total_bytes / (ms_max / 1e3) / 1e12
+    ms_max, value = replica_throughput(ms, total_bytes, dist, "cuda")
     ms_per_step = ms_max / K
 
     # ------------------------------ roofline: the routing stage, timed alone
@@ -354,10 +364,7 @@ def run_gpu(args) -> None:
         e2e_step(i, T0 + i + 1)
     e1.record(stream)
     barrier()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], device="cuda")
-    if dist is not None:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = world * total_bytes / (float(e2e_ms.item()) / 1e3) / 1e12
+    e2e_ms_max, e2e_value = replica_throughput(e0.elapsed_time(e1), total_bytes, dist, "cuda")
     h2d = (queries[0].numel() + k_steps[0].numel() + v_steps[0].numel()) * 2
     d2h = wl.B * wl.hidden * 2
 
@@ -388,7 +395,7 @@ def run_gpu(args) -> None:
                      "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                      "ms_per_launch": route_ms, "algorithmic_bytes": route_bytes},
         "cpu_baseline": cpu,
-        "e2e": {"value": e2e_value, "unit": "TB/s", "us_per_step": float(e2e_ms.item()) / K * 1e3,
+        "e2e": {"value": e2e_value, "unit": "TB/s", "us_per_step": e2e_ms_max / K * 1e3,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "clocks": clocks.summary(),
