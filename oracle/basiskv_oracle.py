@@ -53,6 +53,19 @@ def to_bf16(x) -> np.ndarray:
     return u.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
+def to_e4m3(x) -> np.ndarray:
+    """Round to FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa
+    bits; largest finite 448, subnormal step 2^-9) to nearest even,
+    saturating to +-448; returned as float64.  Table 13 of the pages stores
+    the caches as FP8 E4M3."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))  # below 2^-6: the subnormal step
+    q = 2.0 ** (e - 3)
+    r = np.minimum(np.round(a / q) * q, 448.0)  # np.round: half to even
+    return np.where(x < 0, -r, r)
+
+
 # --------------------------------------------------------------------------
 # (1) cache append — abstract (the Value is compressed to a latent; a
 #     Key-specific residual keeps the part of the Key the latent cannot
@@ -199,7 +212,7 @@ def decode_sequence(q: np.ndarray, K: np.ndarray, Z: np.ndarray, E: np.ndarray,
                     T: int, S: int, top_k: int, P_K: np.ndarray,
                     U_K: np.ndarray, W_fold: np.ndarray,
                     k_new=None, v_new=None, A_V=None, r_b=None, r_q=None,
-                    n_sink: int = 1, n_recent: int = 1) -> dict:
+                    n_sink: int = 1, n_recent: int = 1, fp8: bool = False) -> dict:
     """Decode step for one sequence.
 
     q [Hq][d]; K [Hkv][cap][d], Z [Hkv][cap][r_v], E [Hkv][cap][r_k] logical
@@ -207,9 +220,10 @@ def decode_sequence(q: np.ndarray, K: np.ndarray, Z: np.ndarray, E: np.ndarray,
     P_K [Hkv][r_v][d], U_K [Hkv][d][r_k]); W_fold [Hq][r_v][hidden].
     With k_new / v_new ([Hkv][d]) the token is appended first and the step
     attends over T + 1 tokens.  r_b, r_q, n_sink, n_recent: the router's
-    widths and the kept pages (page_scores, select_pages).  Returns a dict
-    with the appended state, the scores, the selection, near-tie flags, a
-    and y."""
+    widths and the kept pages (page_scores, select_pages).  fp8: the caches
+    hold E4M3 values (the appended K, z and e are stored through to_e4m3
+    instead of K as given and z, e through to_bf16).  Returns a dict with the
+    appended state, the scores, the selection, near-tie flags, a and y."""
     Hkv = K.shape[0]
     Hq = q.shape[0]
     G = Hq // Hkv
@@ -220,9 +234,10 @@ def decode_sequence(q: np.ndarray, K: np.ndarray, Z: np.ndarray, E: np.ndarray,
         for g in range(Hkv):
             z, e = append_latents(k_new[g][None], v_new[g][None], A_V[g],
                                   P_K[g], U_K[g])
-            Z[g, T] = to_bf16(z[0])
-            E[g, T] = to_bf16(e[0])
-            K[g, T] = k_new[g]
+            store = to_e4m3 if fp8 else to_bf16
+            Z[g, T] = store(z[0])
+            E[g, T] = store(e[0])
+            K[g, T] = to_e4m3(k_new[g]) if fp8 else k_new[g]
             zs.append(z[0])
             es.append(e[0])
         out["z_new"], out["e_new"] = np.stack(zs), np.stack(es)

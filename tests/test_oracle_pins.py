@@ -326,3 +326,25 @@ def test_planted_pages_win_routing(wl):
             sel, _ = O.select_pages(sc, wl.top_k)
             want = set(pb.used_pages[b, g * wl.G:(g + 1) * wl.G].reshape(-1).tolist())
             assert want <= set(sel.tolist())
+
+
+# ---------------------------------------------------------------- FP8 cache
+def test_to_e4m3_matches_torch_in_range():
+    """Every value of a dense grid over +-448 (ties included) rounds as
+    torch's float8_e4m3fn conversion does."""
+    rng = np.random.default_rng(12)
+    grid = [rng.uniform(-448, 448, 20000), rng.standard_normal(20000),
+            rng.standard_normal(5000) * 1e-3]
+    # exact halfway points between neighbouring E4M3 values, and the values
+    vals = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    vals = np.sort(vals[np.isfinite(vals)])
+    grid += [vals, (vals[1:] + vals[:-1]) / 2]
+    x = np.concatenate(grid)
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(O.to_e4m3(x.astype(np.float32)), ref)
+
+
+def test_to_e4m3_saturates_and_keeps_steps():
+    np.testing.assert_array_equal(O.to_e4m3([500.0, -1e6, 449.0]), [448.0, -448.0, 448.0])
+    np.testing.assert_array_equal(O.to_e4m3([2.0 ** -9, 2.0 ** -10, 1.0625, 1.09375]),
+                                  [2.0 ** -9, 0.0, 1.0, 1.125])
