@@ -55,8 +55,9 @@ def algorithmic_bytes(wl, T: int, append: bool = True) -> dict:
     P = -(-T // S)
     sel = min(wl.top_k, P)
     r = wl.router  # the router reads z[:, :r_b] and e[:, :r_q]
-    route = wl.B * wl.Hkv * T * (r["r_b"] + r["r_q"]) * 2
-    attend = wl.B * wl.Hkv * sel * S * (wl.d + wl.r_v) * 2
+    cb = 1 if wl.cache_fp8 else 2  # bytes per cached element (E4M3 or bf16)
+    route = wl.B * wl.Hkv * T * (r["r_b"] + r["r_q"]) * cb
+    attend = wl.B * wl.Hkv * sel * S * (wl.d + wl.r_v) * cb
     outproj = wl.Hq * wl.r_v * wl.hidden * 2
     small = (wl.B * wl.Hq * wl.d * 2                      # q (fold + attend)
              + wl.B * wl.hidden * 2                       # y
@@ -66,7 +67,7 @@ def algorithmic_bytes(wl, T: int, append: bool = True) -> dict:
              + wl.B * wl.Hq * wl.r_v * 2 * 2              # latent a (bf16) w + r
              + wl.Hkv * (wl.r_v + wl.r_k) * wl.d * 2)     # P_K, U_K for the fold
     if append:
-        small += (wl.B * wl.Hkv * (2 * wl.d + wl.d + wl.r_v + wl.r_k) * 2
+        small += (wl.B * wl.Hkv * (2 * wl.d * 2 + (wl.d + wl.r_v + wl.r_k) * cb)
                   + wl.Hkv * wl.d * wl.r_v * 2)           # k, v in; K, z, e out; A_V
     return {"route": route, "attend": attend, "outproj": outproj, "small": small,
             "total": route + attend + outproj + small}
@@ -162,7 +163,10 @@ def oracle_group_step(wl, s) -> None:
     Z = c["Z"].copy()
     E = c["E"].copy()
     K = c["K"].copy()
-    Z[T], E[T], K[T] = O.to_bf16(z[0]), O.to_bf16(e[0]), s["k"]
+    if wl.cache_fp8:
+        Z[T], E[T], K[T] = O.to_e4m3(z[0]), O.to_e4m3(e[0]), O.to_e4m3(s["k"])
+    else:
+        Z[T], E[T], K[T] = O.to_bf16(z[0]), O.to_bf16(e[0]), s["k"]
     r = wl.router
     sc = O.page_scores(s["q"], Z, E, f["P_K"][0], f["U_K"][0], T + 1, wl.page_size, r["r_b"],
                        r["r_q"])
@@ -324,7 +328,8 @@ def run_gpu(args) -> None:
     r1.record(stream)
     torch.cuda.synchronize()
     route_ms = r0.elapsed_time(r1) / reps
-    route_bytes = wl.B * wl.Hkv * T_r * (wl.router["r_b"] + wl.router["r_q"]) * 2
+    route_bytes = (wl.B * wl.Hkv * T_r * (wl.router["r_b"] + wl.router["r_q"])
+                   * (1 if wl.cache_fp8 else 2))
     peak, peak_kind = measured_peak()
     achieved = route_bytes / (route_ms / 1e3) / 1e9
     traffic = None
@@ -379,7 +384,8 @@ def run_gpu(args) -> None:
         "metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
         "tokens_per_s": world * wl.B / (ms_per_step / 1e3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 caches, f16 x f16 -> f32" if wl.cache_fp8 else "bf16",
         "data": "synthetic (seeded generators; planted-page queries)",
         "config": {"workload": WL.name if (wl.B, wl.T) == (WL.B, WL.T) else
                    f"{WL.name} at B={wl.B}, T={wl.T}",
@@ -406,7 +412,7 @@ def run_gpu(args) -> None:
 def _route_source_sha() -> str:
     import hashlib
     h = hashlib.sha256()
-    for n in ("route.cu", "common.cuh"):
+    for n in ("route.cu", "route_mma.cuh", "common.cuh"):
         with open(os.path.join(ROOT, "sparse_decode_attention_basiskv_b200", "csrc", n), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -426,10 +432,14 @@ def main():
     ap.add_argument("--router", default="full", choices=["full", "b16r16"],
                     help="full: the default router (all latent and residual dims, sink + "
                          "newest page); b16r16: the pages' narrow router and budget")
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "e4m3"],
+                    help="element type of the K, Z and E caches")
     args = ap.parse_args()
     global WL
     if args.router == "b16r16":
         WL = synth.LLAMA8B_T32K_B16_B16R16
+    if args.cache == "e4m3":
+        WL = synth.with_sizes(WL, cache_fp8=1, name=WL.name + "_e4m3")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

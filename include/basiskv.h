@@ -112,6 +112,22 @@ typedef struct basiskv_dims {
   int32_t route_r_k;
   int32_t sink_pages;
   int32_t recent_pages;
+  /* Cache element type (Table 13 stores the caches as FP8 E4M3):
+   *   0  K_cache, Z_cache and E_cache hold bf16 (the layouts above)
+   *   1  they hold FP8 E4M3 bytes (1 sign, 4 exponent bits with bias 7, 3
+   *      mantissa bits; largest finite value 448) in the same layouts, one
+   *      byte per element; pass the byte buffers through the bf16 pointer
+   *      parameters.  Every write rounds to nearest even and saturates to
+   *      +-448.  Supported when the router has an E4M3 instance (G in {4,
+   *      8}, r_k = 32, r_v in {64, 96, 128} at full width for S in {16, 32};
+   *      the narrow routers listed below) and the attention has one (G in
+   *      {4, 8}, S in {16, 32}); otherwise BASISKV_ERR_UNSUPPORTED_SHAPE.
+   *      The routing and attention kernels widen the bytes to f16 exactly
+   *      and multiply them by f16 copies of the queries, each query group
+   *      (routing) or head (attention) first scaled by a power of two that
+   *      is divided out of the scores, so queries of any fp32 magnitude
+   *      keep about 22 (routing) or all 8 (attention) significant bits. */
+  int32_t cache_fp8;
 } basiskv_dims;
 
 enum basiskv_status {

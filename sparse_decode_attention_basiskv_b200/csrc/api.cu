@@ -162,6 +162,12 @@ int check_dims(const basiskv_dims* d) {
   if ((route_rv(d) < d->r_v || route_rk(d) < d->r_k) &&
       !route_narrow_supported(G, d->r_v, d->r_k, route_rv(d), route_rk(d), d->page_size))
     return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  // cache element type
+  if (d->cache_fp8 != 0 && d->cache_fp8 != 1) return BASISKV_ERR_INVALID_ARG;
+  if (d->cache_fp8 &&
+      !(route_fp8_supported(G, d->r_v, d->r_k, route_rv(d), route_rk(d), d->page_size) &&
+        attend_mma_fp8_supported(G, d->d, d->r_v, d->page_size)))
+    return BASISKV_ERR_UNSUPPORTED_SHAPE;
   return BASISKV_OK;
 }
 
@@ -270,6 +276,7 @@ AppendArgs make_append_args(const basiskv_dims* d, const basiskv_bf16* k_new,
   a.status = device_status_ptr();
   a.zsplit = route_rv(d);
   a.esplit = route_rk(d);
+  a.fp8 = d->cache_fp8;
   return a;
 }
 
@@ -318,8 +325,9 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   const int wz = z_box_cols(d->r_v), we = e_box_cols(d->r_k);
-  CUtensorMap tmZ, tmE;
-  if (!cache_map(&tmZ, Z_cache, d, d->r_v, wz) || !cache_map(&tmE, E_cache, d, d->r_k, we))
+  CUtensorMap tmZ{}, tmE{};  // bf16 caches only: the E4M3 kernels use plain loads
+  if (!d->cache_fp8 &&
+      (!cache_map(&tmZ, Z_cache, d, d->r_v, wz) || !cache_map(&tmE, E_cache, d, d->r_k, we)))
     return BASISKV_ERR_CUDA;
   float* qt = reinterpret_cast<float*>(ws + L.qt);
   int rc = BASISKV_OK;
@@ -348,6 +356,7 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   r.status = status;
   r.rb = route_rv(d);
   r.rq = route_rk(d);
+  r.fp8 = d->cache_fp8;
   rc = launch_status(launch_route_scores(r, tmZ, tmE, wz, we, st, pdl));
   if (rc || !sel) return rc;  // no selection requested: scores only
   SelectArgs s{scores, seq_lens, sel, d->B, d->Hkv, d->page_size, d->max_pages_per_seq, top_k,
@@ -365,8 +374,9 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   const int wz = z_box_cols(d->r_v);
-  CUtensorMap tmK, tmZ;
-  if (!cache_map(&tmK, K_cache, d, d->d, 64) || !cache_map(&tmZ, Z_cache, d, d->r_v, wz))
+  CUtensorMap tmK{}, tmZ{};  // bf16 caches only: the E4M3 kernel uses plain loads
+  if (!d->cache_fp8 &&
+      (!cache_map(&tmK, K_cache, d, d->d, 64) || !cache_map(&tmZ, Z_cache, d, d->r_v, wz)))
     return BASISKV_ERR_CUDA;
   AttendArgs a{};
   a.q = q;
@@ -377,6 +387,7 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
   a.sel = sel;
   a.sel_phys = sel_phys;
   a.zsplit = route_rv(d);
+  a.fp8 = d->cache_fp8;
   a.partial = reinterpret_cast<float*>(ws + L.partial);
   a.B = d->B;
   a.Hq = d->Hq;

@@ -8,6 +8,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -219,6 +220,17 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The same shape with f16 operands.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                              uint32_t a2, uint32_t a3, uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Four 8x8 b16 matrices; lanes 8i..8i+7 give the row addresses of matrix i.
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
                                             uint32_t& r2, uint32_t& r3) {
@@ -252,6 +264,37 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
   const __nv_bfloat16 l1 = __float2bfloat16_rn(x1 - __bfloat162float(h1));
   hi = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
   lo = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+}
+
+// Splits two fp32 values into f16 pairs hi (rounded) and lo (the rounded
+// remainder): x = hi + lo to about 22 significant bits while |x| stays in
+// the f16 normal range.
+__device__ __forceinline__ void split_f16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const __half2 l = __floats2half2_rn(x0 - __low2float(h), x1 - __high2float(h));
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// ------------------------------------------------------------ FP8 (E4M3)
+// E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; largest
+// finite value 448.  Every E4M3 value is an f16 value, so the widening is
+// exact.  Four bytes (byte 0 = the first column) -> two f16x2 words.
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  asm("{ .reg .b16 a, b;\n\t"
+      "mov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, b; }"
+      : "=r"(lo), "=r"(hi)
+      : "r"(x));
+}
+
+// Two fp32 values -> two E4M3 bytes (x0 in the low byte), rounded to
+// nearest even and saturated to +-448.
+__device__ __forceinline__ uint32_t f_to_e4m3x2(float x0, float x1) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
+  return r;
 }
 
 // 16-byte read-only load of streamed data: not kept in L1 (each byte is used
@@ -302,6 +345,18 @@ __device__ __forceinline__ void ldg_stream8(uint4& dst, const void* p) {
   asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
                : "=r"(dst.x), "=r"(dst.y)
                : "l"(p));
+}
+
+// 4-byte form, into dst.x.
+__device__ __forceinline__ void ldg_stream4(uint4& dst, const void* p) {
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(dst.x) : "l"(p));
+}
+
+// Asynchronous 8-byte global -> shared copy (both addresses 8-byte aligned).
+__device__ __forceinline__ void cp_async8(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
 }
 
 // ------------------------------------------------------------- PDL control

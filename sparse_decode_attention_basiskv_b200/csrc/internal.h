@@ -42,6 +42,7 @@ struct AppendArgs {
   int B, Hkv, d, r_v, r_k, S, max_pages, num_phys;
   unsigned int* status;
   int zsplit, esplit;  // Z / E tiles store their first zsplit / esplit columns first
+  int fp8;  // the three caches hold E4M3 bytes (pointers reinterpreted)
 };
 cudaError_t launch_append_small(const AppendArgs& a, cudaStream_t st, bool pdl);
 
@@ -88,10 +89,14 @@ struct RouteArgs {
   int len_offset;  // added to seq_lens[b] (tokens appended in this step, not yet counted)
   unsigned int* status;
   int rb, rq;  // widths the router reads: z[:, :rb], e[:, :rq]
+  int fp8;     // Z and E hold E4M3 bytes
 };
 // Whether the plain-load scoring kernel has an instance for a router
 // narrower than the cached widths.
 bool route_narrow_supported(int G, int r_v, int r_k, int rb, int rq, int S);
+// Whether it has an instance over E4M3 caches for this router.
+bool route_fp8_supported(int G, int r_v, int r_k, int rb, int rq, int S);
+cudaError_t launch_route_scores_fp8(const RouteArgs& a, cudaStream_t st, bool pdl);
 cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
                                 const CUtensorMap& tmE, int wz, int we, cudaStream_t st,
                                 bool pdl);
@@ -139,12 +144,16 @@ struct AttendArgs {
   // grid-dependency wait.
   int early_inputs;
   int zsplit;  // Z tiles store their first zsplit columns first
+  int fp8;     // K and Z hold E4M3 bytes
 };
 int attend_pages_per_split(int S);
 // Plain-load tensor-core attention with its own merge (needs a.cnt zeroed,
 // a.partial of attend_mma_slots(B, Hkv) * G * (r_v + 2) floats); returns
 // cudaErrorNotSupported for shapes it does not cover.
 bool attend_mma_supported(int G, int d, int r_v, int S);
+// Its E4M3 form (a subset of the shapes above).
+bool attend_mma_fp8_supported(int G, int d, int r_v, int S);
+cudaError_t launch_attend_mma_fp8(const AttendArgs& a, cudaStream_t st, bool pdl);
 int attend_mma_slots(int B, int Hkv);
 cudaError_t launch_attend_mma(const AttendArgs& a, cudaStream_t st, bool pdl);
 cudaError_t launch_attend(const AttendArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmZ,

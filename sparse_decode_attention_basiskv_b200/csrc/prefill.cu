@@ -231,13 +231,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!(ok && live)) continue;
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(rr[i]);
+      const size_t tile = slot / a.S;
+      const int trow = (int)(slot - tile * a.S);
+      if (a.fp8) {  // E4M3 caches: 16 bytes per 16 columns
+        uint32_t pb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          pb[i] = f_to_e4m3x2(v[4 * i], v[4 * i + 1]) |
+                  (f_to_e4m3x2(v[4 * i + 2], v[4 * i + 3]) << 16);
+        uint8_t* dst8 =
+            c0 < a.r_v
+                ? reinterpret_cast<uint8_t*>(a.Z_cache) + tile * a.S * a.r_v +
+                      split_off(trow, c0, a.S, a.r_v, a.zsplit)
+                : reinterpret_cast<uint8_t*>(a.E_cache) + tile * a.S * a.r_k +
+                      split_off(trow, c0 - a.r_v, a.S, a.r_k, a.esplit);
+        *reinterpret_cast<uint4*>(dst8) = make_uint4(pb[0], pb[1], pb[2], pb[3]);
+        continue;
+      }
       uint32_t pk[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         pk[i] = (uint32_t)f_to_bf16(v[2 * i]) | ((uint32_t)f_to_bf16(v[2 * i + 1]) << 16);
       // columns c0..c0+15 are z (c < r_v) or e (c >= r_v); r_v, r_k are multiples of 16
-      const size_t tile = slot / a.S;
-      const int trow = (int)(slot - tile * a.S);
       uint16_t* dst =
           c0 < a.r_v
               ? a.Z_cache + tile * a.S * a.r_v + split_off(trow, c0, a.S, a.r_v, a.zsplit)
@@ -247,10 +262,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
-    if (ok && live) {  // the exact Key, copied as is
+    if (ok && live) {  // the exact Key, copied as is (E4M3: rounded)
       const uint4* src = reinterpret_cast<const uint4*>(a.k_new + ((size_t)r * a.Hkv + g) * d);
-      uint4* dstk = reinterpret_cast<uint4*>(a.K_cache + slot * d);
-      for (int i = 0; i < d / 8; ++i) dstk[i] = src[i];
+      if (a.fp8) {
+        uint2* dstk = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(a.K_cache) + slot * d);
+        for (int i = 0; i < d / 8; ++i) {
+          const uint4 x = src[i];
+          const float2 f0 = bf16x2_to_f2(x.x), f1 = bf16x2_to_f2(x.y), f2 = bf16x2_to_f2(x.z),
+                       f3 = bf16x2_to_f2(x.w);
+          dstk[i] = make_uint2(f_to_e4m3x2(f0.x, f0.y) | (f_to_e4m3x2(f1.x, f1.y) << 16),
+                               f_to_e4m3x2(f2.x, f2.y) | (f_to_e4m3x2(f3.x, f3.y) << 16));
+        }
+      } else {
+        uint4* dstk = reinterpret_cast<uint4*>(a.K_cache + slot * d);
+        for (int i = 0; i < d / 8; ++i) dstk[i] = src[i];
+      }
     }
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");

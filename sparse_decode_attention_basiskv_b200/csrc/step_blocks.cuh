@@ -108,6 +108,20 @@ __device__ __forceinline__ void append_block(const AppendArgs& a, int g, int j, 
   }
   const size_t tile = (size_t)pp * a.Hkv + g;
   const int row = pos % a.S;
+  if (a.fp8) {  // E4M3 caches: one byte per value, rounded to nearest even, saturated
+    if (tid < d)
+      reinterpret_cast<uint8_t*>(a.K_cache)[(tile * a.S + row) * d + tid] =
+          (uint8_t)f_to_e4m3x2(bf16_to_f(kb), 0.f);
+    if (tid < r_v)
+      reinterpret_cast<uint8_t*>(a.Z_cache)[tile * a.S * r_v +
+                                            split_off(row, tid, a.S, r_v, a.zsplit)] =
+          (uint8_t)f_to_e4m3x2(zv, 0.f);
+    if (tid < r_k)
+      reinterpret_cast<uint8_t*>(a.E_cache)[tile * a.S * r_k +
+                                            split_off(row, tid, a.S, r_k, a.esplit)] =
+          (uint8_t)f_to_e4m3x2(ev, 0.f);
+    return;
+  }
   if (tid < d) a.K_cache[(tile * a.S + row) * d + tid] = kb;
   if (tid < r_v)
     a.Z_cache[tile * a.S * r_v + split_off(row, tid, a.S, r_v, a.zsplit)] = f_to_bf16(zv);

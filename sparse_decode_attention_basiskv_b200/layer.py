@@ -44,7 +44,8 @@ class DecodeLayer:
         dims = Dims(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, hidden=wl.hidden, r_v=wl.r_v,
                     r_k=wl.r_k, page_size=wl.page_size, max_pages_per_seq=pc,
                     num_phys_pages=wl.B * pc, route_r_v=wl.route_r_v, route_r_k=wl.route_r_k,
-                    sink_pages=wl.sink_pages, recent_pages=wl.recent_pages)
+                    sink_pages=wl.sink_pages, recent_pages=wl.recent_pages,
+                    cache_fp8=wl.cache_fp8)
         factors = {k: v.to(device).contiguous() for k, v in pb.factors.items()}
         caches = {k: v.contiguous() for k, v in pb.paged().items()}
         return cls(dims, factors, caches, pb.table.to(device).contiguous(),

@@ -73,6 +73,7 @@ class Workload:
     route_r_k: int = 0
     sink_pages: int = 0
     recent_pages: int = 0
+    cache_fp8: int = 0  # 1: the K, Z and E caches hold FP8 E4M3 values
 
     @property
     def G(self) -> int:
@@ -109,6 +110,7 @@ class Workload:
             "steps")}
         if (self.route_r_v, self.route_r_k, self.sink_pages, self.recent_pages) != (0, 0, 0, 0):
             out["router"] = self.router
+        out["cache"] = "e4m3" if self.cache_fp8 else "bf16"
         return out
 
 
@@ -130,6 +132,9 @@ LLAMA8B_T32K_B16 = Workload("llama8b_layer_b16_t32k_v64_append1", B=16, Hq=32,
 LLAMA8B_T32K_B16_B16R16 = replace(
     LLAMA8B_T32K_B16, name="llama8b_layer_b16_t32k_v64_router_b16r16_recent64", top_k=132,
     route_r_v=16, route_r_k=16, sink_pages=-1, recent_pages=4)
+# The headline shape with FP8 E4M3 caches (Table 13's KV format).
+LLAMA8B_T32K_B16_FP8 = replace(LLAMA8B_T32K_B16, name="llama8b_layer_b16_t32k_v64_append1_e4m3",
+                               cache_fp8=1)
 QWEN32B_T64K_B8 = Workload("qwen32b_layer_b8_t64k_v96_prefill4k", B=8, Hq=64,
                            Hkv=8, d=128, hidden=5120, T=65536, page_size=32,
                            r_v=96, r_k=32, top_k=64, n_planted=8, seed=3,
@@ -176,6 +181,21 @@ def make_factors(wl: Workload, layer: int = 0) -> dict:
             "B_V": _bf16(B_V), "W_O": _bf16(W_O)}
 
 
+def as_cache_values(wl: Workload, x: torch.Tensor) -> torch.Tensor:
+    """The values a cache of this workload holds for x, as bf16: x rounded to
+    bf16, or for E4M3 caches to E4M3 (nearest even, clamped to +-448), every
+    E4M3 value being a bf16 value."""
+    if not wl.cache_fp8:
+        return x.bfloat16()
+    return x.float().clamp(-448.0, 448.0).to(torch.float8_e4m3fn).to(torch.bfloat16)
+
+
+def storage(wl: Workload, x: torch.Tensor) -> torch.Tensor:
+    """A cache tensor of as_cache_values in the workload's element type (E4M3
+    bytes or bf16)."""
+    return x.to(torch.float8_e4m3fn) if wl.cache_fp8 else x
+
+
 def _dev_gen(device, seed: int) -> torch.Generator:
     return torch.Generator(device=device).manual_seed(seed)
 
@@ -199,9 +219,9 @@ def make_cache(wl: Workload, factors: dict, device="cpu", layer: int = 0,
         e = torch.randn(Hkv, T, wl.r_k, generator=gen, device=dev).bfloat16()
         noise = torch.randn(Hkv, T, wl.d, generator=gen, device=dev) * 0.1
         k = torch.bmm(z.float(), P_K) + torch.bmm(e.float(), U_K.transpose(1, 2)) + noise
-        Z[i, :, :T] = z
-        E[i, :, :T] = e
-        K[i, :, :T] = k.bfloat16()
+        Z[i, :, :T] = as_cache_values(wl, z)
+        E[i, :, :T] = as_cache_values(wl, e)
+        K[i, :, :T] = as_cache_values(wl, k)
     return {"Z": Z, "E": E, "K": K}
 
 
@@ -344,7 +364,8 @@ class Problem:
     def paged(self) -> dict:
         n = self.wl.B * self.wl.pages_capacity()
         lead = self.wl.tile_lead()
-        return {k: paginate(v, self.table.to(v.device), self.wl.page_size, n, lead.get(k, 0))
+        return {k: storage(self.wl, paginate(v, self.table.to(v.device), self.wl.page_size, n,
+                                             lead.get(k, 0)))
                 for k, v in self.cache.items()}
 
 

@@ -91,8 +91,23 @@ def cache_row(paged, wl, name: str, phys: int, g: int, rows):
     """Rows of one (page, KV head) tile of a paged cache in logical column
     order (undoing the narrow router's column split)."""
     lead = wl.tile_lead().get(name, paged.shape[-1])
-    tiles = synth.unsplit_tiles(paged[phys, g], lead)
+    fp8 = paged.dtype == torch.float8_e4m3fn
+    src = paged.view(torch.uint8) if fp8 else paged  # byte moves only
+    tiles = synth.unsplit_tiles(src[phys, g], lead)
     if tiles.dim() == 2:  # one tile
-        return tiles[rows]
-    return tiles[torch.arange(tiles.shape[0], device=tiles.device),
-                 torch.as_tensor(rows).to(tiles.device)]
+        out = tiles[rows]
+    else:
+        out = tiles[torch.arange(tiles.shape[0], device=tiles.device),
+                    torch.as_tensor(rows).to(tiles.device)]
+    return out.view(torch.float8_e4m3fn).float() if fp8 else out
+
+
+def assert_e4m3_bracket(x, ref, tol, what=""):
+    """x (E4M3 values) is the E4M3 rounding of some value within tol
+    (elementwise absolute) of ref: to_e4m3(ref - tol) <= x <= to_e4m3(ref +
+    tol), to_e4m3 being monotone."""
+    x, ref = np.asarray(x, dtype=np.float64), np.asarray(ref, dtype=np.float64)
+    lo, hi = O.to_e4m3(ref - tol), O.to_e4m3(ref + tol)
+    bad = (x < lo) | (x > hi)
+    assert not bad.any(), (f"{what}: {int(bad.sum())} values outside their E4M3 bracket, "
+                           f"first x={x[bad][0]} ref={ref[bad][0]}")

@@ -148,3 +148,25 @@ def test_other_entry_points_validate(lib):
                                     None) == bkv.ERR_UNSUPPORTED_SHAPE
     flags = ctypes.c_uint32(7)
     assert lib.basiskv_read_device_status(None, None) == bkv.ERR_INVALID_ARG
+
+
+def test_e4m3_cache_validation(lib):
+    """cache_fp8 is 0 or 1; E4M3 caches need an E4M3 router and attention
+    instance (validated before any launch)."""
+    assert bkv.workspace_size(_dims(cache_fp8=1), 8, 1000) > 0          # G 4, r_v 64, S 16
+    assert bkv.workspace_size(_dims(cache_fp8=1, Hq=16, Hkv=2, page_size=32, r_v=96), 8,
+                              1000) > 0                                  # G 8, S 32
+    assert bkv.workspace_size(_dims(cache_fp8=1, route_r_v=16, route_r_k=16, sink_pages=-1,
+                                    recent_pages=4), 8, 1000) > 0        # narrow router
+    assert bkv.workspace_size(_dims(cache_fp8=2), 8, 1000) == 0          # not a type
+    assert bkv.workspace_size(_dims(cache_fp8=-1), 8, 1000) == 0
+    assert bkv.workspace_size(_dims(cache_fp8=1, Hq=2), 8, 1000) == 0   # G 1: no instance
+    assert bkv.workspace_size(_dims(cache_fp8=1, page_size=8), 8, 1000) == 0
+    assert bkv.workspace_size(_dims(cache_fp8=1, r_k=16), 8, 1000) == 0
+    d = _dims(cache_fp8=1, Hq=2)
+    assert lib.basiskv_route(ctypes.byref(d), FAKE, FAKE, 100, FAKE, FAKE, FAKE, FAKE, FAKE, 8,
+                             None, FAKE, FAKE, 1 << 30, None) == bkv.ERR_UNSUPPORTED_SHAPE
+    d = _dims(cache_fp8=3)
+    assert lib.basiskv_decode(ctypes.byref(d), FAKE, None, None, FAKE, 100, FAKE, FAKE, FAKE,
+                              FAKE, FAKE, FAKE, FAKE, FAKE, 8, None, FAKE, FAKE, 1 << 30,
+                              None) == bkv.ERR_INVALID_ARG
