@@ -347,6 +347,16 @@ __device__ __forceinline__ void ldg_stream8(uint4& dst, const void* p) {
                : "l"(p));
 }
 
+// The same forms into a uint2.
+__device__ __forceinline__ void ldg_stream8(uint2& dst, const void* p) {
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+               : "=r"(dst.x), "=r"(dst.y)
+               : "l"(p));
+}
+__device__ __forceinline__ void ldg_stream4(uint2& dst, const void* p) {
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(dst.x) : "l"(p));
+}
+
 // 4-byte form, into dst.x.
 __device__ __forceinline__ void ldg_stream4(uint4& dst, const void* p) {
   asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(dst.x) : "l"(p));
@@ -357,6 +367,18 @@ __device__ __forceinline__ void cp_async8(void* smem_dst, const void* gmem_src) 
   asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem_dst)),
                "l"(gmem_src)
                : "memory");
+}
+
+// 4-byte form (both addresses 4-byte aligned).
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+// Waits until at most N committed groups of the calling thread are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ------------------------------------------------------------- PDL control

@@ -36,13 +36,6 @@ __device__ __forceinline__ int clamp_len(int T, int max_seq_len, unsigned int* s
 // (part, head) x token dot product of exact bf16 x bf16 products; the parts
 // are added in fp32 and the page maximum is a warp reduction.  A token past
 // the length only reaches its own accumulator column, which is masked.
-//
-// E4M3 caches (F8): a lane loads the same 8 columns as 8 bytes and widens
-// them to f16 (exact); the MMA takes f16 operands, and each folded query is
-// split into f16 hi + lo (rows r and r + 8 of one set) after scaling the
-// group by a power of two that brings its largest magnitude into
-// [2^14, 2^15), so both parts stay in the f16 normal range.  The scale is
-// divided out of the page maximum (exactly: a power of two).
 constexpr int kRmThreads = 256;
 constexpr int kRmWarps = kRmThreads / 32;
 
@@ -50,44 +43,11 @@ constexpr int kRmWarps = kRmThreads / 32;
 // and accumulators fit, else two.  Measured at the 32K-context, B = 16
 // Llama-8B shape: one page in flight per warp with 24 warps per SM beats two
 // pages per warp with 16 warps (136 vs 153 us for fold + scoring + select).
-// Load registers of one page per lane with E4M3 caches: 2 per 32-column
-// chunk, 1 per 16-column chunk, per 8-token tile.
-template <int RB, int RQ, int S>
-__host__ __device__ constexpr int rm_f8_page_regs() {
-  return (S / 8) * (2 * (RB / 32 + RQ / 32) + (RB % 32) / 16 + (RQ % 32) / 16);
-}
-
-// Pages a warp loads before scoring them: the full-width router keeps one
-// page (24 load registers at r_v 64) in flight with 24 warps per SM; a narrow
-// router's pages are a few registers each, so a warp batches more of them to
-// keep about as many bytes in flight.  E4M3 pages are half the registers of
-// bf16 ones, so they batch by the same rule one step further.
-template <int RB, int RQ, int S, bool F8>
-__host__ __device__ constexpr int rm_pages_per_batch() {
-  return F8 ? (rm_f8_page_regs<RB, RQ, S>() <= 4
-                   ? 4
-                   : (rm_f8_page_regs<RB, RQ, S>() <= 8
-                          ? 3
-                          : (rm_f8_page_regs<RB, RQ, S>() <= 16 ? 2 : 1)))
-            : ((S / 8) * (4 * (RB / 32 + RQ / 32) + 2 * ((RB % 32) / 16 + (RQ % 32) / 16)) <= 8
-                   ? 3
-                   : ((S / 8) * (4 * (RB / 32 + RQ / 32) + 2 * ((RB % 32) / 16 + (RQ % 32) / 16)) <=
-                              12
-                          ? 2
-                          : 1));
-}
-
-template <int G, int RB, int RQ, int S, bool F8>
+template <int G, int RB, int RQ, int S>
 __host__ __device__ constexpr int rm_ctas_per_sm() {
-  return F8 ? (rm_pages_per_batch<RB, RQ, S, true>() * rm_f8_page_regs<RB, RQ, S>() +
-                           (S / 8) * 4 <=
-                       40
-                   ? 3
-                   : 2)
-            : ((S / 8) * ((RB + 31) / 32 + (RQ + 31) / 32) * 4 + (S / 8) * (G == 8 ? 2 : 1) * 4 <=
-                       40
-                   ? 3
-                   : 2);
+  return (S / 8) * ((RB + 31) / 32 + (RQ + 31) / 32) * 4 + (S / 8) * (G == 8 ? 2 : 1) * 4 <= 40
+             ? 3
+             : 2;
 }
 
 // A-operand row r of row set `set`: the head it holds (-1: a zero row) and
@@ -136,14 +96,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // (lane c loads columns 8c .. 8c+7, 16 bytes: two k-steps of the MMA) and at
 // most one 16-column tail chunk (lane c loads columns 4c .. 4c+3, 8 bytes:
 // one k-step), so every lane loads and every loaded byte is used.
-template <int G, int RV, int RK, int RB, int RQ, int S, int PW, bool F8>
-__global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S, F8>()))
+template <int G, int RV, int RK, int RB, int RQ, int S, int PW>
+__global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S>()))
     route_mma_kernel(RouteArgs a) {
   extern __shared__ uint4 rm_frags[];
   constexpr int NZF = RB / 32, NZH = (RB % 32) / 16, NEF = RQ / 32, NEH = (RQ % 32) / 16;
   constexpr int NCZ = NZF + NZH, NC = NCZ + NEF + NEH, NT = S / 8, RQ_ = RV + RK;
   constexpr int ZP = RB, EP = RQ;  // row pitch of the columns read (== RV, RK when full)
-  constexpr int SETS = (G == 8 && !F8) ? 2 : 1;
+  constexpr int SETS = G == 8 ? 2 : 1;
   const int lane = threadIdx.x & 31, lr = lane >> 2, lc = lane & 3;
   const long wid = (long)blockIdx.x * kRmWarps + (threadIdx.x >> 5);
   const long nw = (long)gridDim.x * kRmWarps;
@@ -213,50 +173,9 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S, F8>(
   // reads only its own entries.
   uint4* qa = rm_frags + (size_t)(threadIdx.x >> 5) * (SETS * NC * 2 * 32) + lane;
   int frag_bg = -1;
-  float qscale_inv = 1.f;  // E4M3: the group's power-of-two query scale, inverted
   auto load_frags = [&](int bb, int gg) {
     pdl_wait();
     const float* qs = a.qt + ((size_t)bb * a.Hkv + gg) * G * RQ_;
-    if constexpr (F8) {
-      // rows lr (hi) and lr + 8 (lo) of head lr; zero rows past G.  Two
-      // passes over the (cached) folded queries: the group maximum, then
-      // the scaled split, so few values are live at once.
-      auto qv = [&](int c, int k) -> float4 {
-        const bool zc = c < NCZ;
-        const int cc = zc ? c : c - NCZ;
-        const bool half = zc ? (NZH && cc == NZF) : (NEH && cc == NEF);
-        const bool live = lr < G && !(half && k == 1);
-        const int col = (zc ? 0 : RV) + 32 * cc + (half ? 4 * lc : 8 * lc + 4 * k);
-        return live ? *reinterpret_cast<const float4*>(qs + lr * RQ_ + col)
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
-      };
-      float m = 0.f;
-#pragma unroll
-      for (int c = 0; c < NC; ++c)
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const float4 v = qv(c, k);
-          m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-        }
-      m = warp_max(m);
-      // m = f 2^ex with f in [1/2, 1): scale 2^(15 - ex), kept within the
-      // normal fp32 powers of two
-      const int ex = m > 0.f ? (int)((__float_as_uint(m) >> 23) & 0xffu) - 126 : 15;
-      const int sh = max(-126, min(126, 15 - ex));
-      const float sc = __uint_as_float((uint32_t)(127 + sh) << 23);
-      qscale_inv = __uint_as_float((uint32_t)(127 - sh) << 23);
-#pragma unroll 1
-      for (int c = 0; c < NC; ++c)
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const float4 v = qv(c, k);
-          uint32_t h01, l01, h23, l23;
-          split_f16x2(v.x * sc, v.y * sc, h01, l01);
-          split_f16x2(v.z * sc, v.w * sc, h23, l23);
-          qa[(c * 2 + k) * 32] = make_uint4(h01, l01, h23, l23);
-        }
-      return;
-    }
 #pragma unroll
     for (int set = 0; set < SETS; ++set) {
       int h0, p0, h1, p1;
@@ -306,30 +225,6 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S, F8>(
         }
         // a narrow router's columns lead each tile: [S][RB] then the rest
         const size_t tile = (size_t)pp * a.Hkv + g;
-        if constexpr (F8) {  // one byte per column
-          const uint8_t* zr = reinterpret_cast<const uint8_t*>(a.Z) + tile * S * RV + lr * ZP + 8 * lc;
-          const uint8_t* er = reinterpret_cast<const uint8_t*>(a.E) + tile * S * RK + lr * EP + 8 * lc;
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-#pragma unroll
-            for (int c = 0; c < NCZ; ++c) {
-              if (NZH && c == NZF)
-                ldg_stream4(x[k][t][c], zr - 4 * lc + t * 8 * ZP + 32 * c);
-              else
-                ldg_stream8(x[k][t][c], zr + t * 8 * ZP + 32 * c);
-            }
-#pragma unroll
-            for (int c = NCZ; c < NC; ++c) {
-              if (NEH && c - NCZ == NEF)
-                ldg_stream4(x[k][t][c], er - 4 * lc + t * 8 * EP + 32 * (c - NCZ));
-              else
-                ldg_stream8(x[k][t][c], er + t * 8 * EP + 32 * (c - NCZ));
-            }
-          }
-          advance();
-          skip();
-          continue;
-        }
         const uint16_t* zr = a.Z + tile * S * RV + lr * ZP + 8 * lc;
         const uint16_t* er = a.E + tile * S * RK + lr * EP + 8 * lc;
 #pragma unroll
@@ -364,34 +259,6 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S, F8>(
 #pragma unroll
         for (int set = 0; set < SETS; ++set)
           acc[t][set][0] = acc[t][set][1] = acc[t][set][2] = acc[t][set][3] = 0.f;
-      if constexpr (F8) {
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-          const bool half = c < NCZ ? (NZH && c == NZF) : (NEH && c - NCZ == NEF);
-          const uint4 f0 = qa[(c * 2 + 0) * 32];
-          const uint4 f1 = qa[(c * 2 + 1) * 32];
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            uint32_t w0, w1;
-            e4m3x4_to_f16(x[k][t][c].x, w0, w1);
-            mma_f16_16816(acc[t][0], f0.x, f0.y, f0.z, f0.w, w0, w1);
-            if (!half) {
-              e4m3x4_to_f16(x[k][t][c].y, w0, w1);
-              mma_f16_16816(acc[t][0], f1.x, f1.y, f1.z, f1.w, w0, w1);
-            }
-          }
-        }
-        float best = -INFINITY;
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {  // hi (row lr) + lo (row lr + 8) of head lr
-          const float s0 = lr < G ? acc[t][0][0] + acc[t][0][2] : -INFINITY;
-          const float s1 = lr < G ? acc[t][0][1] + acc[t][0][3] : -INFINITY;
-          const int tok = ulp[k] * S + t * 8 + 2 * lc;
-          if (tok < uT[k]) best = fmaxf(best, s0);
-          if (tok + 1 < uT[k]) best = fmaxf(best, s1);
-        }
-        return best * qscale_inv;
-      }
 #pragma unroll
       for (int c = 0; c < NC; ++c)
 #pragma unroll
@@ -460,24 +327,36 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S, F8>(
   }
 }
 
-template <int G, int RV, int RK, int RB, int RQ, int S, bool F8 = false>
+// Pages a warp loads before scoring them: the full-width router keeps one
+// page (24 load registers at r_v 64) in flight with 24 warps per SM; a narrow
+// router's pages are a few registers each, so a warp batches more of them to
+// keep about as many bytes in flight.
+template <int RB, int RQ, int S>
+constexpr int rm_pages_per_batch() {
+  return (S / 8) * (4 * (RB / 32 + RQ / 32) + 2 * ((RB % 32) / 16 + (RQ % 32) / 16)) <= 8
+             ? 3
+             : ((S / 8) * (4 * (RB / 32 + RQ / 32) + 2 * ((RB % 32) / 16 + (RQ % 32) / 16)) <= 12
+                    ? 2
+                    : 1);
+}
+
+template <int G, int RV, int RK, int RB, int RQ, int S>
 cudaError_t launch_route_mma(const RouteArgs& a, cudaStream_t st, bool pdl) {
-  constexpr int PW = rm_pages_per_batch<RB, RQ, S, F8>();
+  constexpr int PW = rm_pages_per_batch<RB, RQ, S>();
   constexpr int NC = (RB + 31) / 32 + (RQ + 31) / 32;
-  constexpr int SETS = (G == 8 && !F8) ? 2 : 1;
   const int P_max = (a.max_seq_len + S - 1) / S;
   const long pages = (long)a.B * a.Hkv * P_max;
-  long grid = (long)num_sms() * rm_ctas_per_sm<G, RB, RQ, S, F8>();
+  long grid = (long)num_sms() * rm_ctas_per_sm<G, RB, RQ, S>();
   const long need = (pages + kRmWarps - 1) / kRmWarps;
   if (grid > need) grid = need;
   if (grid < 1) grid = 1;
-  const size_t smem = (size_t)kRmWarps * SETS * NC * 2 * 32 * 16;
+  const size_t smem = (size_t)kRmWarps * (G == 8 ? 2 : 1) * NC * 2 * 32 * 16;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(route_mma_kernel<G, RV, RK, RB, RQ, S, PW, F8>,
+    cudaError_t e = cudaFuncSetAttribute(route_mma_kernel<G, RV, RK, RB, RQ, S, PW>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_k(route_mma_kernel<G, RV, RK, RB, RQ, S, PW, F8>, dim3((unsigned)grid),
+  return launch_k(route_mma_kernel<G, RV, RK, RB, RQ, S, PW>, dim3((unsigned)grid),
                   dim3(kRmThreads), smem, st, pdl, a);
 }
 
