@@ -409,6 +409,165 @@ def run_gpu(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_stack(args) -> None:
+    """The 32 attention layers of the Llama-8B shape, each with its own Value
+    width (Table 12's per-layer V ranks with the given average): one fused
+    decode step per layer per model step, the layers in order on one stream."""
+    import sparse_decode_attention_basiskv_b200 as bkv
+    from sparse_decode_attention_basiskv_b200.layer import DecodeLayer, DecodeStack
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    K, W = args.steps, args.warmup
+    avg = int(args.stack[3:])
+    base = synth.with_sizes(synth.LLAMA8B_32L_T32K_B16_AVG64, steps=K + W,
+                            B=args.batch or synth.LLAMA8B_32L_T32K_B16_AVG64.B,
+                            T=args.context or synth.LLAMA8B_32L_T32K_B16_AVG64.T)
+    if avg != 64:
+        base = synth.with_sizes(base, name=base.name.replace("avg_v64", f"avg_v{avg}"))
+    widths = synth.v_rank_schedule(avg, base.layers)
+    wls = synth.stack_layers(base, widths)
+    layers, qs, ks, vs = [], [], [], []
+    for l, wl in enumerate(wls):  # one layer at a time bounds the temporaries
+        pb = synth.make_problem(wl, device="cuda", layer=l)
+        layers.append(DecodeLayer.from_problem(pb))
+        qs.append([pb.q, synth.make_query(wl, pb.cache["K"], wl.T, step=1)[0]])
+        k_all, v_all = synth.make_tokens(wl, pb.factors, K + W, device="cuda", stream_id=l)
+        ks.append([k_all[:, i].contiguous() for i in range(K + W)])
+        vs.append([v_all[:, i].contiguous() for i in range(K + W)])
+        del pb, k_all, v_all
+        torch.cuda.empty_cache()
+    stack = DecodeStack(layers)
+    T0 = base.T
+    stream = torch.cuda.current_stream()
+
+    def step(i, T_after):
+        stack.decode([q[i % 2] for q in qs], [k[i] for k in ks], [v[i] for v in vs],
+                     max_seq_len=T_after)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(W):
+        step(i, T0 + i + 1)
+    barrier()
+    assert bkv.read_device_status() == 0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = bkv.launch_count()
+    with ClockSampler(local) as clocks:
+        barrier()
+        ev0.record(stream)
+        for i in range(W, W + K):
+            step(i, T0 + i + 1)
+        ev1.record(stream)
+        barrier()
+    launches = bkv.launch_count() - launches0
+    assert bkv.read_device_status() == 0
+    per_layer = [sum(algorithmic_bytes(wl, T0 + i + 1)["total"] for i in range(W, W + K))
+                 for wl in wls]
+    total_bytes = sum(per_layer)
+    ms_max, value = replica_throughput(ev0.elapsed_time(ev1), total_bytes, dist, "cuda")
+
+    # roofline: the scoring kernel (+ its fold) of every layer, back to back
+    T_r = T0 + W + K
+    for L in layers:
+        L.seq_lens.fill_(T_r)
+    scores = [torch.empty(base.B, base.Hkv, L.dims.max_pages_per_seq, device="cuda")
+              for L in layers]
+
+    def route_all():
+        for L, sc, q in zip(layers, scores, qs):
+            bkv.basiskv_route(L.dims, q[0], L.seq_lens, T_r, L.block_table, L.P_K, L.U_K, L.Z,
+                              L.E, base.top_k, sc, None, L.workspace)
+    for _ in range(3):
+        route_all()
+    torch.cuda.synchronize()
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 10
+    r0.record(stream)
+    for _ in range(reps):
+        route_all()
+    r1.record(stream)
+    torch.cuda.synchronize()
+    route_ms = r0.elapsed_time(r1) / reps
+    route_bytes = sum(base.B * base.Hkv * T_r * (wl.r_v + wl.r_k) * 2 for wl in wls)
+    peak, peak_kind = measured_peak()
+    achieved = route_bytes / (route_ms / 1e3) / 1e9
+
+    # end to end through the public API: q, k, v of every layer in, y out
+    for L in layers:
+        L.seq_lens.fill_(T0)
+    q_h = [[q.cpu().pin_memory() for q in ql] for ql in qs]
+    k_h = [[k.cpu().pin_memory() for k in kl] for kl in ks]
+    v_h = [[v.cpu().pin_memory() for v in vl] for vl in vs]
+    q_d = [torch.empty_like(ql[0]) for ql in qs]
+    k_d = [torch.empty_like(kl[0]) for kl in ks]
+    v_d = [torch.empty_like(vl[0]) for vl in vs]
+    y_h = [torch.empty(base.B, base.hidden, dtype=torch.bfloat16).pin_memory() for _ in layers]
+
+    def e2e_step(i, T_after):
+        for l in range(len(layers)):
+            q_d[l].copy_(q_h[l][i % 2], non_blocking=True)
+            k_d[l].copy_(k_h[l][i], non_blocking=True)
+            v_d[l].copy_(v_h[l][i], non_blocking=True)
+        ys = stack.decode(q_d, k_d, v_d, max_seq_len=T_after)
+        for l, y in enumerate(ys):
+            y_h[l].copy_(y, non_blocking=True)
+
+    for i in range(W):
+        e2e_step(i, T0 + i + 1)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(W, W + K):
+        e2e_step(i, T0 + i + 1)
+    e1.record(stream)
+    barrier()
+    e2e_ms, e2e_value = replica_throughput(e0.elapsed_time(e1), total_bytes, dist, "cuda")
+    h2d = sum((q[0].numel() + k[0].numel() + v[0].numel()) * 2 for q, k, v in zip(qs, ks, vs))
+    d2h = len(layers) * base.B * base.hidden * 2
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    cpu = cpu_baseline(wls[0]) if world == 1 and not args.no_cpu_baseline else None
+    line = {
+        "metric": METRIC + f" — {base.layers}-layer stack, per-layer Value widths",
+        "value": value, "unit": "TB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_max / K, "us_per_layer_step": ms_max / K * 1e3 / len(layers),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generators; planted-page queries)",
+        "config": {"workload": base.name, "layers": len(layers), "v_widths": widths,
+                   "avg_v_width": sum(widths) / len(widths), "global_batch": base.B * world,
+                   "seq_len": T0, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs far larger than L2; no flush"},
+        "bytes_per_step": total_bytes / K,
+        "frac_of_peak": value / world / (peak / 1e3),
+        "roofline": {"bound": "hbm", "kernel": "route_mma_kernel (+ its query fold), all layers",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "ms_per_launch": route_ms / len(layers),
+                     "algorithmic_bytes": route_bytes / len(layers)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TB/s", "ms_per_step": e2e_ms / K,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def _route_source_sha() -> str:
     import hashlib
     h = hashlib.sha256()
@@ -434,6 +593,9 @@ def main():
                          "newest page); b16r16: the pages' narrow router and budget")
     ap.add_argument("--cache", default="bf16", choices=["bf16", "e4m3"],
                     help="element type of the K, Z and E caches")
+    ap.add_argument("--stack", default="", choices=["", "avg64", "avg96"],
+                    help="time the 32-layer stack with per-layer Value widths of this average "
+                         "instead of one layer")
     args = ap.parse_args()
     global WL
     if args.router == "b16r16":
@@ -444,6 +606,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.stack:
+        run_stack(args)
     else:
         run_gpu(args)
 

@@ -759,6 +759,10 @@ cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
 #define BKV_RM(GG, V, K, SS)                                     \
   if (a.G == GG && a.r_v == V && a.r_k == K && a.S == SS) \
     return launch_route_mma<GG, V, K, V, K, SS>(a, st, pdl);
+    BKV_RM(4, 32, 32, 16)
+    BKV_RM(4, 32, 32, 32)
+    BKV_RM(8, 32, 32, 16)
+    BKV_RM(8, 32, 32, 32)
     BKV_RM(4, 64, 32, 16)
     BKV_RM(4, 96, 32, 16)
     BKV_RM(4, 128, 32, 16)

@@ -69,3 +69,27 @@ class DecodeLayer:
                        self.block_table, self.A_V, self.P_K, self.U_K, self.W_fold, self.K,
                        self.Z, self.E, self.top_k, sel, y, self.workspace, stream)
         return y
+
+
+class DecodeStack:
+    """The attention blocks of a layer stack run in order on one stream, each
+    layer with its own Value width (and so its own cache widths, factors and
+    workspace): the per-layer Value ranks of Table 12 ("Avg. V rank")."""
+
+    def __init__(self, layers: list):
+        self.layers = layers
+
+    @property
+    def widths(self) -> list:
+        return [L.dims.r_v for L in self.layers]
+
+    def decode(self, qs, ks=None, vs=None, max_seq_len=None, ys=None, stream=None) -> list:
+        """One decode step of every layer: layer l gets qs[l] (and ks[l],
+        vs[l] when appending).  Returns the layers' y (views of their output
+        buffers unless ys is given)."""
+        out = []
+        for i, L in enumerate(self.layers):
+            out.append(L.decode(qs[i], None if ks is None else ks[i],
+                                None if vs is None else vs[i], max_seq_len=max_seq_len,
+                                y=None if ys is None else ys[i], stream=stream))
+        return out

@@ -152,6 +152,31 @@ def sweep_point(B: int, T: int, r_v: int, layers: int = 32,
                     append_tokens=1, layers=layers, steps=steps)
 
 
+def v_rank_schedule(avg: int, layers: int = 32, seed: int = 0) -> list:
+    """Per-layer Value widths with average `avg` over `layers` layers (Table
+    12 reports an average V rank per model, the widths chosen per layer):
+    half the layers at the average, a quarter 32 below, a quarter 32 above,
+    in a seeded order.  avg in {64, 96}; layers a multiple of 4."""
+    if avg not in (64, 96) or layers % 4:
+        raise ValueError("schedules exist for avg 64 / 96 and layers % 4 == 0")
+    q = layers // 4
+    widths = [avg - 32] * q + [avg] * (2 * q) + [avg + 32] * q
+    order = torch.randperm(layers, generator=torch.Generator().manual_seed(seed + 17))
+    return [widths[i] for i in order.tolist()]
+
+
+def stack_layers(wl: Workload, widths: list) -> list:
+    """The per-layer workloads of a layer stack: wl with layer l's Value
+    width (and its own seeds through the layer index of make_problem)."""
+    return [replace(wl, name=f"{wl.name}_layer{l}_v{r}", r_v=r) for l, r in enumerate(widths)]
+
+
+# The 32 attention layers of Llama-3.1-8B at the headline batch and context,
+# Value widths varying per layer with average 64.
+LLAMA8B_32L_T32K_B16_AVG64 = replace(LLAMA8B_T32K_B16, name="llama8b_32layers_b16_t32k_avg_v64_append1",
+                                     layers=32)
+
+
 SWEEP = [sweep_point(B, T, r_v) for B in (1, 8, 32, 64)
          for T in (4096, 32768, 131072) for r_v in (96, 64)]
 

@@ -348,3 +348,15 @@ def test_to_e4m3_saturates_and_keeps_steps():
     np.testing.assert_array_equal(O.to_e4m3([500.0, -1e6, 449.0]), [448.0, -448.0, 448.0])
     np.testing.assert_array_equal(O.to_e4m3([2.0 ** -9, 2.0 ** -10, 1.0625, 1.09375]),
                                   [2.0 ** -9, 0.0, 1.0, 1.125])
+
+
+# ------------------------------------------------- per-layer Value widths
+def test_v_rank_schedule_average_and_members():
+    from sparse_decode_attention_basiskv_b200 import synth
+    for avg in (64, 96):
+        w = synth.v_rank_schedule(avg, 32)
+        assert len(w) == 32 and sum(w) == 32 * avg
+        assert sorted(set(w)) == [avg - 32, avg, avg + 32]
+        assert w == synth.v_rank_schedule(avg, 32)  # seeded
+    layers = synth.stack_layers(synth.LLAMA8B_T32K_B16, [32, 64, 128])
+    assert [L.r_v for L in layers] == [32, 64, 128] and len({L.name for L in layers}) == 3
