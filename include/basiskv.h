@@ -265,6 +265,43 @@ BASISKV_API int basiskv_decode(const basiskv_dims* dims, const basiskv_bf16* q,
                    int32_t* sel, basiskv_bf16* y, void* workspace,
                    size_t workspace_bytes, void* stream);
 
+/* Tensor parallelism (Figure 1): each GPU holds some KV heads (with their
+ * query heads) of a layer, compresses its local attention output into the
+ * heads' Value latents, the GPUs exchange those latents with an AllGather,
+ * and each rebuilds the complete output from all of them.  The two calls
+ * below are the per-GPU compute on either side of that AllGather (which
+ * the caller issues, e.g. NCCL over NVLink).
+ *
+ * basiskv_decode_latents: basiskv_decode without the out-projection, for
+ * the heads described by dims (a rank's share: its Hq and Hkv).  Writes the
+ * Value latents a_out bf16 [B][Hq][r_v] (fp32 softmax accumulation, one
+ * bf16 rounding) and, with an append, advances seq_lens after every reader.
+ * Uses no W_fold. */
+BASISKV_API int basiskv_decode_latents(const basiskv_dims* dims, const basiskv_bf16* q,
+                                       const basiskv_bf16* k_new, const basiskv_bf16* v_new,
+                                       int32_t* seq_lens, int max_seq_len,
+                                       const int32_t* block_table, const basiskv_bf16* A_V,
+                                       const basiskv_bf16* P_K, const basiskv_bf16* U_K,
+                                       basiskv_bf16* K_cache, basiskv_bf16* Z_cache,
+                                       basiskv_bf16* E_cache, int top_k, int32_t* sel,
+                                       basiskv_bf16* a_out, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/* basiskv_outproj_sources: the complete output from the latents of n_src
+ * sources, stored source-major as an AllGather leaves them:
+ *   a_src bf16 [n_src][B][Hq / n_src][r_v]   (source s holds query heads
+ *                                             s*Hq/n_src .. (s+1)*Hq/n_src-1)
+ *   y[b][o] = sum_h sum_j a[b][h][j] * W_fold[o][h*r_v + j]
+ * on the tcgen05 tensor cores (fp32 accumulation).  dims describes the whole
+ * layer (all Hq heads; W_fold [H][Hq*r_v] as built by basiskv_fold_outproj).
+ * Hq % n_src != 0 is BASISKV_ERR_INVALID_ARG; (Hq / n_src) * r_v must be a
+ * multiple of 64 (else BASISKV_ERR_UNSUPPORTED_SHAPE).  n_src = 1 is the
+ * out-projection of bf16 latents [B][Hq][r_v]. */
+BASISKV_API int basiskv_outproj_sources(const basiskv_dims* dims, const basiskv_bf16* a_src,
+                                        int n_src, const basiskv_bf16* W_fold,
+                                        basiskv_bf16* y, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
 /* Size of the static device scratch array behind basiskv_decode_noalloc. */
 #define BASISKV_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 

@@ -71,6 +71,9 @@ _SIGNATURES = {
                             _P, _P, _P, _SZ, _P]),
     "basiskv_decode_noalloc": (_I, [_DIMS, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
                                     _I, _P, _P, _P]),
+    "basiskv_decode_latents": (_I, [_DIMS, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _I,
+                                    _P, _P, _P, _SZ, _P]),
+    "basiskv_outproj_sources": (_I, [_DIMS, _P, _I, _P, _P, _P, _SZ, _P]),
     "basiskv_read_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "basiskv_strerror": (ctypes.c_char_p, [_I]),
     "basiskv_launch_count": (ctypes.c_uint64, []),
@@ -194,6 +197,27 @@ def basiskv_decode_noalloc(dims: Dims, q, k_new, v_new, seq_lens, max_seq_len: i
         _ptr(block_table), _ptr(A_V), _ptr(P_K), _ptr(U_K), _ptr(W_fold), _ptr(K_cache),
         _ptr(Z_cache), _ptr(E_cache), top_k, _ptr(sel), _ptr(y), _stream(stream)),
         "basiskv_decode_noalloc")
+
+
+def basiskv_decode_latents(dims: Dims, q, k_new, v_new, seq_lens, max_seq_len: int, block_table,
+                           A_V, P_K, U_K, K_cache, Z_cache, E_cache, top_k: int, sel, a_out,
+                           workspace, stream=None) -> None:
+    """The fused step up to the Value latents a_out (bf16 [B][Hq][r_v]) of
+    the heads in dims: one GPU's share of a tensor-parallel layer."""
+    _check(load_library().basiskv_decode_latents(
+        ctypes.byref(dims), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(seq_lens), max_seq_len,
+        _ptr(block_table), _ptr(A_V), _ptr(P_K), _ptr(U_K), _ptr(K_cache), _ptr(Z_cache),
+        _ptr(E_cache), top_k, _ptr(sel), _ptr(a_out), _ptr(workspace), _nbytes(workspace),
+        _stream(stream)), "basiskv_decode_latents")
+
+
+def basiskv_outproj_sources(dims: Dims, a_src, n_src: int, W_fold, y, workspace,
+                            stream=None) -> None:
+    """y from the latents of n_src sources stored source-major
+    ([n_src][B][Hq/n_src][r_v] bf16, as an AllGather leaves them)."""
+    _check(load_library().basiskv_outproj_sources(
+        ctypes.byref(dims), _ptr(a_src), n_src, _ptr(W_fold), _ptr(y), _ptr(workspace),
+        _nbytes(workspace), _stream(stream)), "basiskv_outproj_sources")
 
 
 def read_device_status(stream=None) -> int:

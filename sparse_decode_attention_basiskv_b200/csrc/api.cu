@@ -430,17 +430,19 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
   return launch_status(launch_combine(c, st, pdl));
 }
 
+// n_src > 1: the latents are stored source-major, [n_src][B][K / n_src].
 int run_outproj(const basiskv_dims* d, const uint16_t* a_bf16, const basiskv_bf16* W_fold,
                 basiskv_bf16* y, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl,
-                int32_t* bump_lens = nullptr, int* cnt = nullptr) {
+                int32_t* bump_lens = nullptr, int* cnt = nullptr, int n_src = 1) {
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
-  const int K = d->Hq * d->r_v;
+  const int K = d->Hq * d->r_v, K_src = K / n_src;
   const int bn = outproj_bn(d->B);
   CUtensorMap tmW, tmA;
   if (!make_tmap_2d(&tmW, W_fold, d->hidden, K, (uint64_t)K * 2, 128, 64,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&tmA, a_bf16, d->B, K, (uint64_t)K * 2, bn, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_tmap_2d(&tmA, a_bf16, (uint64_t)n_src * d->B, K_src, (uint64_t)K_src * 2, bn, 64,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
     return BASISKV_ERR_CUDA;
   OutprojArgs o{};
   o.partial = reinterpret_cast<float*>(ws + L.op_part);
@@ -456,6 +458,7 @@ int run_outproj(const basiskv_dims* d, const uint16_t* a_bf16, const basiskv_bf1
   o.bump_n = 1;
   o.bump_cap = d->max_pages_per_seq * d->page_size;
   o.cnt = cnt;
+  o.k_src = K_src;
   return launch_status(launch_outproj(o, tmW, tmA, st, pdl));
 }
 
@@ -689,6 +692,80 @@ int basiskv_decode(const basiskv_dims* dims, const basiskv_bf16* q, const basisk
   if (rc) return rc;
   return run_outproj(dims, a16, W_fold, y, ws, L, st, pdl, append ? seq_lens : nullptr,
                      cnt + L.n_att_cnt);
+}
+
+int basiskv_decode_latents(const basiskv_dims* dims, const basiskv_bf16* q,
+                           const basiskv_bf16* k_new, const basiskv_bf16* v_new,
+                           int32_t* seq_lens, int max_seq_len, const int32_t* block_table,
+                           const basiskv_bf16* A_V, const basiskv_bf16* P_K,
+                           const basiskv_bf16* U_K, basiskv_bf16* K_cache, basiskv_bf16* Z_cache,
+                           basiskv_bf16* E_cache, int top_k, int32_t* sel, basiskv_bf16* a_out,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_len_topk(dims, top_k, max_seq_len);
+  if (rc) return rc;
+  const bool append = k_new || v_new;
+  if (append) {
+    BKV_REQUIRE(k_new);
+    BKV_REQUIRE(v_new);
+    BKV_REQUIRE(A_V);
+  }
+  BKV_REQUIRE(q);
+  BKV_REQUIRE4(seq_lens);
+  BKV_REQUIRE4(block_table);
+  BKV_REQUIRE(P_K);
+  BKV_REQUIRE(U_K);
+  BKV_REQUIRE(K_cache);
+  BKV_REQUIRE(Z_cache);
+  BKV_REQUIRE(E_cache);
+  BKV_REQUIRE(a_out);
+  if (sel && !aligned4(sel)) return BASISKV_ERR_INVALID_ARG;
+  WsLayout L;
+  rc = check_ws(dims, top_k, workspace, workspace_bytes, &L);
+  if (rc) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool pdl = pdl_enabled();
+  int32_t* sel_buf = sel ? sel : reinterpret_cast<int32_t*>(ws + L.sel);
+  const int off = append ? 1 : 0;
+  int* cnt = reinterpret_cast<int*>(ws + L.counters);
+  AppendArgs app = make_append_args(dims, append ? k_new : nullptr, v_new, 1, seq_lens,
+                                    block_table, A_V, P_K, U_K, K_cache, Z_cache, E_cache);
+  if (!app.status) return BASISKV_ERR_CUDA;
+  {
+    AppendArgs none = app;
+    none.k_new = nullptr;
+    FoldQArgs f{q, P_K, U_K, reinterpret_cast<float*>(ws + L.qt), dims->B, dims->Hq, dims->Hkv,
+                dims->d, dims->r_v, dims->r_k};
+    rc = launch_status(launch_decode_prologue(f, none, cnt, L.n_att_cnt, st, pdl));
+    if (rc) return rc;
+  }
+  rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache, top_k,
+                 reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl, off,
+                 /*do_fold=*/false, append ? &app : nullptr);
+  if (rc) return rc;
+  rc = run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel_buf, top_k, nullptr, a_out,
+                  ws, L, st, pdl, off, cnt, reinterpret_cast<const int32_t*>(ws + L.selp));
+  if (rc || !append) return rc;
+  return launch_status(launch_bump_lengths(app, st, pdl));  // after every reader
+}
+
+int basiskv_outproj_sources(const basiskv_dims* dims, const basiskv_bf16* a_src, int n_src,
+                            const basiskv_bf16* W_fold, basiskv_bf16* y, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (n_src < 1 || dims->Hq % n_src) return BASISKV_ERR_INVALID_ARG;
+  if ((dims->Hq / n_src * dims->r_v) % 64) return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  BKV_REQUIRE(a_src);
+  BKV_REQUIRE(W_fold);
+  BKV_REQUIRE(y);
+  WsLayout L;
+  rc = check_ws(dims, 2, workspace, workspace_bytes, &L);
+  if (rc) return rc;
+  return run_outproj(dims, a_src, W_fold, y, static_cast<uint8_t*>(workspace), L,
+                     static_cast<cudaStream_t>(stream), pdl_enabled(), nullptr, nullptr, n_src);
 }
 
 int basiskv_read_device_status(void* stream, uint32_t* flags) {

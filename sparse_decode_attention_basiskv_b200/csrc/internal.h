@@ -184,6 +184,10 @@ struct OutprojArgs {
   // arrival counter, zeroed before the launch; the tile's last CTA sums the
   // partials and writes y.
   int* cnt;
+  // Latents stored source-major, [K / k_src sources][src_rows = B][k_src]:
+  // column k of row b is element (k % k_src) of row (k / k_src) * B + b.
+  // k_src = K for the plain [B][K] layout.
+  int k_src;
 };
 // Chooses the K split for a given problem.
 int outproj_ksplit(int H, int K, int B);

@@ -154,14 +154,18 @@ __global__ void __launch_bounds__(kOpThreads, 1)
         tma_load_2d(a_tiles + it * kOpATile, &tmW, (kb0 + it) * kOpBK, m0, &full[it]);
       }
       pdl_wait();
-      for (int it = 0; it < pre; ++it)
-        tma_load_2d(b_tiles + it * kBTile, &tmA, (kb0 + it) * kOpBK, 0, &full[it]);
+      // latent column k = source k / k_src, column k % k_src of its B rows
+      auto load_a = [&](uint8_t* dst, int kb, uint64_t* bar) {
+        const int kc = kb * kOpBK;
+        tma_load_2d(dst, &tmA, kc % a.k_src, (kc / a.k_src) * a.B, bar);
+      };
+      for (int it = 0; it < pre; ++it) load_a(b_tiles + it * kBTile, kb0 + it, &full[it]);
       for (int kb = kb0 + pre, it = pre; kb < kb1; ++kb, ++it) {
         const int s = it % kOpStages;
         if (!mbar_wait(&empty[s], ((it / kOpStages) & 1) ^ 1, a.status)) break;
         mbar_arrive_expect_tx(&full[s], kOpATile + kBTile);
         tma_load_2d(a_tiles + s * kOpATile, &tmW, kb * kOpBK, m0, &full[s]);
-        tma_load_2d(b_tiles + s * kBTile, &tmA, kb * kOpBK, 0, &full[s]);
+        load_a(b_tiles + s * kBTile, kb, &full[s]);
       }
     }
   } else if (warp == 1) {

@@ -9,6 +9,7 @@ import ctypes
 import subprocess
 
 import pytest
+import torch
 
 import sparse_decode_attention_basiskv_b200 as bkv
 
@@ -29,7 +30,7 @@ def lib():
 
 def test_header_symbols_are_exported(lib):
     names = bkv.header_symbols()
-    assert len(names) == 12
+    assert len(names) == 14
     out = subprocess.run(["nm", "-D", "--defined-only", bkv.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
@@ -170,3 +171,51 @@ def test_e4m3_cache_validation(lib):
     assert lib.basiskv_decode(ctypes.byref(d), FAKE, None, None, FAKE, 100, FAKE, FAKE, FAKE,
                               FAKE, FAKE, FAKE, FAKE, FAKE, 8, None, FAKE, FAKE, 1 << 30,
                               None) == bkv.ERR_INVALID_ARG
+
+
+def test_tensor_parallel_entry_points_validate(lib):
+    big = 1 << 30
+    d = _dims()
+    # sources must divide the query heads
+    assert lib.basiskv_outproj_sources(ctypes.byref(d), FAKE, 3, FAKE, FAKE, FAKE, big,
+                                       None) == bkv.ERR_INVALID_ARG
+    assert lib.basiskv_outproj_sources(ctypes.byref(d), FAKE, 0, FAKE, FAKE, FAKE, big,
+                                       None) == bkv.ERR_INVALID_ARG
+    # (Hq / n_src) * r_v = 1 * 32 is not a multiple of 64
+    assert lib.basiskv_outproj_sources(ctypes.byref(_dims(r_v=32)), FAKE, 8, FAKE, FAKE, FAKE,
+                                       big, None) == bkv.ERR_UNSUPPORTED_SHAPE
+    assert lib.basiskv_outproj_sources(ctypes.byref(d), None, 2, FAKE, FAKE, FAKE, big,
+                                       None) == bkv.ERR_INVALID_ARG
+    assert lib.basiskv_outproj_sources(ctypes.byref(d), FAKE, 2, FAKE, FAKE, FAKE, 16,
+                                       None) == bkv.ERR_WORKSPACE_TOO_SMALL
+    # latents: output buffer required, k_new without v_new refused
+    assert lib.basiskv_decode_latents(ctypes.byref(d), FAKE, None, None, FAKE, 100, FAKE, FAKE,
+                                      FAKE, FAKE, FAKE, FAKE, FAKE, 8, None, None, FAKE, big,
+                                      None) == bkv.ERR_INVALID_ARG
+    assert lib.basiskv_decode_latents(ctypes.byref(d), FAKE, FAKE, None, FAKE, 100, FAKE, FAKE,
+                                      FAKE, FAKE, FAKE, FAKE, FAKE, 8, None, FAKE, FAKE, big,
+                                      None) == bkv.ERR_INVALID_ARG
+    assert lib.basiskv_decode_latents(ctypes.byref(d), FAKE, None, None, FAKE, 100, FAKE, FAKE,
+                                      FAKE, FAKE, FAKE, FAKE, FAKE, 8, None, FAKE, FAKE, 64,
+                                      None) == bkv.ERR_WORKSPACE_TOO_SMALL
+
+
+def test_head_shard_covers_every_head_once():
+    from sparse_decode_attention_basiskv_b200.tp import head_shard, local_dims, shard_factors
+    for Hq, Hkv, world in ((32, 8, 2), (32, 8, 4), (32, 8, 8), (64, 8, 8), (8, 2, 2)):
+        hs, gs = [], []
+        for r in range(world):
+            g0, g1, h0, h1 = head_shard(Hq, Hkv, world, r)
+            gs += range(g0, g1)
+            hs += range(h0, h1)
+            assert h0 == g0 * (Hq // Hkv) and h1 == g1 * (Hq // Hkv)
+        assert gs == list(range(Hkv)) and hs == list(range(Hq))
+    with pytest.raises(ValueError):
+        head_shard(32, 8, 3, 0)
+    ld = local_dims(_dims(), 2)
+    assert (ld.Hq, ld.Hkv, ld.d, ld.r_v) == (4, 1, 128, 64)
+    f = {"A_V": torch.arange(2)[:, None], "P_K": torch.arange(2)[:, None],
+         "U_K": torch.arange(2)[:, None], "B_V": torch.arange(2)[:, None],
+         "W_O": torch.arange(8 * 3)[:, None]}
+    s1 = shard_factors(f, 8, 2, 3, 2, 1)
+    assert s1["A_V"].tolist() == [[1]] and s1["W_O"][:, 0].tolist() == list(range(12, 24))
