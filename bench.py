@@ -591,6 +591,119 @@ def run_stack(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_prefill(args) -> None:
+    """The prefill-chunk append on the tensor cores: a 4096-token chunk of
+    the Qwen3-32B layer appended to every sequence of the batch in one call
+    ([z | e] = [v | k] W_app^T per KV head, scattered into the pages)."""
+    import sparse_decode_attention_basiskv_b200 as bkv
+    from sparse_decode_attention_basiskv_b200.layer import DecodeLayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    K, W = args.steps, args.warmup
+    base = synth.QWEN32B_T64K_B8
+    wl = synth.with_sizes(base, B=args.batch or base.B, T=args.context or base.T, steps=1)
+    if args.cache == "e4m3":
+        wl = synth.with_sizes(wl, cache_fp8=1, name=wl.name + "_e4m3")
+    n = wl.prefill_tokens
+    pb = synth.make_problem(wl, device="cuda")
+    layer = DecodeLayer.from_problem(pb)
+    k, v = synth.make_tokens(wl, pb.factors, n, device="cuda", stream_id=1)
+    del pb
+    torch.cuda.empty_cache()
+    lens = [torch.full((wl.B,), wl.T, dtype=torch.int32, device="cuda") for _ in range(K + W)]
+    stream = torch.cuda.current_stream()
+
+    def step(i, kk=k, vv=v):
+        bkv.basiskv_append(layer.dims, kk, vv, n, lens[i], layer.block_table, layer.A_V,
+                           layer.P_K, layer.U_K, layer.K, layer.Z, layer.E, layer.workspace,
+                           W_app=layer.W_app)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(W):
+        step(i)
+    barrier()
+    assert bkv.read_device_status() == 0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = bkv.launch_count()
+    with ClockSampler(local) as clocks:
+        barrier()
+        ev0.record(stream)
+        for i in range(W, W + K):
+            step(i)
+        ev1.record(stream)
+        barrier()
+    launches = bkv.launch_count() - launches0
+    assert bkv.read_device_status() == 0
+    assert all(int(x) == wl.T + n for x in lens[W + K - 1].tolist())
+    cb = 1 if wl.cache_fp8 else 2
+    rows = wl.B * n
+    per_step = (rows * wl.Hkv * (2 * wl.d * 2 + (wl.d + wl.r_v + wl.r_k) * cb)
+                + wl.Hkv * (wl.r_v + wl.r_k) * 2 * wl.d * 2)
+    ms_max, value = replica_throughput(ev0.elapsed_time(ev1), per_step * K, dist, "cuda")
+    ms_step = ms_max / K
+    flops = 2.0 * rows * wl.Hkv * (wl.r_v + wl.r_k) * 2 * wl.d
+    peak, peak_kind = measured_peak()
+
+    # end to end: the chunk's k and v from pinned host memory, one step after another
+    k_h, v_h = k.cpu().pin_memory(), v.cpu().pin_memory()
+    k_d, v_d = torch.empty_like(k), torch.empty_like(v)
+    probe_h = torch.empty(wl.B, dtype=torch.int32).pin_memory()
+    for t in lens:
+        t.fill_(wl.T)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(W, W + K):
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        step(i, k_d, v_d)
+        probe_h.copy_(lens[i], non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms, e2e_value = replica_throughput(e0.elapsed_time(e1), per_step * K, dist, "cuda")
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": "BasisKV prefill-chunk append, achieved HBM TB/s (Qwen3-32B layer, 4096-token chunks)",
+        "value": value, "unit": "TB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_step, "us_per_chunk": ms_step * 1e3 / wl.B,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 operands, fp32 accumulate" + (", e4m3 caches" if wl.cache_fp8 else ""),
+        "data": "synthetic (seeded generators)",
+        "config": {"workload": wl.name, "chunks_per_step": wl.B, "chunk_tokens": n,
+                   "rows_per_step": rows, "global_batch": wl.B * world, "seq_len": wl.T,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": f"{per_step / 1e6:.0f} MB streamed per step; no flush"},
+        "bytes_per_step": per_step,
+        "roofline": {"bound": "hbm", "kernel": "append_tc_kernel (+ the length update)",
+                     "achieved": per_step / (ms_step / 1e3) / 1e9, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": per_step / (ms_step / 1e3) / 1e9 / peak, "traffic": None,
+                     "tensor_tflops": flops / (ms_step / 1e3) / 1e12},
+        "cpu_baseline": None,
+        "e2e": {"value": e2e_value, "unit": "TB/s", "ms_per_step": e2e_ms / K,
+                "h2d_bytes_per_step": 2 * k.numel() * 2, "d2h_bytes_per_step": wl.B * 4},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def _route_source_sha() -> str:
     import hashlib
     h = hashlib.sha256()
@@ -616,6 +729,9 @@ def main():
                          "newest page); b16r16: the pages' narrow router and budget")
     ap.add_argument("--cache", default="bf16", choices=["bf16", "e4m3"],
                     help="element type of the K, Z and E caches")
+    ap.add_argument("--prefill", action="store_true",
+                    help="time the prefill-chunk append (Qwen3-32B layer, 4096-token chunks) "
+                         "instead of the decode step")
     ap.add_argument("--stack", default="", choices=["", "avg64", "avg96"],
                     help="time the 32-layer stack with per-layer Value widths of this average "
                          "instead of one layer")
@@ -631,6 +747,8 @@ def main():
         run_reference(args)
     elif args.stack:
         run_stack(args)
+    elif args.prefill:
+        run_prefill(args)
     else:
         run_gpu(args)
 

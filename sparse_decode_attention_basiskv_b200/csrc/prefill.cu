@@ -8,7 +8,9 @@
 // with W_app,g of shape (r_v + r_k) x 2d.  fold_append_kernel builds W_app
 // (fp32 products, stored bf16) and append_tc_kernel runs the product:
 // 128-token M tiles, N = r_v + r_k, K = 2d, operands staged by TMA in
-// 128-byte-swizzled K-major tiles, a single thread issuing tcgen05.mma
+// 128-byte-swizzled K-major tiles through a two-slot ring (so two or three
+// CTAs share an SM and one CTA's loads overlap another's epilogue), a
+// single thread issuing tcgen05.mma
 // (kind::f16, bf16 inputs, fp32 accumulator in tensor memory), and four
 // epilogue warps that read the accumulator with tcgen05.ld and scatter the
 // bf16 z / e rows, and the exact Key, into the paged caches.  The folded
@@ -108,6 +110,7 @@ __global__ void __launch_bounds__(kFoldAppThreads) fold_append_kernel(FoldAppArg
 // ------------------------------------------------------------------- GEMM
 constexpr int kTcThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
 constexpr int kTcBM = 128, kTcBK = 64;
+constexpr int kTcSlots = 2;  // k-block ring
 
 __host__ __device__ constexpr uint32_t tc_idesc(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
@@ -131,17 +134,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* smem = align_smem_1k(smem_raw);
   const int d = a.d, nkb = 2 * d / kTcBK;  // k-blocks: first d/64 from v, then from k
   const int a_bytes = kTcBM * kTcBK * 2, b_bytes = N * kTcBK * 2;
-  uint8_t* a_tiles = smem;                       // nkb x 16 KB
-  uint8_t* b_tiles = smem + nkb * a_bytes;       // nkb x N*128 B
-  uint64_t* full = reinterpret_cast<uint64_t*>(b_tiles + nkb * b_bytes);
-  uint64_t* accum = full + 1;
+  uint8_t* a_tiles = smem;                           // kTcSlots x 16 KB
+  uint8_t* b_tiles = smem + kTcSlots * a_bytes;      // kTcSlots x N*128 B
+  uint64_t* full = reinterpret_cast<uint64_t*>(b_tiles + kTcSlots * b_bytes);
+  uint64_t* empty = full + kTcSlots;
+  uint64_t* accum = empty + kTcSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = blockIdx.y, m0 = blockIdx.x * kTcBM;
   const int rows = a.B * a.n_new;
 
   if (tid == 0) {
-    mbar_init(full, 1);
+    for (int s = 0; s < kTcSlots; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
     mbar_init(accum, 1);
     fence_barrier_init();
   }
@@ -162,36 +169,47 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmW);
-    mbar_arrive_expect_tx(full, nkb * (a_bytes + b_bytes));
     for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % kTcSlots;
+      // the slot is free once the MMAs that read its previous k-block are done
+      if (kb >= kTcSlots && !mbar_wait(&empty[s], ((kb / kTcSlots) - 1) & 1, a.status)) break;
+      mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
       const bool from_v = kb < nkb / 2;
       const int col = (from_v ? kb : kb - nkb / 2) * kTcBK;
       // 3-D maps over [rows][Hkv][d]: coordinates (column, head, row)
-      tma_load_3d(a_tiles + kb * a_bytes, from_v ? &tmV : &tmK, col, g, m0, full);
-      tma_load_2d(b_tiles + kb * b_bytes, &tmW, kb * kTcBK, g * N, full);
+      tma_load_3d(a_tiles + s * a_bytes, from_v ? &tmV : &tmK, col, g, m0, &full[s]);
+      tma_load_2d(b_tiles + s * b_bytes, &tmW, kb * kTcBK, g * N, &full[s]);
     }
   } else if (warp == 1 && lane == 0) {  // ------------------------------ MMA
-    if (mbar_wait(full, 0, a.status)) {
+    const uint32_t idesc = tc_idesc(kTcBM, N);
+    bool ok = true;
+    for (int kb = 0; kb < nkb && ok; ++kb) {
+      const int s = kb % kTcSlots;
+      ok = mbar_wait(&full[s], (kb / kTcSlots) & 1, a.status);
+      if (!ok) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t idesc = tc_idesc(kTcBM, N);
-      for (int kb = 0; kb < nkb; ++kb) {
-        const uint64_t da = tc_sdesc(smem_u32(a_tiles + kb * a_bytes));
-        const uint64_t db = tc_sdesc(smem_u32(b_tiles + kb * b_bytes));
+      const uint64_t da = tc_sdesc(smem_u32(a_tiles + s * a_bytes));
+      const uint64_t db = tc_sdesc(smem_u32(b_tiles + s * b_bytes));
 #pragma unroll
-        for (int k = 0; k < kTcBK / 16; ++k) {
-          const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-          asm volatile(
-              "{ .reg .pred p; setp.ne.b32 p, %4, 0;"
-              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem),
-              "l"(da + 2 * k), "l"(db + 2 * k), "r"(idesc), "r"(acc)
-              : "memory");
-        }
+      for (int k = 0; k < kTcBK / 16; ++k) {
+        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+        asm volatile(
+            "{ .reg .pred p; setp.ne.b32 p, %4, 0;"
+            " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem),
+            "l"(da + 2 * k), "l"(db + 2 * k), "r"(idesc), "r"(acc)
+            : "memory");
       }
+      // slot s is released when these MMAs complete
+      asm volatile(
+          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+              smem_u32(&empty[s]))
+          : "memory");
+    }
+    if (ok)
       asm volatile(
           "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
               smem_u32(accum))
           : "memory");
-    }
   } else if (warp >= 2) {  // ---------------------------------------- epilogue
     const int quarter = warp & 3;
     const int r = m0 + quarter * 32 + lane;  // token row of the chunk
@@ -263,19 +281,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
     if (ok && live) {  // the exact Key, copied as is (E4M3: rounded)
-      const uint4* src = reinterpret_cast<const uint4*>(a.k_new + ((size_t)r * a.Hkv + g) * d);
-      if (a.fp8) {
+      // The row is still in shared memory: the last d/64 k-blocks staged for
+      // the product are the Key's columns (128-byte rows, 16-byte chunk j of
+      // row t stored at chunk j ^ (t & 7)).
+      const int t = quarter * 32 + lane;
+      // acquire the staged tiles' TMA writes (their last phases are complete)
+      bool kok = true;
+      for (int kb = nkb / 2; kb < nkb; ++kb)
+        kok = kok && mbar_wait(&full[kb % kTcSlots], (kb / kTcSlots) & 1, a.status);
+      uint4 kr[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (i < d / 8) {
+          const int kb = nkb / 2 + i / 8;  // the k-block of columns 8i .. 8i + 7
+          const uint8_t* tile = a_tiles + (kb % kTcSlots) * a_bytes;
+          kr[i] = *reinterpret_cast<const uint4*>(tile + t * 128 + (((i & 7) ^ (t & 7)) << 4));
+        }
+      }
+      if (!kok) {
+      } else if (a.fp8) {
         uint2* dstk = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(a.K_cache) + slot * d);
-        for (int i = 0; i < d / 8; ++i) {
-          const uint4 x = src[i];
-          const float2 f0 = bf16x2_to_f2(x.x), f1 = bf16x2_to_f2(x.y), f2 = bf16x2_to_f2(x.z),
-                       f3 = bf16x2_to_f2(x.w);
-          dstk[i] = make_uint2(f_to_e4m3x2(f0.x, f0.y) | (f_to_e4m3x2(f1.x, f1.y) << 16),
-                               f_to_e4m3x2(f2.x, f2.y) | (f_to_e4m3x2(f3.x, f3.y) << 16));
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (i < d / 8) {
+            const uint4 x = kr[i];
+            const float2 f0 = bf16x2_to_f2(x.x), f1 = bf16x2_to_f2(x.y), f2 = bf16x2_to_f2(x.z),
+                         f3 = bf16x2_to_f2(x.w);
+            dstk[i] = make_uint2(f_to_e4m3x2(f0.x, f0.y) | (f_to_e4m3x2(f1.x, f1.y) << 16),
+                                 f_to_e4m3x2(f2.x, f2.y) | (f_to_e4m3x2(f3.x, f3.y) << 16));
+          }
         }
       } else {
         uint4* dstk = reinterpret_cast<uint4*>(a.K_cache + slot * d);
-        for (int i = 0; i < d / 8; ++i) dstk[i] = src[i];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (i < d / 8) dstk[i] = kr[i];
       }
     }
   }
@@ -312,8 +352,10 @@ cudaError_t launch_append_tc(const AppendArgs& a, const CUtensorMap& tmV, const 
                              const CUtensorMap& tmW, cudaStream_t st, bool pdl) {
   const int N = a.r_v + a.r_k;
   const int tmem_cols = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
-  const int nkb = 2 * a.d / kTcBK;
-  const size_t smem = (size_t)nkb * (kTcBM * kTcBK * 2 + N * kTcBK * 2) + 64 + 1024;
+  size_t smem = (size_t)kTcSlots * (kTcBM * kTcBK * 2 + N * kTcBK * 2) + 64 + 1024;
+  // At most 512 / tmem_cols CTAs per SM may hold tensor memory at once: with
+  // 256 columns keep it to two by shared memory (three would need <= 75 KB).
+  if (tmem_cols > 128 && smem < 76 * 1024) smem = 76 * 1024;
   cudaError_t e = cudaFuncSetAttribute(append_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
