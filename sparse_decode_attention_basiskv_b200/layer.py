@@ -58,6 +58,14 @@ class DecodeLayer:
                        self.P_K, self.U_K, self.K, self.Z, self.E, self.workspace, stream,
                        W_app=self.W_app)
 
+    def capture(self, q, k_new=None, v_new=None, max_seq_len=None) -> "DecodeGraph":
+        """Captures one decode step reading q (and k_new, v_new) as static
+        buffers into a CUDA graph; replaying it runs the step again with
+        whatever those buffers hold.  Run one eager step first (the library
+        looks up its device state on its first call)."""
+        msl = self.max_seq_len if max_seq_len is None else max_seq_len
+        return DecodeGraph(lambda: self.decode(q, k_new, v_new, max_seq_len=msl))
+
     def decode(self, q, k_new=None, v_new=None, sel=None, max_seq_len=None, y=None,
                stream=None) -> torch.Tensor:
         """One decode step: optional append of (k_new, v_new), then routing,
@@ -71,6 +79,32 @@ class DecodeLayer:
         return y
 
 
+class DecodeGraph:
+    """A CUDA graph of decode steps replayed without host launch overhead.
+
+    The captured step reads its inputs from static device buffers (copy the
+    step's q, k_new, v_new into them before each replay) and writes y into a
+    static buffer; the sequence lengths live on the device and advance inside
+    the step, so one graph serves every step while the lengths stay within
+    the max_seq_len it was captured with."""
+
+    def __init__(self, fn, warmup_stream=None):
+        import torch
+        s = torch.cuda.Stream() if warmup_stream is None else warmup_stream
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            self.graph.capture_begin()
+            try:
+                self.out = fn()
+            finally:
+                self.graph.capture_end()
+        torch.cuda.current_stream().wait_stream(s)
+
+    def replay(self):
+        self.graph.replay()
+        return self.out
+
+
 class DecodeStack:
     """The attention blocks of a layer stack run in order on one stream, each
     layer with its own Value width (and so its own cache widths, factors and
@@ -82,6 +116,11 @@ class DecodeStack:
     @property
     def widths(self) -> list:
         return [L.dims.r_v for L in self.layers]
+
+    def capture(self, qs, ks=None, vs=None, max_seq_len=None) -> DecodeGraph:
+        """One CUDA graph of a decode step through every layer (static input
+        buffers qs, ks, vs; see DecodeLayer.capture)."""
+        return DecodeGraph(lambda: self.decode(qs, ks, vs, max_seq_len=max_seq_len))
 
     def decode(self, qs, ks=None, vs=None, max_seq_len=None, ys=None, stream=None) -> list:
         """One decode step of every layer: layer l gets qs[l] (and ks[l],
