@@ -461,6 +461,7 @@ struct SelShared {
   int sh[32];        // scan scratch
   uint32_t digit;
   int rem;
+  int done;  // the chosen bucket is taken whole: later digits are not needed
 };
 
 // Exclusive prefix sum over a block of NT threads; *total receives the sum.
@@ -592,6 +593,7 @@ __device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32
             if (start + hist[dg] >= rem) {
               ss.digit = (uint32_t)dg;
               ss.rem = rem - start;
+              ss.done = hist[dg] == rem - start;
               break;
             }
             start += hist[dg];
@@ -604,6 +606,13 @@ __device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32
       prefix |= ss.digit << shift;
       pmask |= 0xffu << shift;
       rem = ss.rem;
+      // Every key of the bucket is taken: with the remaining digits zero the
+      // threshold is at or below all of them, so the keys above it plus all
+      // keys equal to it are exactly the bucket and everything above.
+      if (ss.done) {
+        rem = n;
+        break;
+      }
     }
   }
   const uint32_t thr = prefix;
