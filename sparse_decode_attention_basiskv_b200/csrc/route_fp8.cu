@@ -44,12 +44,20 @@ template <int RB, int RQ, int S>
 constexpr int r8_pages_per_batch() {
   return r8_page_regs<RB, RQ, S>() <= 8 ? 2 : 1;
 }
+// CTAs per SM from the registers a lane holds for two batches and its
+// accumulators: four (64 registers a thread) up to 28 for the full-width
+// routers, three up to 40.  Measured at the 32K-context, B = 16 Llama-8B
+// shape (28): four CTAs 77.9 us, three 81.1 us; the narrow routers' batch
+// bookkeeping spills at 64 registers.
+template <int RB, int RQ, int S, int G>
+constexpr int r8_live_regs() {
+  return 2 * r8_pages_per_batch<RB, RQ, S>() * r8_page_regs<RB, RQ, S>() + (S / 16) * (G / 4) * 4;
+}
 template <int G, int RB, int RQ, int S>
 constexpr int r8_ctas_per_sm() {
-  return 2 * r8_pages_per_batch<RB, RQ, S>() * r8_page_regs<RB, RQ, S>() + (S / 16) * (G / 4) * 4 <=
-                 40
-             ? 3
-             : 2;
+  return (RB >= 64 && r8_live_regs<RB, RQ, S, G>() <= 28)
+             ? 4
+             : (r8_live_regs<RB, RQ, S, G>() <= 40 ? 3 : 2);
 }
 
 template <int G, int RV, int RK, int RB, int RQ, int S, int PW>
