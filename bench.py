@@ -47,6 +47,7 @@ from sparse_decode_attention_basiskv_b200 import synth  # noqa: E402
 METRIC = "BasisKV decode µs/step & achieved HBM TB/s vs peak (Llama-8B shape, 32K ctx)"
 WL = synth.LLAMA8B_T32K_B16
 N_QUERIES = 4  # distinct planted query sets cycled over the steps
+N_TOKENS = 8   # distinct appended tokens per layer cycled over the steps (--stack)
 
 
 def algorithmic_bytes(wl, T: int, append: bool = True) -> dict:
@@ -463,9 +464,10 @@ def run_stack(args) -> None:
         pb = synth.make_problem(wl, device="cuda", layer=l)
         layers.append(DecodeLayer.from_problem(pb))
         qs.append([pb.q, synth.make_query(wl, pb.cache["K"], wl.T, step=1)[0]])
-        k_all, v_all = synth.make_tokens(wl, pb.factors, K + W, device="cuda", stream_id=l)
-        ks.append([k_all[:, i].contiguous() for i in range(K + W)])
-        vs.append([v_all[:, i].contiguous() for i in range(K + W)])
+        # eight distinct tokens per layer, cycled over the steps (bounded memory)
+        k_all, v_all = synth.make_tokens(wl, pb.factors, N_TOKENS, device="cuda", stream_id=l)
+        ks.append([k_all[:, i].contiguous() for i in range(N_TOKENS)])
+        vs.append([v_all[:, i].contiguous() for i in range(N_TOKENS)])
         del pb, k_all, v_all
         torch.cuda.empty_cache()
     stack = DecodeStack(layers)
@@ -473,8 +475,8 @@ def run_stack(args) -> None:
     stream = torch.cuda.current_stream()
 
     def step(i, T_after):
-        stack.decode([q[i % 2] for q in qs], [k[i] for k in ks], [v[i] for v in vs],
-                     max_seq_len=T_after)
+        stack.decode([q[i % 2] for q in qs], [k[i % N_TOKENS] for k in ks],
+                     [v[i % N_TOKENS] for v in vs], max_seq_len=T_after)
 
     def barrier():
         if dist is not None:
@@ -527,38 +529,68 @@ def run_stack(args) -> None:
     peak, peak_kind = measured_peak()
     achieved = route_bytes / (route_ms / 1e3) / 1e9
 
-    # end to end through the public API: q, k, v of every layer in, y out
+    # end to end through the public API: every layer's q, k, v of a step as
+    # one packed copy from pinned host memory into one of two device slots,
+    # and every layer's y back as one copy, on a copy stream that overlaps
+    # the neighbouring steps' compute (as in the single-layer bench)
     for L in layers:
         L.seq_lens.fill_(T0)
-    q_h = [[q.cpu().pin_memory() for q in ql] for ql in qs]
-    k_h = [[k.cpu().pin_memory() for k in kl] for kl in ks]
-    v_h = [[v.cpu().pin_memory() for v in vl] for vl in vs]
-    q_d = [torch.empty_like(ql[0]) for ql in qs]
-    k_d = [torch.empty_like(kl[0]) for kl in ks]
-    v_d = [torch.empty_like(vl[0]) for vl in vs]
-    y_h = [torch.empty(base.B, base.hidden, dtype=torch.bfloat16).pin_memory() for _ in layers]
+    nL = len(layers)
+    nq, nk = qs[0][0].numel(), ks[0][0].numel()
+    per = nq + 2 * nk
+    packed_h = []
+    for i in range(N_TOKENS):  # step i uses packed_h[i % N_TOKENS]
+        parts = []
+        for l in range(nL):
+            parts += [qs[l][i % 2].reshape(-1), ks[l][i].reshape(-1), vs[l][i].reshape(-1)]
+        packed_h.append(torch.cat(parts).cpu().pin_memory())
+    slots = [torch.empty(nL * per, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    views = [[(sl[l * per:l * per + nq].view_as(qs[l][0]),
+               sl[l * per + nq:l * per + nq + nk].view_as(ks[l][0]),
+               sl[l * per + nq + nk:(l + 1) * per].view_as(vs[l][0])) for l in range(nL)]
+             for sl in slots]
+    ybuf = [torch.empty(nL, base.B, base.hidden, dtype=torch.bfloat16, device="cuda")
+            for _ in range(2)]
+    y_h = [torch.empty(nL, base.B, base.hidden, dtype=torch.bfloat16).pin_memory()
+           for _ in range(2)]
+    cs = torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step(i, T_after):
-        for l in range(len(layers)):
-            q_d[l].copy_(q_h[l][i % 2], non_blocking=True)
-            k_d[l].copy_(k_h[l][i], non_blocking=True)
-            v_d[l].copy_(v_h[l][i], non_blocking=True)
-        ys = stack.decode(q_d, k_d, v_d, max_seq_len=T_after)
-        for l, y in enumerate(ys):
-            y_h[l].copy_(y, non_blocking=True)
+    def e2e_run(first, last, start_ev=None):
+        if start_ev is not None:
+            cs.wait_event(start_ev)
+        with torch.cuda.stream(cs):
+            slots[first % 2].copy_(packed_h[first % N_TOKENS], non_blocking=True)
+            ev_in[first % 2].record(cs)
+        for i in range(first, last):
+            s_ = i % 2
+            if i + 1 < last:  # next inputs while this step computes
+                with torch.cuda.stream(cs):
+                    if i >= first + 1:
+                        cs.wait_event(ev_out[(i + 1) % 2])  # step i - 1 has read its slot
+                    slots[(i + 1) % 2].copy_(packed_h[(i + 1) % N_TOKENS], non_blocking=True)
+                    ev_in[(i + 1) % 2].record(cs)
+            stream.wait_event(ev_in[s_])
+            v_ = views[s_]
+            stack.decode([x[0] for x in v_], [x[1] for x in v_], [x[2] for x in v_],
+                         max_seq_len=T0 + i + 1, ys=list(ybuf[s_].unbind(0)))
+            ev_out[s_].record(stream)
+            with torch.cuda.stream(cs):
+                cs.wait_event(ev_out[s_])
+                y_h[s_].copy_(ybuf[s_], non_blocking=True)
+        stream.wait_stream(cs)
 
-    for i in range(W):
-        e2e_step(i, T0 + i + 1)
+    e2e_run(0, W)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(W, W + K):
-        e2e_step(i, T0 + i + 1)
+    e2e_run(W, W + K, e0)
     e1.record(stream)
     barrier()
     e2e_ms, e2e_value = replica_throughput(e0.elapsed_time(e1), total_bytes, dist, "cuda")
-    h2d = sum((q[0].numel() + k[0].numel() + v[0].numel()) * 2 for q, k, v in zip(qs, ks, vs))
-    d2h = len(layers) * base.B * base.hidden * 2
+    h2d = nL * per * 2
+    d2h = nL * base.B * base.hidden * 2
 
     if dist is not None:
         dist.barrier()

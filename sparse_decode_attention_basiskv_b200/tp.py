@@ -123,7 +123,6 @@ class TPDecodeLayer:
         g0, g1, _, _ = head_shard(wl.Hq, wl.Hkv, world, rank)
         fl = {k: v.to(device).contiguous()
               for k, v in shard_factors(pb.factors, wl.Hq, wl.Hkv, wl.d, world, rank).items()}
-        wl_l = synth.with_sizes(wl, Hq=wl.Hq // world, Hkv=wl.Hkv // world)
         lead = wl.tile_lead()
         table = pb.table.to(device).contiguous()
         caches = {k: synth.storage(wl, synth.paginate(v[:, g0:g1].to(device), table,
@@ -134,7 +133,6 @@ class TPDecodeLayer:
             W_fold = torch.empty(wl.hidden, wl.Hq * wl.r_v, dtype=torch.bfloat16, device=device)
             basiskv_fold_outproj(full, pb.factors["B_V"].to(device).contiguous(),
                                  pb.factors["W_O"].to(device).contiguous(), W_fold)
-        del wl_l
         return cls(full, world, rank, fl, caches, table, pb.seq_lens.to(device).clone(),
                    wl.top_k, pc * wl.page_size, W_fold, gather, compute, a_src)
 
