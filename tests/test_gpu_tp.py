@@ -27,6 +27,9 @@ CASES = {
     "qwen_tp2": (synth.with_sizes(synth.QWEN32B_T64K_B8, B=2, T=1200, prefill_tokens=0,
                                   top_k=16), 2),
     "llama_tp2_e4m3": (synth.with_sizes(synth.LLAMA8B_T32K_B16_FP8, B=4, T=1500, top_k=24), 2),
+    # the pages' narrow router (split tiles) across two ranks
+    "llama_b16r16_tp2": (synth.with_sizes(synth.LLAMA8B_T32K_B16_B16R16, B=4, T=1500, top_k=24),
+                         2),
 }
 
 
