@@ -77,57 +77,8 @@ __global__ void __launch_bounds__(kR8Threads, (r8_ctas_per_sm<G, RB, RQ, S>()))
   // The lengths, block table and caches are not written by the launch this
   // kernel follows; the grid-dependency wait comes before the folded
   // queries are read.
-  const int P_max = (a.max_seq_len + S - 1) / S;
-  const long total = (long)a.B * a.Hkv * P_max;
-  long u = total * wid / nw;
-  const long u_end = total * (wid + 1) / nw;
-  if (u >= u_end) return;
-  int bg = (int)(u / P_max), lp = (int)(u - (long)bg * P_max);
-  int b = bg / a.Hkv, g = bg - b * a.Hkv;
-  int T = clamp_len(a.seq_lens[b] + a.len_offset, a.max_seq_len, a.status, lane == 0 && lp == 0);
-  int P = (T + S - 1) / S;
-  auto advance = [&]() {
-    ++u;
-    if (++lp == P_max) {
-      lp = 0;
-      ++bg;
-      if (++g == a.Hkv) {
-        g = 0;
-        ++b;
-        if (u < u_end) {
-          T = clamp_len(a.seq_lens[b] + a.len_offset, a.max_seq_len, a.status, lane == 0);
-          P = (T + S - 1) / S;
-        }
-      }
-    }
-  };
-  auto skip = [&]() {
-    while (u < u_end && lp >= P) {
-      u += P_max - 1 - lp;
-      lp = P_max - 1;
-      advance();
-    }
-  };
-  // Block-table window: lane i holds entry win_base + i of sequence win_b,
-  // the next 32 entries requested as soon as a window opens.
-  int win_b = -1, win_base = 0, tb_cur = 0, tb_nxt = 0;
-  auto tbl = [&](int bb, int i) -> int {
-    return i < a.max_pages ? __ldg(a.block_table + (size_t)bb * a.max_pages + i) : 0;
-  };
-  auto page_of = [&](int bb, int l) -> int {
-    if (bb != win_b || l < win_base || l >= win_base + 32) {
-      if (bb == win_b && l >= win_base + 32 && l < win_base + 64) {
-        tb_cur = tb_nxt;
-        win_base += 32;
-      } else {
-        win_b = bb;
-        win_base = l;
-        tb_cur = tbl(bb, l + lane);
-      }
-      tb_nxt = tbl(bb, win_base + 32 + lane);
-    }
-    return __shfl_sync(0xffffffffu, tb_cur, l - win_base);
-  };
+  PageWalk<S> w(a, wid, nw, lane);
+  if (!w.more()) return;
 
   // B fragments of the current group, per warp in shared memory:
   // [chunk][k-step][N-tile][lane] -> (b0, b1); each lane writes and reads
@@ -185,17 +136,17 @@ __global__ void __launch_bounds__(kR8Threads, (r8_ctas_per_sm<G, RB, RQ, S>()))
   auto issue = [&](Batch& bt, uint2 (&x)[PW][NT][NC]) {
 #pragma unroll
     for (int k = 0; k < PW; ++k) {
-      bt.bg[k] = bg;
-      bt.lp[k] = lp;
-      bt.nv[k] = u < u_end ? min(S, T - lp * S) : 0;
+      bt.bg[k] = w.bg;
+      bt.lp[k] = w.lp;
+      bt.nv[k] = w.more() ? min(S, w.T - w.lp * S) : 0;
       if (bt.nv[k] > 0) {
-        int pp = page_of(b, lp);
+        int pp = w.page_of(w.b, w.lp);
         if (pp < 0 || pp >= a.num_phys) {
           if (lane == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
           pp = 0;  // the page's score is flagged garbage
         }
         // a narrow router's columns lead each tile: [S][RB] then the rest
-        const size_t tile = (size_t)pp * a.Hkv + g;
+        const size_t tile = (size_t)pp * a.Hkv + w.g;
         const uint8_t* zr =
             reinterpret_cast<const uint8_t*>(a.Z) + tile * S * RV + lr * ZP + 8 * lc;
         const uint8_t* er =
@@ -217,8 +168,8 @@ __global__ void __launch_bounds__(kR8Threads, (r8_ctas_per_sm<G, RB, RQ, S>()))
               ldg_stream8(x[k][t][c], er + t * 8 * EP + 32 * (c - NCZ));
           }
         }
-        advance();
-        skip();
+        w.advance();
+        w.skip();
       }
     }
   };
@@ -295,7 +246,7 @@ __global__ void __launch_bounds__(kR8Threads, (r8_ctas_per_sm<G, RB, RQ, S>()))
     }
   };
 
-  skip();
+  w.skip();
   Batch b0, b1;
   uint2 x0[PW][NT][NC], x1[PW][NT][NC];
   issue(b0, x0);

@@ -19,6 +19,82 @@ __device__ __forceinline__ int clamp_len(int T, int max_seq_len, unsigned int* s
   return T;
 }
 
+// A warp's contiguous range of pages in (sequence, KV head, logical page)
+// order, skipping pages past each sequence's length, with a 32-entry window
+// of the block table per lane: the next window is requested as soon as one
+// opens, so walking a sequence's pages never waits on the table.
+template <int S>
+struct PageWalk {
+  const int32_t* seq_lens;
+  const int32_t* block_table;
+  unsigned int* status;
+  int Hkv, max_pages, max_seq_len, len_offset, lane, P_max;
+  long u, u_end;
+  int bg, lp, b, g, T, P;
+  int win_b, win_base, tb_cur, tb_nxt;
+
+  __device__ __forceinline__ PageWalk(const RouteArgs& a, long wid, long nw, int lane_)
+      : seq_lens(a.seq_lens), block_table(a.block_table), status(a.status), Hkv(a.Hkv),
+        max_pages(a.max_pages), max_seq_len(a.max_seq_len), len_offset(a.len_offset),
+        lane(lane_), bg(0), lp(0), b(0), g(0), T(0), P(0), win_b(-1), win_base(0), tb_cur(0),
+        tb_nxt(0) {
+    P_max = (max_seq_len + S - 1) / S;
+    const long total = (long)a.B * Hkv * P_max;
+    u = total * wid / nw;
+    u_end = total * (wid + 1) / nw;
+    if (u < u_end) {
+      bg = (int)(u / P_max);
+      lp = (int)(u - (long)bg * P_max);
+      b = bg / Hkv;
+      g = bg - b * Hkv;
+      T = clamp_len(seq_lens[b] + len_offset, max_seq_len, status, lane == 0 && lp == 0);
+      P = (T + S - 1) / S;
+    }
+  }
+  __device__ __forceinline__ bool more() const { return u < u_end; }
+  __device__ __forceinline__ void advance() {
+    ++u;
+    if (++lp == P_max) {
+      lp = 0;
+      ++bg;
+      if (++g == Hkv) {
+        g = 0;
+        ++b;
+        if (u < u_end) {
+          T = clamp_len(seq_lens[b] + len_offset, max_seq_len, status, lane == 0);
+          P = (T + S - 1) / S;
+        }
+      }
+    }
+  }
+  // to the next page inside its sequence's length
+  __device__ __forceinline__ void skip() {
+    while (u < u_end && lp >= P) {
+      u += P_max - 1 - lp;
+      lp = P_max - 1;
+      advance();
+    }
+  }
+  __device__ __forceinline__ int tbl(int bb, int i) const {
+    return i < max_pages ? __ldg(block_table + (size_t)bb * max_pages + i) : 0;
+  }
+  // Physical page of logical page l of sequence bb (warp-uniform arguments).
+  __device__ __forceinline__ int page_of(int bb, int l) {
+    if (bb != win_b || l < win_base || l >= win_base + 32) {
+      if (bb == win_b && l >= win_base + 32 && l < win_base + 64) {
+        tb_cur = tb_nxt;
+        win_base += 32;
+      } else {
+        win_b = bb;
+        win_base = l;
+        tb_cur = tbl(bb, l + lane);
+      }
+      tb_nxt = tbl(bb, win_base + 32 + lane);
+    }
+    return __shfl_sync(0xffffffffu, tb_cur, l - win_base);
+  }
+};
+
 // -------------------------------------- page scoring, plain loads + MMA
 // The same scores without TMA or a staging ring: one warp scores one page
 // at a time straight from plain 16-byte global loads (PW pages per batch,
@@ -114,59 +190,8 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S>()))
 
   // Work: pages (sequence, KV head, logical page) in that order; warp wid
   // takes a contiguous range.  Pages past a sequence's length are skipped.
-  const int P_max = (a.max_seq_len + S - 1) / S;
-  const long total = (long)a.B * a.Hkv * P_max;
-  long u = total * wid / nw;
-  const long u_end = total * (wid + 1) / nw;
-  if (u >= u_end) return;
-  int bg = (int)(u / P_max), lp = (int)(u - (long)bg * P_max);
-  int b = bg / a.Hkv, g = bg - b * a.Hkv;
-  int T = clamp_len(a.seq_lens[b] + a.len_offset, a.max_seq_len, a.status, lane == 0 && lp == 0);
-  int P = (T + S - 1) / S;
-  auto advance = [&]() {
-    ++u;
-    if (++lp == P_max) {
-      lp = 0;
-      ++bg;
-      if (++g == a.Hkv) {
-        g = 0;
-        ++b;
-        if (u < u_end) {
-          T = clamp_len(a.seq_lens[b] + a.len_offset, a.max_seq_len, a.status, lane == 0);
-          P = (T + S - 1) / S;
-        }
-      }
-    }
-  };
-  auto skip = [&]() {  // to the next page inside its sequence's length
-    while (u < u_end && lp >= P) {
-      u += P_max - 1 - lp;
-      lp = P_max - 1;
-      advance();
-    }
-  };
-
-  // Block-table window: lane i holds entry win_base + i of sequence win_b;
-  // the next 32 entries are fetched as soon as a window opens, so walking a
-  // sequence's pages never waits on the table.
-  int win_b = -1, win_base = 0, tb_cur = 0, tb_nxt = 0;
-  auto tbl = [&](int bb, int i) -> int {
-    return i < a.max_pages ? __ldg(a.block_table + (size_t)bb * a.max_pages + i) : 0;
-  };
-  auto page_of = [&](int bb, int l) -> int {
-    if (bb != win_b || l < win_base || l >= win_base + 32) {
-      if (bb == win_b && l >= win_base + 32 && l < win_base + 64) {
-        tb_cur = tb_nxt;
-        win_base += 32;
-      } else {
-        win_b = bb;
-        win_base = l;
-        tb_cur = tbl(bb, l + lane);
-      }
-      tb_nxt = tbl(bb, win_base + 32 + lane);
-    }
-    return __shfl_sync(0xffffffffu, tb_cur, l - win_base);
-  };
+  PageWalk<S> w(a, wid, nw, lane);
+  if (!w.more()) return;
 
   // A fragments of the current group, per warp in shared memory:
   // [set][chunk][k-step][lane] -> (a0, a1, a2, a3).  Each lane writes and
@@ -204,27 +229,27 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S>()))
     }
   };
 
-  skip();
-  while (u < u_end) {
+  w.skip();
+  while (w.more()) {
     uint4 x[PW][NT][NC];
     int ubg[PW], ub[PW], ug[PW], ulp[PW], uT[PW];
     bool uok[PW];
 #pragma unroll
     for (int k = 0; k < PW; ++k) {  // issue every load of the batch
-      uok[k] = u < u_end;
-      ubg[k] = bg;
-      ub[k] = b;
-      ug[k] = g;
-      ulp[k] = lp;
-      uT[k] = T;
+      uok[k] = w.more();
+      ubg[k] = w.bg;
+      ub[k] = w.b;
+      ug[k] = w.g;
+      ulp[k] = w.lp;
+      uT[k] = w.T;
       if (uok[k]) {
-        int pp = page_of(b, lp);
+        int pp = w.page_of(w.b, w.lp);
         if (pp < 0 || pp >= a.num_phys) {
           if (lane == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
           pp = 0;  // the page's score is flagged garbage
         }
         // a narrow router's columns lead each tile: [S][RB] then the rest
-        const size_t tile = (size_t)pp * a.Hkv + g;
+        const size_t tile = (size_t)pp * a.Hkv + w.g;
         const uint16_t* zr = a.Z + tile * S * RV + lr * ZP + 8 * lc;
         const uint16_t* er = a.E + tile * S * RK + lr * EP + 8 * lc;
 #pragma unroll
@@ -246,8 +271,8 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S>()))
             }
           }
         }
-        advance();
-        skip();
+        w.advance();
+        w.skip();
       }
     }
     // This lane's maximum over page k's live tokens and the group's heads
