@@ -17,7 +17,9 @@ pytestmark = pytest.mark.gpu
     (synth.with_sizes(synth.LLAMA8B_T32K_B16, B=2, T=1500, top_k=24), [32, 64, 128, 96]),
     (synth.with_sizes(synth.QWEN32B_T64K_B8, B=2, T=1200, prefill_tokens=0, top_k=16),
      [64, 32, 96]),
-], ids=["llama", "qwen"])
+    # E4M3 caches (their scoring instances start at r_v 64)
+    (synth.with_sizes(synth.LLAMA8B_T32K_B16_FP8, B=2, T=1500, top_k=24), [96, 64, 128]),
+], ids=["llama", "qwen", "llama_e4m3"])
 def test_stack_with_per_layer_widths(base, widths):
     wls = synth.stack_layers(base, widths)
     pbs = [synth.make_problem(wl, device="cuda", layer=l) for l, wl in enumerate(wls)]
@@ -37,7 +39,8 @@ def test_stack_with_per_layer_widths(base, widths):
             c = {k: np64(v[b]) for k, v in pb.cache.items()}
             out = O.decode_sequence(np64(pb.q[b]), c["K"], c["Z"], c["E"], wl.T, wl.page_size,
                                     wl.top_k, f["P_K"], f["U_K"], W, k_new=np64(ks[l][b]),
-                                    v_new=np64(vs[l][b]), A_V=f["A_V"], **wl.router)
+                                    v_new=np64(vs[l][b]), A_V=f["A_V"], fp8=bool(wl.cache_fp8),
+                                    **wl.router)
             assert out["a"].shape[1] == widths[l]
             if not out["near_tie"].any():
                 assert_within(np64(ys[l][b]), out["y"], Y_REL, Y_ABS, what=f"layer {l} y b{b}")
