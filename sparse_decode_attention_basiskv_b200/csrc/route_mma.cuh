@@ -1,6 +1,6 @@
-// Page scoring from plain loads on the warp-level tensor cores (shared by
-// the bf16 instances in route.cu and the E4M3 instances in route_fp8.cu, so
-// the two sets compile in parallel).
+// Page scoring from plain loads on the warp-level tensor cores: the bf16
+// scoring kernel (instantiated in route.cu) and the page walk that the E4M3
+// scoring kernel (route_fp8.cu) shares with it.
 #pragma once
 
 #include "common.cuh"
@@ -118,7 +118,8 @@ constexpr int kRmWarps = kRmThreads / 32;
 // CTAs per SM: three (at most 85 registers a thread) when one page's loads
 // and accumulators fit, else two.  Measured at the 32K-context, B = 16
 // Llama-8B shape: one page in flight per warp with 24 warps per SM beats two
-// pages per warp with 16 warps (136 vs 153 us for fold + scoring + select).
+// pages per warp with 16 warps (136 vs 153 us for fold + scoring + select),
+// and four CTAs per SM at 64 registers (fold + scoring 130.4 vs 135.7 us).
 template <int G, int RB, int RQ, int S>
 __host__ __device__ constexpr int rm_ctas_per_sm() {
   return (S / 8) * ((RB + 31) / 32 + (RQ + 31) / 32) * 4 + (S / 8) * (G == 8 ? 2 : 1) * 4 <= 40
