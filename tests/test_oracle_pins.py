@@ -360,3 +360,16 @@ def test_v_rank_schedule_average_and_members():
         assert w == synth.v_rank_schedule(avg, 32)  # seeded
     layers = synth.stack_layers(synth.LLAMA8B_T32K_B16, [32, 64, 128])
     assert [L.r_v for L in layers] == [32, 64, 128] and len({L.name for L in layers}) == 3
+
+
+def test_synthetic_e4m3_caches_hold_e4m3_values():
+    """The E4M3 workloads' cache values are E4M3 numbers: the oracle's
+    rounding leaves them unchanged (and the filler past the length too)."""
+    from sparse_decode_attention_basiskv_b200 import synth
+    wl = synth.with_sizes(synth.TINY, T=100, cache_fp8=1)
+    pb = synth.make_problem(wl)
+    for name in ("K", "Z", "E"):
+        x = pb.cache[name].double().numpy()
+        np.testing.assert_array_equal(O.to_e4m3(x), x)
+    paged = pb.paged()
+    assert all(v.dtype == torch.float8_e4m3fn for v in paged.values())

@@ -1,5 +1,5 @@
-"""Host logic of the tensor-parallel layer (Figure 1): two gloo ranks on the
-CPU, each holding half of the KV heads, compute their heads' latents, gather
+"""Host logic of the tensor-parallel layer (Figure 1): two or four gloo ranks
+on the CPU, each holding its share of the KV heads, compute their heads' latents, gather
 them source-major and rebuild the complete output.  The per-rank compute is
 the oracle standing in for the kernels (no GPU here), so the test checks the
 head split, the factor and cache slicing, the gather order and the
@@ -9,11 +9,11 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-WORLD = 2
 
 
 def _free_port() -> int:
@@ -22,9 +22,10 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
-def _workload():
+def _workload(world):
     from sparse_decode_attention_basiskv_b200 import synth
-    return synth.with_sizes(synth.TINY, Hq=8, Hkv=2, T=200, top_k=6, n_planted=2)
+    return synth.with_sizes(synth.TINY, Hq=2 * world * 2, Hkv=2 * world, T=200, top_k=6,
+                            n_planted=2)
 
 
 class OracleCompute:
@@ -65,7 +66,7 @@ def _rank(rank: int, world: int, port: int, out):
     try:
         from sparse_decode_attention_basiskv_b200 import synth
         from sparse_decode_attention_basiskv_b200.tp import LatentGather, TPDecodeLayer, head_shard
-        wl = _workload()
+        wl = _workload(world)
         pb = synth.make_problem(wl)
         layer = TPDecodeLayer.from_problem(pb, world, rank, gather=LatentGather(),
                                            compute=OracleCompute(pb, world, rank), device="cpu")
@@ -78,27 +79,29 @@ def _rank(rank: int, world: int, port: int, out):
         dist.destroy_process_group()
 
 
-def test_tensor_parallel_two_gloo_ranks():
+@pytest.mark.parametrize("world", [2, 4])
+def test_tensor_parallel_gloo_ranks(world):
     from oracle import basiskv_oracle as O
     from sparse_decode_attention_basiskv_b200 import synth
     port = _free_port()
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(_rank, args=(WORLD, port, out), nprocs=WORLD, join=True,
+    mp.start_processes(_rank, args=(world, port, out), nprocs=world, join=True,
                        start_method="spawn")
-    wl = _workload()
+    wl = _workload(world)
     pb = synth.make_problem(wl)
     f = {k: v.double().numpy() for k, v in pb.factors.items()}
     W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
     y0, a0 = out[0]
-    y1, a1 = out[1]
-    np.testing.assert_array_equal(a0, a1)  # every rank holds every source's latents
-    np.testing.assert_array_equal(y0, y1)  # and rebuilds the same output
+    for r in range(1, world):
+        y1, a1 = out[r]
+        np.testing.assert_array_equal(a0, a1)  # every rank holds every source's latents
+        np.testing.assert_array_equal(y0, y1)  # and rebuilds the same output
     for b in range(wl.B):  # the unsharded step
         c = {k: v[b].double().numpy() for k, v in pb.cache.items()}
         r = O.decode_sequence(pb.q[b].double().numpy(), c["K"], c["Z"], c["E"], wl.T,
                               wl.page_size, wl.top_k, f["P_K"], f["U_K"], W)
-        a_ref = r["a"].reshape(WORLD, wl.Hq // WORLD, wl.r_v)
+        a_ref = r["a"].reshape(world, wl.Hq // world, wl.r_v)
         np.testing.assert_allclose(a0[:, b], a_ref, rtol=1e-2, atol=1e-2)  # bf16 latents
         ref = np.abs(r["y"]).max()
         assert np.abs(y0[b] - r["y"]).max() <= 1e-2 * ref + 1e-3
