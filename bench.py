@@ -420,7 +420,9 @@ def run_gpu(args) -> None:
                    **{k: v for k, v in wl.describe().items() if k not in ("name", "steps")}},
         "bytes_per_step": avg,
         "frac_of_peak": value / world / (peak / 1e3),
-        "roofline": {"bound": "hbm", "kernel": "route_mma_kernel (+ its query fold)",
+        "roofline": {"bound": "hbm",
+                     "kernel": ("route_f8_kernel" if wl.cache_fp8 else "route_mma_kernel")
+                     + " (+ its query fold)",
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                      "ms_per_launch": route_ms, "algorithmic_bytes": route_bytes},
