@@ -318,8 +318,10 @@ BASISKV_API int basiskv_outproj_sources(const basiskv_dims* dims, const basiskv_
  * process exits.  It allocates nothing itself.
  *   - Shapes whose basiskv_workspace_size exceeds the array return
  *     BASISKV_ERR_SCRATCH_LIMIT and launch nothing.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress with that device current); make that first call
+ *   - The array's device address belongs to the current CUDA context; each
+ *     call made outside stream capture looks it up (cudaGetSymbolAddress in
+ *     that context), and a call inside a capture uses the address its
+ *     context's last call found.  Make the first call in each context
  *     before any stream capture.
  *   - Every call on a device shares the one array, which keeps the previous
  *     call's contents (nothing in it needs to start at zero).  Calls that may
@@ -340,6 +342,19 @@ BASISKV_API int basiskv_decode_noalloc(const basiskv_dims* dims, const basiskv_b
  * BASISKV_ERR_DEVICE when it was non-zero, BASISKV_ERR_CUDA when the stream
  * itself reported an error. */
 BASISKV_API int basiskv_read_device_status(void* stream, uint32_t* flags);
+
+/* Self-test of the library's bounded waits.  The paper has no counterpart:
+ * this checks the failure path every kernel relies on.  Every wait of a
+ * kernel here on an mbarrier gives up after a time limit, records
+ * BASISKV_DEV_TIMEOUT in the device status word and lets the kernel return,
+ * so a wait that can never complete (a logic error, a copy that never
+ * lands) ends with a status the host can read instead of a hung GPU.  This
+ * call launches one CTA on `stream` that waits, through that same bounded
+ * wait, on an mbarrier nothing arrives on, with a limit of limit_ns
+ * nanoseconds (1 .. 1e9; anything else is BASISKV_ERR_INVALID_ARG before
+ * any CUDA call).  Afterwards basiskv_read_device_status reports
+ * BASISKV_DEV_TIMEOUT (and clears it); the context stays usable. */
+BASISKV_API int basiskv_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 
 /* Kernels this library has launched in this process so far (a host-side
  * counter; lets a caller count the launches inside a timed region). */

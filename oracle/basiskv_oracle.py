@@ -223,7 +223,8 @@ def decode_sequence(q: np.ndarray, K: np.ndarray, Z: np.ndarray, E: np.ndarray,
     widths and the kept pages (page_scores, select_pages).  fp8: the caches
     hold E4M3 values (the appended K, z and e are stored through to_e4m3
     instead of K as given and z, e through to_bf16).  Returns a dict with the
-    appended state, the scores, the selection, near-tie flags, a and y."""
+    appended state, the scores, the selection, near-tie flags, a and y, and
+    the caches the step read (K, Z, E: with the appended token, if any)."""
     Hkv = K.shape[0]
     Hq = q.shape[0]
     G = Hq // Hkv
@@ -252,5 +253,5 @@ def decode_sequence(q: np.ndarray, K: np.ndarray, Z: np.ndarray, E: np.ndarray,
         sels.append(sel)
         ties.append(tie)
     out.update(T=T, scores=scores, sel=np.stack(sels), near_tie=np.array(ties),
-               a=a, y=outproj(a, W_fold))
+               a=a, y=outproj(a, W_fold), K=K, Z=Z, E=E)
     return out

@@ -77,6 +77,7 @@ _SIGNATURES = {
     "basiskv_read_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "basiskv_strerror": (ctypes.c_char_p, [_I]),
     "basiskv_launch_count": (ctypes.c_uint64, []),
+    "basiskv_selftest_bounded_wait": (_I, [ctypes.c_uint64, _P]),
 }
 
 _lib = None
@@ -227,6 +228,13 @@ def read_device_status(stream=None) -> int:
     if rc not in (OK, ERR_DEVICE):
         raise BasisKVError(rc, "basiskv_read_device_status")
     return flags.value
+
+
+def basiskv_selftest_bounded_wait(limit_ns: int, stream=None) -> None:
+    """Launches the bounded-wait self-test (a wait that cannot complete,
+    given up after limit_ns); read_device_status() then shows DEV_TIMEOUT."""
+    _check(load_library().basiskv_selftest_bounded_wait(limit_ns, _stream(stream)),
+           "basiskv_selftest_bounded_wait")
 
 
 def launch_count() -> int:

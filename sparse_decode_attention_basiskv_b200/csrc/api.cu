@@ -182,6 +182,16 @@ int check_len_topk(const basiskv_dims* d, int top_k, int max_seq_len) {
   return BASISKV_OK;
 }
 
+}  // namespace
+
+// Shape, length and top_k checks of the decode entry points (host only).
+int basiskv::validate_decode_shape(const basiskv_dims* d, int top_k, int max_seq_len) {
+  const int rc = check_dims(d);
+  return rc ? rc : check_len_topk(d, top_k, max_seq_len);
+}
+
+namespace {
+
 struct WsLayout {
   size_t qt, scores, sel, selp, partial, a_f32, a_bf16, op_part, w_app, counters, total;
   int n_att_cnt, n_op_cnt;

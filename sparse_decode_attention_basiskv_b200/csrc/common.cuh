@@ -78,13 +78,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete; false on timeout.
+// Waits for the phase with the given parity to complete; false on timeout
+// (after limit_ns, with BASISKV_DEV_TIMEOUT raised in *status).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          unsigned int* status) {
+                                          unsigned int* status,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit_ns) {
       raise_status(status, BASISKV_DEV_TIMEOUT);
       return false;
     }

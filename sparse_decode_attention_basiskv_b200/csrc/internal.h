@@ -22,6 +22,9 @@ bool make_tmap_3d(CUtensorMap* out, const void* base, const uint64_t dims[3],
 
 // Address of this library's device status word on the current device.
 unsigned int* device_status_ptr();
+// BASISKV_OK, or the status basiskv_decode returns for these dims, top_k and
+// max_seq_len (host arithmetic only, before any CUDA call).
+int validate_decode_shape(const basiskv_dims* d, int top_k, int max_seq_len);
 
 int num_sms();
 

@@ -13,14 +13,16 @@
 // The array is a file-scope __device__ object, so every GPU that loads the
 // library holds kNoallocScratchBytes of it until the process exits.  Host
 // code must not hand the array's symbol to a kernel (on the host it is only
-// a stand-in, not a device address): its device address is looked up once
-// per device with cudaGetSymbolAddress, with that device current, the first
-// time the entry point runs there.
+// a stand-in, not a device address): its device address is looked up with
+// cudaGetSymbolAddress in the caller's current context, on every call made
+// outside stream capture.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 #include "../../include/basiskv.h"
+#include "internal.h"
 
 namespace {
 
@@ -28,22 +30,57 @@ constexpr size_t kNoallocScratchBytes = BASISKV_NOALLOC_SCRATCH_BYTES;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 64;
+// The array's address belongs to one CUDA context (the module is loaded per
+// context), so it is cached per context, not per device number: after a
+// cudaDeviceReset, or under another context on the same device, the old
+// address is stale.  Outside stream capture every call looks the address up
+// again (a cheap table lookup once the module is loaded) and refreshes the
+// cache; during capture, where a lookup that loads the module is not
+// allowed, the cached address of the current context is used.
+constexpr int kMaxContexts = 64;
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices];
+CUcontext g_ctx[kMaxContexts];
+void* g_ptr[kMaxContexts];
+int g_n;
 
-// Device address of the scratch array on the current device (set-up on the
-// first call per device).  Returns nullptr if the lookup fails.
-void* scratch_for_current_device() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_scratch_ptr[dev]) {
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CUcontext current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_scratch_ptr[dev] = p;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+// Device address of the scratch array in the current context, or nullptr.
+void* scratch_for_current_context(cudaStream_t st) {
+  // (a runtime call first: it makes the device's primary context current
+  // when the caller has none yet)
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return nullptr;
+  const CUcontext ctx = current_context();
+  if (!ctx) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  int slot = -1;
+  for (int i = 0; i < g_n; ++i)
+    if (g_ctx[i] == ctx) slot = i;
+  if (cap != cudaStreamCaptureStatusNone) return slot >= 0 ? g_ptr[slot] : nullptr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  if (slot < 0) {
+    slot = g_n < kMaxContexts ? g_n++ : (int)(reinterpret_cast<uintptr_t>(ctx) % kMaxContexts);
+    g_ctx[slot] = ctx;
   }
-  return g_scratch_ptr[dev];
+  g_ptr[slot] = p;
+  return p;
 }
 
 }  // namespace
@@ -57,13 +94,12 @@ int basiskv_decode_noalloc(const basiskv_dims* dims, const basiskv_bf16* q,
                            const basiskv_bf16* U_K, const basiskv_bf16* W_fold,
                            basiskv_bf16* K_cache, basiskv_bf16* Z_cache, basiskv_bf16* E_cache,
                            int top_k, int32_t* sel, basiskv_bf16* y, void* stream) {
-  const size_t need = basiskv_workspace_size(dims, top_k, max_seq_len);
-  if (need == 0)  // dims, top_k or length rejected: let the decode report which
-    return basiskv_decode(dims, q, k_new, v_new, seq_lens, max_seq_len, block_table, A_V, P_K,
-                          U_K, W_fold, K_cache, Z_cache, E_cache, top_k, sel, y, nullptr, 0,
-                          stream);
-  if (need > kNoallocScratchBytes) return BASISKV_ERR_SCRATCH_LIMIT;
-  void* scratch = scratch_for_current_device();
+  const int rc = basiskv::validate_decode_shape(dims, top_k, max_seq_len);
+  if (rc) return rc;
+  if (basiskv_workspace_size(dims, top_k, max_seq_len) > kNoallocScratchBytes)
+    return BASISKV_ERR_SCRATCH_LIMIT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* scratch = scratch_for_current_context(st);
   if (!scratch) return BASISKV_ERR_CUDA;
   return basiskv_decode(dims, q, k_new, v_new, seq_lens, max_seq_len, block_table, A_V, P_K, U_K,
                         W_fold, K_cache, Z_cache, E_cache, top_k, sel, y, scratch,

@@ -39,17 +39,27 @@ class DecodeLayer:
     @classmethod
     def from_problem(cls, pb, device="cuda", stream=None) -> "DecodeLayer":
         """Builds the layer of a synthetic workload (``synth.Problem``)."""
-        wl = pb.wl
+        return cls.from_parts(pb.wl, pb.factors, pb.paged(), pb.table, pb.seq_lens, device,
+                              stream)
+
+    @classmethod
+    def from_parts(cls, wl, factors: dict, paged: dict, table, seq_lens=None, device="cuda",
+                   stream=None) -> "DecodeLayer":
+        """Builds the layer of workload ``wl`` from its factors, its paged
+        caches (``synth.make_paged_cache`` or ``Problem.paged``) and block
+        table; lengths default to wl.T for every sequence."""
         pc = wl.pages_capacity()
         dims = Dims(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, hidden=wl.hidden, r_v=wl.r_v,
                     r_k=wl.r_k, page_size=wl.page_size, max_pages_per_seq=pc,
                     num_phys_pages=wl.B * pc, route_r_v=wl.route_r_v, route_r_k=wl.route_r_k,
                     sink_pages=wl.sink_pages, recent_pages=wl.recent_pages,
                     cache_fp8=wl.cache_fp8)
-        factors = {k: v.to(device).contiguous() for k, v in pb.factors.items()}
-        caches = {k: v.contiguous() for k, v in pb.paged().items()}
-        return cls(dims, factors, caches, pb.table.to(device).contiguous(),
-                   pb.seq_lens.to(device).clone(), wl.top_k, pc * wl.page_size, stream)
+        factors = {k: v.to(device).contiguous() for k, v in factors.items()}
+        caches = {k: v.contiguous() for k, v in paged.items()}
+        if seq_lens is None:
+            seq_lens = torch.full((wl.B,), wl.T, dtype=torch.int32)
+        return cls(dims, factors, caches, table.to(device).contiguous(),
+                   seq_lens.to(device).clone(), wl.top_k, pc * wl.page_size, stream)
 
     def append(self, k_new, v_new, n_new: int, stream=None) -> None:
         """Appends n_new tokens ([B][n_new][Hkv][d] bf16) to every sequence

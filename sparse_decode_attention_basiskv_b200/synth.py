@@ -225,6 +225,19 @@ def _dev_gen(device, seed: int) -> torch.Generator:
     return torch.Generator(device=device).manual_seed(seed)
 
 
+def _draw_sequence(wl: Workload, factors: dict, dev, layer: int, b: int) -> tuple:
+    """Cache values (z, e, K) [Hkv][T][*] of sequence b, as the cache holds
+    them (bf16 values, or E4M3 values for E4M3 caches)."""
+    P_K = factors["P_K"].to(dev, torch.float32)
+    U_K = factors["U_K"].to(dev, torch.float32)
+    gen = _dev_gen(dev, wl.seed * 1000 + 1 + 100003 * layer + 7919 * b)
+    z = torch.randn(wl.Hkv, wl.T, wl.r_v, generator=gen, device=dev).bfloat16()
+    e = torch.randn(wl.Hkv, wl.T, wl.r_k, generator=gen, device=dev).bfloat16()
+    noise = torch.randn(wl.Hkv, wl.T, wl.d, generator=gen, device=dev) * 0.1
+    k = torch.bmm(z.float(), P_K) + torch.bmm(e.float(), U_K.transpose(1, 2)) + noise
+    return as_cache_values(wl, z), as_cache_values(wl, e), as_cache_values(wl, k)
+
+
 def make_cache(wl: Workload, factors: dict, device="cpu", layer: int = 0,
                seqs=None) -> dict:
     """Logical caches [len(seqs)][Hkv][capacity][*] holding T tokens for each
@@ -232,22 +245,56 @@ def make_cache(wl: Workload, factors: dict, device="cpu", layer: int = 0,
     dev = torch.device(device)
     seqs = list(range(wl.B)) if seqs is None else list(seqs)
     Hkv, T, cap = wl.Hkv, wl.T, wl.capacity_tokens()
-    P_K = factors["P_K"].to(dev, torch.float32)
-    U_K = factors["U_K"].to(dev, torch.float32)
     n = len(seqs)
     Z = torch.full((n, Hkv, cap, wl.r_v), FILLER, dtype=torch.bfloat16, device=dev)
     E = torch.full((n, Hkv, cap, wl.r_k), FILLER, dtype=torch.bfloat16, device=dev)
     K = torch.full((n, Hkv, cap, wl.d), FILLER, dtype=torch.bfloat16, device=dev)
     for i, b in enumerate(seqs):  # one sequence at a time bounds the temporaries
-        gen = _dev_gen(dev, wl.seed * 1000 + 1 + 100003 * layer + 7919 * b)
-        z = torch.randn(Hkv, T, wl.r_v, generator=gen, device=dev).bfloat16()
-        e = torch.randn(Hkv, T, wl.r_k, generator=gen, device=dev).bfloat16()
-        noise = torch.randn(Hkv, T, wl.d, generator=gen, device=dev) * 0.1
-        k = torch.bmm(z.float(), P_K) + torch.bmm(e.float(), U_K.transpose(1, 2)) + noise
-        Z[i, :, :T] = as_cache_values(wl, z)
-        E[i, :, :T] = as_cache_values(wl, e)
-        K[i, :, :T] = as_cache_values(wl, k)
+        Z[i, :, :T], E[i, :, :T], K[i, :, :T] = _draw_sequence(wl, factors, dev, layer, b)
     return {"Z": Z, "E": E, "K": K}
+
+
+def make_paged_cache(wl: Workload, factors: dict, table: torch.Tensor, device="cpu",
+                     layer: int = 0) -> dict:
+    """The paged caches of ``Problem.paged()`` (same values, same layout and
+    element type) drawn one sequence at a time straight into the pages,
+    without the logical copy: for workloads whose cache is tens of GB."""
+    dev = torch.device(device)
+    S, pc, T = wl.page_size, wl.pages_capacity(), wl.T
+    n_phys = wl.B * pc
+    lead = wl.tile_lead()
+    widths = {"Z": wl.r_v, "E": wl.r_k, "K": wl.d}
+    dt = torch.float8_e4m3fn if wl.cache_fp8 else torch.bfloat16
+    out = {k: torch.full((n_phys, wl.Hkv, S, w), FILLER, dtype=torch.bfloat16,
+                         device=dev).to(dt) for k, w in widths.items()}
+    full = T // S  # whole pages; the partial last page keeps its filler rows
+    for b in range(wl.B):
+        vals = dict(zip(("Z", "E", "K"), _draw_sequence(wl, factors, dev, layer, b)))
+        phys = table[b].long().to(dev)
+        for name, x in vals.items():
+            w = widths[name]
+            if full:
+                tiles = x[:, :full * S].reshape(wl.Hkv, full, S, w).permute(1, 0, 2, 3)
+                out[name][phys[:full]] = storage(wl, split_tiles(tiles, lead.get(name, w)))
+            if T % S:
+                tail = torch.full((wl.Hkv, S, w), FILLER, dtype=torch.bfloat16, device=dev)
+                tail[:, :T % S] = x[:, full * S:T]
+                out[name][phys[full]] = storage(wl, split_tiles(tail, lead.get(name, w)))
+    return out
+
+
+class PagedKeys:
+    """Logical indexing K[b, g, t] of a paged Key cache through the block
+    table (what ``make_query`` reads when no logical cache exists)."""
+
+    def __init__(self, K_paged: torch.Tensor, table: torch.Tensor, page_size: int):
+        self.K, self.table, self.S = K_paged, table, page_size
+        self.device = K_paged.device
+
+    def __getitem__(self, idx) -> torch.Tensor:
+        b, g, t = idx
+        row = self.K[int(self.table[b, t // self.S]), g, t % self.S]
+        return row.float() if row.dtype == torch.float8_e4m3fn else row
 
 
 def planted_pages(wl: Workload, P: int | None = None) -> torch.Tensor:

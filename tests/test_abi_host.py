@@ -30,7 +30,7 @@ def lib():
 
 def test_header_symbols_are_exported(lib):
     names = bkv.header_symbols()
-    assert len(names) == 14
+    assert len(names) == 15
     out = subprocess.run(["nm", "-D", "--defined-only", bkv.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
@@ -219,3 +219,31 @@ def test_head_shard_covers_every_head_once():
          "W_O": torch.arange(8 * 3)[:, None]}
     s1 = shard_factors(f, 8, 2, 3, 2, 1)
     assert s1["A_V"].tolist() == [[1]] and s1["W_O"][:, 0].tolist() == list(range(12, 24))
+
+
+def test_selftest_wait_limit_validated(lib):
+    """The bounded-wait self-test refuses a limit of 0 or above one second
+    before any CUDA call."""
+    for bad in (0, 1_000_000_001, 2**63):
+        assert lib.basiskv_selftest_bounded_wait(bad, None) == bkv.ERR_INVALID_ARG
+
+
+def _noalloc(lib, dims, top_k, max_seq_len):
+    return lib.basiskv_decode_noalloc(ctypes.byref(dims), FAKE, FAKE, FAKE, FAKE, max_seq_len,
+                                      FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, top_k,
+                                      None, FAKE, None)
+
+
+def test_noalloc_reports_the_validation_status(lib):
+    """The no-allocation entry returns the same shape / argument status as
+    basiskv_decode, and refuses workspaces above its static array, all
+    before any CUDA call."""
+    assert _noalloc(lib, _dims(d=100), 8, 256) == bkv.ERR_UNSUPPORTED_SHAPE
+    assert _noalloc(lib, _dims(Hq=7), 8, 256) == bkv.ERR_UNSUPPORTED_SHAPE
+    assert _noalloc(lib, _dims(), 1, 256) == bkv.ERR_INVALID_ARG  # top_k below sink + newest
+    assert _noalloc(lib, _dims(), 8, 0) == bkv.ERR_INVALID_ARG
+    assert _noalloc(lib, _dims(), 8, 64 * 16 + 1) == bkv.ERR_INVALID_ARG  # above the table
+    big = _dims(B=256, Hq=32, Hkv=8, hidden=4096, max_pages_per_seq=25000,
+                num_phys_pages=256 * 25000 // 8)
+    assert lib.basiskv_workspace_size(ctypes.byref(big), 64, 400000) > bkv.NOALLOC_SCRATCH_BYTES
+    assert _noalloc(lib, big, 64, 400000) == bkv.ERR_SCRATCH_LIMIT

@@ -10,7 +10,7 @@ from oracle import basiskv_oracle as O
 from sparse_decode_attention_basiskv_b200 import synth
 
 from harness import (A_REL, S_REL, Y_ABS, Y_REL, ZE_REL, assert_e4m3_bracket, assert_within,
-                     cache_row, compare_selection, factors_np, gpu_layer, np64, oracle_route,
+                     cache_row, StepChecker, factors_np, gpu_layer, np64, oracle_route,
                      status_clean)
 
 pytestmark = pytest.mark.gpu
@@ -48,13 +48,13 @@ def test_route_and_select(setup):
     bkv.basiskv_route(layer.dims, pb.q, layer.seq_lens, wl.T, layer.block_table, layer.P_K,
                       layer.U_K, layer.Z, layer.E, wl.top_k, scores, sel, layer.workspace)
     status_clean()
-    stats = {}
+    chk = StepChecker(wl, None, wl.name + " route")
     for b in range(B):
         for g in range(Hkv):
             sc, ref_sel, tie = oracle_route(pb, b, g, wl.T)
             assert_within(np64(scores[b, g, :wl.pages]), sc, S_REL, what=f"scores b{b} g{g}")
-            compare_selection(sel[b, g].cpu().numpy(), ref_sel, tie, stats)
-    assert stats.get("clean_mismatch", 0) == 0, stats
+            chk.group(b, g, sel[b, g].cpu().numpy(), sc, ref_sel, tie)
+    chk.report()
 
 
 def test_attend_on_oracle_selection(setup):
@@ -91,7 +91,7 @@ def test_decode_step_with_append(setup):
     status_clean()
     assert torch.equal(layer.seq_lens, seq0 + 1)
     W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
-    stats = {}
+    chk = StepChecker(wl, W, wl.name)
     for b in range(wl.B):
         c = {k: np64(v[b]) for k, v in pb.cache.items()}
         out = O.decode_sequence(np64(pb.q[b]), c["K"], c["Z"], c["E"], wl.T, wl.page_size,
@@ -106,10 +106,8 @@ def test_decode_step_with_append(setup):
                                 Z_APPEND_TOL * np.abs(e_ref).max(), what="e")
             np.testing.assert_array_equal(np64(layer.K[slot].float()),
                                           O.to_e4m3(np64(k_new[b, g])))
-            compare_selection(sel[b, g].cpu().numpy(), out["sel"][g], out["near_tie"][g], stats)
-        if not out["near_tie"].any():
-            assert_within(np64(y[b]), out["y"], Y_REL, Y_ABS, what=f"y b{b}")
-    assert stats.get("clean_mismatch", 0) == 0, stats
+        chk.check(b, out, sel[b].cpu().numpy(), np64(y[b]), np64(pb.q[b]))
+    chk.report()
     layer.seq_lens.copy_(seq0)
 
 

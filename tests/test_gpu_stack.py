@@ -8,7 +8,7 @@ from oracle import basiskv_oracle as O
 from sparse_decode_attention_basiskv_b200 import synth
 from sparse_decode_attention_basiskv_b200.layer import DecodeLayer, DecodeStack
 
-from harness import Y_ABS, Y_REL, assert_within, factors_np, np64, status_clean
+from harness import StepChecker, factors_np, np64, status_clean
 
 pytestmark = pytest.mark.gpu
 
@@ -31,10 +31,19 @@ def test_stack_with_per_layer_widths(base, widths):
     vs = [v[:, 0].contiguous() for _, v in toks]
     ys = [y.clone() for y in stack.decode([pb.q for pb in pbs], ks, vs, max_seq_len=base.T + 1)]
     status_clean()
+    # the same step of each layer again (lengths reset), with its selection
+    # written out: equal outputs, and the selection to check
+    for L in stack.layers:
+        L.seq_lens.fill_(base.T)
+    sels = [torch.empty(wl.B, wl.Hkv, wl.top_k, dtype=torch.int32, device="cuda") for wl in wls]
+    for L, pb, k, v, s_, y in zip(stack.layers, pbs, ks, vs, sels, ys):
+        assert torch.equal(L.decode(pb.q, k, v, sel=s_, max_seq_len=base.T + 1), y)
+    status_clean()
     for l, (wl, pb) in enumerate(zip(wls, pbs)):
         f = factors_np(pb)
         W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
         assert stack.layers[l].seq_lens.tolist() == [base.T + 1] * wl.B
+        chk = StepChecker(wl, W, f"layer {l}")
         for b in range(wl.B):
             c = {k: np64(v[b]) for k, v in pb.cache.items()}
             out = O.decode_sequence(np64(pb.q[b]), c["K"], c["Z"], c["E"], wl.T, wl.page_size,
@@ -42,5 +51,5 @@ def test_stack_with_per_layer_widths(base, widths):
                                     v_new=np64(vs[l][b]), A_V=f["A_V"], fp8=bool(wl.cache_fp8),
                                     **wl.router)
             assert out["a"].shape[1] == widths[l]
-            if not out["near_tie"].any():
-                assert_within(np64(ys[l][b]), out["y"], Y_REL, Y_ABS, what=f"layer {l} y b{b}")
+            chk.check(b, out, sels[l][b].cpu().numpy(), np64(ys[l][b]), np64(pb.q[b]))
+        chk.report()

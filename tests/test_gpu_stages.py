@@ -10,7 +10,7 @@ from oracle import basiskv_oracle as O
 from sparse_decode_attention_basiskv_b200 import synth
 
 from harness import (A_REL, S_REL, Y_ABS, Y_REL, ZE_REL, assert_within, cache_row,
-                     compare_selection,
+                     StepChecker,
                      factors_np, gpu_layer, np64, oracle_route, status_clean)
 
 pytestmark = pytest.mark.gpu
@@ -63,13 +63,13 @@ def test_route_and_select(setup):
                       layer.U_K, layer.Z, layer.E, wl.top_k, scores, sel, layer.workspace)
     status_clean()
     P = wl.pages
-    stats = {}
+    chk = StepChecker(wl, None, wl.name + " route")
     for b in range(B):
         for g in range(Hkv):
             sc, ref_sel, tie = oracle_route(pb, b, g, wl.T)
             assert_within(np64(scores[b, g, :P]), sc, S_REL, what=f"scores b{b} g{g}")
-            compare_selection(sel[b, g].cpu().numpy(), ref_sel, tie, stats)
-    assert stats.get("clean_mismatch", 0) == 0, stats
+            chk.group(b, g, sel[b, g].cpu().numpy(), sc, ref_sel, tie)
+    chk.report()
 
 
 def test_attend_on_oracle_selection(setup):
@@ -119,7 +119,7 @@ def test_decode_step_with_append(setup):
     status_clean()
     assert torch.equal(layer.seq_lens, seq0 + 1)
     W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
-    stats = {}
+    chk = StepChecker(wl, W, wl.name)
     for b in range(wl.B):
         c = {k: np64(v[b]) for k, v in pb.cache.items()}
         out = O.decode_sequence(np64(pb.q[b]), c["K"], c["Z"], c["E"], wl.T, wl.page_size,
@@ -133,10 +133,8 @@ def test_decode_step_with_append(setup):
             assert_within(np64(cache_row(layer.E, wl, "E", *slot)), out["e_new"][g], ZE_REL,
                           what="e")
             assert torch.equal(layer.K[slot], k_new[b, g])
-            compare_selection(sel[b, g].cpu().numpy(), out["sel"][g], out["near_tie"][g], stats)
-        if not out["near_tie"].any():
-            assert_within(np64(y[b]), out["y"], Y_REL, Y_ABS, what=f"y b{b}")
-    assert stats.get("clean_mismatch", 0) == 0, stats
+        chk.check(b, out, sel[b].cpu().numpy(), np64(y[b]), np64(pb.q[b]))
+    chk.report()
     # undo the append for the other tests of this module
     layer.seq_lens.copy_(seq0)
 
@@ -152,13 +150,13 @@ def test_ragged_lengths_and_degenerate_pages():
     status_clean()
     f = factors_np(pb)
     W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
+    chk = StepChecker(wl, W, "ragged")
     for b, T in enumerate(lens):
         c = {k: np64(v[b]) for k, v in pb.cache.items()}
         out = O.decode_sequence(np64(pb.q[b]), c["K"], c["Z"], c["E"], T, wl.page_size,
                                 wl.top_k, f["P_K"], f["U_K"], W)
-        if not out["near_tie"].any():
-            assert np.array_equal(sel[b].cpu().numpy(), out["sel"]), b
-            assert_within(np64(y[b]), out["y"], Y_REL, Y_ABS, what=f"y b{b}")
+        chk.check(b, out, sel[b].cpu().numpy(), np64(y[b]), np64(pb.q[b]))
+    chk.report()
     assert sel[0, 0, 0].item() == 0 and (sel[0, 0, 1:] == -1).all()  # one page
 
 
@@ -179,8 +177,14 @@ def test_empty_sequence_gives_zero_output():
     c = {k: np64(v[1]) for k, v in pb.cache.items()}
     out = O.decode_sequence(np64(pb.q[1]), c["K"], c["Z"], c["E"], 600, wl.page_size,
                             wl.top_k, f["P_K"], f["U_K"], W)
-    if not out["near_tie"].any():
-        assert_within(np64(y[1]), out["y"], Y_REL, Y_ABS)
+    sel = torch.empty(wl.B, wl.Hkv, wl.top_k, dtype=torch.int32, device="cuda")
+    layer.seq_lens[0] = 0
+    y2 = layer.decode(pb.q, sel=sel, max_seq_len=600).clone()
+    status_clean()
+    assert torch.equal(y2, y)  # the same step again, now with the selection written out
+    chk = StepChecker(wl, W, "empty")
+    chk.check(1, out, sel[1].cpu().numpy(), np64(y[1]), np64(pb.q[1]))
+    chk.report()
 
 
 def test_dense_when_top_k_covers_context():

@@ -16,7 +16,7 @@ from oracle import basiskv_oracle as O
 from sparse_decode_attention_basiskv_b200 import synth
 from sparse_decode_attention_basiskv_b200.tp import LatentGather, TPDecodeLayer, head_shard
 
-from harness import Y_ABS, Y_REL, assert_within, factors_np, np64, status_clean
+from harness import StepChecker, Y_ABS, Y_REL, assert_within, factors_np, np64, status_clean
 
 pytestmark = pytest.mark.gpu
 
@@ -43,27 +43,32 @@ def test_sharded_step_matches_unsharded_oracle(case):
     ranks = [TPDecodeLayer.from_problem(pb, world, r, a_src=a_src) for r in range(world)]
     k_new, v_new = synth.make_tokens(wl, pb.factors, 1, device="cuda")
     k_new, v_new = k_new[:, 0].contiguous(), v_new[:, 0].contiguous()
+    sel = torch.empty(wl.B, wl.Hkv, wl.top_k, dtype=torch.int32, device="cuda")
     for r, L in enumerate(ranks):
         g0, g1, h0, h1 = head_shard(wl.Hq, wl.Hkv, world, r)
+        sel_r = torch.empty(wl.B, g1 - g0, wl.top_k, dtype=torch.int32, device="cuda")
         L.compute.latents(L, pb.q[:, h0:h1].contiguous(), k_new[:, g0:g1].contiguous(),
-                          v_new[:, g0:g1].contiguous(), wl.T + 1, None, a_src[r], None)
+                          v_new[:, g0:g1].contiguous(), wl.T + 1, sel_r, a_src[r], None)
+        sel[:, g0:g1] = sel_r
     y = torch.empty(wl.B, wl.hidden, dtype=torch.bfloat16, device="cuda")
     ranks[0].compute.outproj(ranks[0], a_src, y, None)
     status_clean()
     for L in ranks:
         assert L.seq_lens.tolist() == [wl.T + 1] * wl.B
     W = O.fold_outproj(f["B_V"], f["W_O"], wl.Hq)
+    chk = StepChecker(wl, W, case)
     for b in range(wl.B):
         c = {k: np64(v[b]) for k, v in pb.cache.items()}
         out = O.decode_sequence(np64(pb.q[b]), c["K"], c["Z"], c["E"], wl.T, wl.page_size,
                                 wl.top_k, f["P_K"], f["U_K"], W, k_new=np64(k_new[b]),
                                 v_new=np64(v_new[b]), A_V=f["A_V"], fp8=bool(wl.cache_fp8),
                                 **wl.router)
-        if out["near_tie"].any():
-            continue
+        gsel = sel[b].cpu().numpy()
+        a_ref, y_ref = chk.expected(out, np64(pb.q[b]), gsel, chk.selection(b, out, gsel))
         a = np64(a_src[:, b].reshape(wl.Hq, wl.r_v))
-        assert_within(a, out["a"], 1e-2, what=f"latents b{b}")  # one bf16 rounding
-        assert_within(np64(y[b]), out["y"], Y_REL, Y_ABS, what=f"y b{b}")
+        assert_within(a, a_ref, 1e-2, what=f"latents b{b}")  # one bf16 rounding
+        assert_within(np64(y[b]), y_ref, Y_REL, Y_ABS, what=f"y b{b}")
+    chk.report()
 
 
 def _free_port() -> int:

@@ -373,3 +373,48 @@ def test_synthetic_e4m3_caches_hold_e4m3_values():
         np.testing.assert_array_equal(O.to_e4m3(x), x)
     paged = pb.paged()
     assert all(v.dtype == torch.float8_e4m3fn for v in paged.values())
+
+
+def test_decode_sequence_fp8_stores_and_reads_e4m3_values():
+    """The E4M3 branch of the decode step (Table 13's FP8 E4M3 caches): with
+    A_V = I the new token's latent is v itself, so the stored z must be
+    torch's float8_e4m3fn rounding of v, the stored K torch's rounding of
+    k, and a new key that dominates the scores makes a equal that stored
+    z; the bf16 branch stores the bf16 roundings instead (the two differ on
+    these values, so swapping the branches' roundings fails)."""
+    rng = np.random.default_rng(21)
+    Hkv, G, d, r_k, S, T = 1, 2, 16, 4, 8, 31
+    r_v = d
+    A_V = np.eye(d)[None]
+    P_K = rng.standard_normal((Hkv, r_v, d)) / 4
+    U_K = np.stack([_orth(rng, d, r_k)])
+    K = rng.standard_normal((Hkv, 40, d))
+    Z = rng.standard_normal((Hkv, 40, r_v))
+    E = rng.standard_normal((Hkv, 40, r_k))
+    u = rng.standard_normal(d)
+    k_new = (8 * u / np.linalg.norm(u))[None] + rng.standard_normal((1, d)) * 1e-2
+    v_new = rng.standard_normal((Hkv, d)) * 3
+    q = np.tile(10 * u / np.linalg.norm(u), (G, 1))
+    W = O.fold_outproj(rng.standard_normal((Hkv, r_v, d)), rng.standard_normal((G * d, 3)), G)
+
+    def torch_round(x, dt):
+        return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(dt).double().numpy()
+
+    out8 = O.decode_sequence(q, K, Z, E, T, S, 2, P_K, U_K, W, k_new=k_new, v_new=v_new,
+                             A_V=A_V, fp8=True)
+    out16 = O.decode_sequence(q, K, Z, E, T, S, 2, P_K, U_K, W, k_new=k_new, v_new=v_new,
+                              A_V=A_V)
+    z8, k8 = torch_round(v_new[0], torch.float8_e4m3fn), torch_round(k_new[0], torch.float8_e4m3fn)
+    z16 = torch_round(v_new[0], torch.bfloat16)
+    np.testing.assert_array_equal(out8["Z"][0, T], z8)
+    np.testing.assert_array_equal(out8["K"][0, T], k8)
+    np.testing.assert_array_equal(out8["E"][0, T],
+                                  torch_round(out8["e_new"][0], torch.float8_e4m3fn))
+    np.testing.assert_array_equal(out16["Z"][0, T], z16)
+    np.testing.assert_array_equal(out16["K"][0, T], k_new[0])
+    assert not np.array_equal(z8, z16) and not np.array_equal(k8, k_new[0])
+    assert list(out8["sel"][0]) == [0, 3]
+    np.testing.assert_allclose(out8["a"], np.tile(z8, (G, 1)), atol=1e-6)
+    np.testing.assert_allclose(out16["a"], np.tile(z16, (G, 1)), atol=1e-6)
+    # the caches the caller passed are not modified
+    assert not np.array_equal(Z[0, T], out8["Z"][0, T])
