@@ -376,18 +376,11 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   return launch_status(launch_select(s, st, pdl));
 }
 
-int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_lens,
-               const int32_t* block_table, const basiskv_bf16* K_cache,
-               const basiskv_bf16* Z_cache, const int32_t* sel, int top_k, float* a_lat,
-               uint16_t* a_bf16, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl,
-               int len_offset = 0, int* cnt = nullptr, const int32_t* sel_phys = nullptr) {
-  unsigned int* status = device_status_ptr();
-  if (!status) return BASISKV_ERR_CUDA;
-  const int wz = z_box_cols(d->r_v);
-  CUtensorMap tmK{}, tmZ{};  // bf16 caches only: the E4M3 kernel uses plain loads
-  if (!d->cache_fp8 &&
-      (!cache_map(&tmK, K_cache, d, d->d, 64) || !cache_map(&tmZ, Z_cache, d, d->r_v, wz)))
-    return BASISKV_ERR_CUDA;
+AttendArgs make_attend_args(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_lens,
+                            const int32_t* block_table, const basiskv_bf16* K_cache,
+                            const basiskv_bf16* Z_cache, const int32_t* sel,
+                            const int32_t* sel_phys, int top_k, uint8_t* ws, const WsLayout& L,
+                            int len_offset, unsigned int* status) {
   AttendArgs a{};
   a.q = q;
   a.K = K_cache;
@@ -414,6 +407,48 @@ int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_
   a.len_offset = len_offset;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d->d));
   a.status = status;
+  return a;
+}
+
+// The cluster size of the fused selection + attention launch for this step
+// (0: the step takes the separate selection and attention launches).
+int fused_cluster(const basiskv_dims* d, int top_k, int max_seq_len) {
+  return select_attend_cluster_size(d->Hq / d->Hkv, d->d, d->r_v, d->page_size, d->cache_fp8,
+                                    d->B, d->Hkv, max_seq_len, top_k);
+}
+
+// Selection and attention of a fused step in one launch (after the scores):
+// the bf16 latents to a_bf16, the selection to sel when it is set.
+int run_select_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_lens,
+                      int max_seq_len, const int32_t* block_table, const basiskv_bf16* K_cache,
+                      const basiskv_bf16* Z_cache, int top_k, int32_t* sel, uint16_t* a_bf16,
+                      uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl, int len_offset) {
+  unsigned int* status = device_status_ptr();
+  if (!status) return BASISKV_ERR_CUDA;
+  SelectArgs s{reinterpret_cast<float*>(ws + L.scores), seq_lens, sel, d->B, d->Hkv,
+               d->page_size, d->max_pages_per_seq, top_k, max_seq_len, len_offset, block_table,
+               nullptr, sink_pages(d), recent_pages(d)};
+  AttendArgs a = make_attend_args(d, q, seq_lens, block_table, K_cache, Z_cache, nullptr, nullptr,
+                                  top_k, ws, L, len_offset, status);
+  a.early_inputs = 1;
+  a.a_bf16 = a_bf16;
+  return launch_status(launch_select_attend(s, a, st, pdl));
+}
+
+int run_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_lens,
+               const int32_t* block_table, const basiskv_bf16* K_cache,
+               const basiskv_bf16* Z_cache, const int32_t* sel, int top_k, float* a_lat,
+               uint16_t* a_bf16, uint8_t* ws, const WsLayout& L, cudaStream_t st, bool pdl,
+               int len_offset = 0, int* cnt = nullptr, const int32_t* sel_phys = nullptr) {
+  unsigned int* status = device_status_ptr();
+  if (!status) return BASISKV_ERR_CUDA;
+  const int wz = z_box_cols(d->r_v);
+  CUtensorMap tmK{}, tmZ{};  // bf16 caches only: the E4M3 kernel uses plain loads
+  if (!d->cache_fp8 &&
+      (!cache_map(&tmK, K_cache, d, d->d, 64) || !cache_map(&tmZ, Z_cache, d, d->r_v, wz)))
+    return BASISKV_ERR_CUDA;
+  AttendArgs a = make_attend_args(d, q, seq_lens, block_table, K_cache, Z_cache, sel, sel_phys,
+                                  top_k, ws, L, len_offset, status);
   if (attend_mma_supported(a.G, a.d, a.r_v, a.S)) {
     a.early_inputs = cnt != nullptr;  // inside the fused step: follows the selection launch
     if (!cnt) {  // a standalone call: the arrival counters start from zero here
@@ -675,30 +710,44 @@ int basiskv_decode(const basiskv_dims* dims, const basiskv_bf16* q, const basisk
   // stages in between read seq_lens[b] + 1.
   const int off = append ? 1 : 0;
   // Launch 1: the query fold; it also zeroes the arrival counters of the
-  // fused merge and reduction below.  The token append runs in the selection
-  // launch (launch 3): the scoring reads the newest page before the new token
-  // is in it, which only changes that page's score, and the newest page is
-  // selected whatever its score.
+  // fused merges and reduction below.  When the selection and the attention
+  // share one launch (groups that fit one wave of CTA clusters), launch 1
+  // also appends the token, and the scoring (launch 2) may start before the
+  // token lands: it reads the newest page either way, which only changes
+  // that page's score, and the newest page is selected whatever its score
+  // (its score is not an output of this call).  Otherwise the append runs in
+  // the selection launch, after the scoring.
   int* cnt = reinterpret_cast<int*>(ws + L.counters);
   AppendArgs app = make_append_args(dims, append ? k_new : nullptr, v_new, 1, seq_lens,
                                     block_table, A_V, P_K, U_K, K_cache, Z_cache, E_cache);
   if (!app.status) return BASISKV_ERR_CUDA;
+  const bool fused = fused_cluster(dims, top_k, max_seq_len) > 0;
   {
-    AppendArgs none = app;
-    none.k_new = nullptr;
     FoldQArgs f{q, P_K, U_K, reinterpret_cast<float*>(ws + L.qt), dims->B, dims->Hq, dims->Hkv,
                 dims->d, dims->r_v, dims->r_k};
+    AppendArgs first = app;
+    if (!fused) first.k_new = nullptr;  // the append then runs in the selection launch
     rc = launch_status(
-        launch_decode_prologue(f, none, cnt, L.n_att_cnt + L.n_op_cnt, st, pdl));
+        launch_decode_prologue(f, first, cnt, L.n_att_cnt + L.n_op_cnt, st, pdl));
     if (rc) return rc;
   }
-  rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache, top_k,
-                 reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl, off,
-                 /*do_fold=*/false, append ? &app : nullptr);
-  if (rc) return rc;
   uint16_t* a16 = reinterpret_cast<uint16_t*>(ws + L.a_bf16);
-  rc = run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel_buf, top_k, nullptr, a16,
-                  ws, L, st, pdl, off, cnt, reinterpret_cast<const int32_t*>(ws + L.selp));
+  if (fused) {
+    rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache, top_k,
+                   reinterpret_cast<float*>(ws + L.scores), nullptr, ws, L, st, pdl, off,
+                   /*do_fold=*/false);
+    if (rc) return rc;
+    rc = run_select_attend(dims, q, seq_lens, max_seq_len, block_table, K_cache, Z_cache, top_k,
+                           sel, a16, ws, L, st, pdl, off);
+  } else {
+    rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache,
+                   top_k, reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl, off,
+                   /*do_fold=*/false, append ? &app : nullptr);
+    if (rc) return rc;
+    rc = run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel_buf, top_k, nullptr,
+                    a16, ws, L, st, pdl, off, cnt,
+                    reinterpret_cast<const int32_t*>(ws + L.selp));
+  }
   if (rc) return rc;
   return run_outproj(dims, a16, W_fold, y, ws, L, st, pdl, append ? seq_lens : nullptr,
                      cnt + L.n_att_cnt);
@@ -743,20 +792,31 @@ int basiskv_decode_latents(const basiskv_dims* dims, const basiskv_bf16* q,
   AppendArgs app = make_append_args(dims, append ? k_new : nullptr, v_new, 1, seq_lens,
                                     block_table, A_V, P_K, U_K, K_cache, Z_cache, E_cache);
   if (!app.status) return BASISKV_ERR_CUDA;
+  const bool fused = fused_cluster(dims, top_k, max_seq_len) > 0;  // as in basiskv_decode
   {
-    AppendArgs none = app;
-    none.k_new = nullptr;
     FoldQArgs f{q, P_K, U_K, reinterpret_cast<float*>(ws + L.qt), dims->B, dims->Hq, dims->Hkv,
                 dims->d, dims->r_v, dims->r_k};
-    rc = launch_status(launch_decode_prologue(f, none, cnt, L.n_att_cnt, st, pdl));
+    AppendArgs first = app;
+    if (!fused) first.k_new = nullptr;
+    rc = launch_status(launch_decode_prologue(f, first, cnt, L.n_att_cnt, st, pdl));
     if (rc) return rc;
   }
-  rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache, top_k,
-                 reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl, off,
-                 /*do_fold=*/false, append ? &app : nullptr);
-  if (rc) return rc;
-  rc = run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel_buf, top_k, nullptr, a_out,
-                  ws, L, st, pdl, off, cnt, reinterpret_cast<const int32_t*>(ws + L.selp));
+  if (fused) {
+    rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache, top_k,
+                   reinterpret_cast<float*>(ws + L.scores), nullptr, ws, L, st, pdl, off,
+                   /*do_fold=*/false);
+    if (rc) return rc;
+    rc = run_select_attend(dims, q, seq_lens, max_seq_len, block_table, K_cache, Z_cache, top_k,
+                           sel, a_out, ws, L, st, pdl, off);
+  } else {
+    rc = run_route(dims, q, seq_lens, max_seq_len, block_table, P_K, U_K, Z_cache, E_cache,
+                   top_k, reinterpret_cast<float*>(ws + L.scores), sel_buf, ws, L, st, pdl, off,
+                   /*do_fold=*/false, append ? &app : nullptr);
+    if (rc) return rc;
+    rc = run_attend(dims, q, seq_lens, block_table, K_cache, Z_cache, sel_buf, top_k, nullptr,
+                    a_out, ws, L, st, pdl, off, cnt,
+                    reinterpret_cast<const int32_t*>(ws + L.selp));
+  }
   if (rc || !append) return rc;
   return launch_status(launch_bump_lengths(app, st, pdl));  // after every reader
 }

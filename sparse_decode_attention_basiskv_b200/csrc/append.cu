@@ -24,36 +24,34 @@ __global__ void __launch_bounds__(kAppendThreads) append_small_kernel(AppendArgs
   append_block(a, blockIdx.x, blockIdx.y, blockIdx.z, fac, vs, ks, zs, rs, threadIdx.x, 0);
 }
 
-// The first launch of a fused decode step, one block per (sequence, KV
-// head): 128-thread group i < n_fold folds the group's queries for outputs
-// 32i .. 32i + 31, and (when the step appends) the last group appends the
-// step's token; each group synchronises on its own named barrier, so the
-// fold and the append run side by side in one wave.  Block 0 also zeroes
-// the step's arrival counters.
-constexpr int kPrologueMaxThreads = 7 * 128;  // up to 6 fold groups + the append group
-
-__global__ void __launch_bounds__(kPrologueMaxThreads)
+// The first launch of a fused decode step: block (bg, i < n_fold) folds the
+// queries of (sequence, KV head) bg for outputs 32i .. 32i + 31 (one
+// 128-thread group each, so a small batch still spreads the fold over many
+// SMs); when the step appends, block (bg, n_fold) appends the step's token of
+// bg without staging the factors; block (0, 0) also zeroes the step's
+// arrival counters.  Every block needs only a few KB of shared memory, so
+// the scoring grid, let in once the wait below has returned, takes the rest
+// of the SMs and starts on its page loads while this grid finishes.  The
+// scoring may read the newest page before the token lands: that only
+// changes that page's score, and the newest page is selected whatever its
+// score.
+__global__ void __launch_bounds__(kFoldThreads)
     decode_prologue_kernel(FoldQArgs f, AppendArgs a, int n_fold, int* counters,
                            int n_counters) {
-  extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ float vs[kAppendThreads], ks[kAppendThreads], zs[kAppendThreads],
-      rs[kAppendThreads];
-  const int bg = blockIdx.x, grp = threadIdx.x / kFoldThreads, gtid = threadIdx.x % kFoldThreads;
-  // One wave of blocks: the scoring grid may take the rest of the SMs and
-  // start on its page loads while the fold finishes.
+  extern __shared__ __align__(16) float fsm[];
+  // The next launches read the step's inputs before their own waits: they
+  // are let in only once this wait has seen the caller's work complete.
+  pdl_wait();
   pdl_launch_dependents();
-  if (bg == 0 && counters) {
-    pdl_wait();
+  if (blockIdx.x == 0 && blockIdx.y == 0 && counters)
     for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
-  }
-  const size_t fold_bytes = fold_block_smem(f.Hq / f.Hkv, f.d);
-  if (grp < n_fold) {
-    fold_query_block(f, bg, grp, reinterpret_cast<float*>(dyn + grp * fold_bytes), gtid,
-                     1 + grp);
-  } else {
-    append_block(a, bg % a.Hkv, 0, bg / a.Hkv,
-                 reinterpret_cast<uint16_t*>(dyn + n_fold * fold_bytes), vs, ks, zs, rs, gtid,
-                 1 + grp);
+  if ((int)blockIdx.y < n_fold) {
+    fold_query_block(f, blockIdx.x, blockIdx.y, fsm, threadIdx.x, 0);
+  } else if (a.k_new) {
+    float* vs = fsm;
+    append_block_direct(a, blockIdx.x % a.Hkv, blockIdx.x / a.Hkv, vs, vs + kAppendThreads,
+                        vs + 2 * kAppendThreads, vs + 3 * kAppendThreads,
+                        vs + 4 * kAppendThreads, threadIdx.x, 0);
   }
 }
 
@@ -96,17 +94,12 @@ cudaError_t launch_decode_prologue(const FoldQArgs& f, const AppendArgs& a, int*
                                    int n_counters, cudaStream_t st, bool pdl) {
   const int n_fold = (f.r_v + f.r_k + 31) / 32;
   const bool app = a.k_new != nullptr;
-  const int threads = (n_fold + (app ? 1 : 0)) * kFoldThreads;
-  if (threads > kPrologueMaxThreads) return cudaErrorInvalidConfiguration;
-  size_t smem = (size_t)n_fold * fold_block_smem(f.Hq / f.Hkv, f.d);
-  if (app) smem += append_block_smem(a.d, a.r_v, a.r_k);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(decode_prologue_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  return launch_k(decode_prologue_kernel, dim3(f.B * f.Hkv), dim3(threads), smem, st, pdl, f, a,
-                  n_fold, counters, n_counters);
+  size_t smem = fold_block_smem(f.Hq / f.Hkv, f.d);
+  const size_t app_smem =
+      (size_t)(4 * kAppendThreads + append_direct_red_floats(a.d, a.r_v, a.r_k)) * sizeof(float);
+  if (app && app_smem > smem) smem = app_smem;
+  return launch_k(decode_prologue_kernel, dim3(f.B * f.Hkv, n_fold + (app ? 1 : 0)),
+                  dim3(kFoldThreads), smem, st, pdl, f, a, n_fold, counters, n_counters);
 }
 
 }  // namespace basiskv

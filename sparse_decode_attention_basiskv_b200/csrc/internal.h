@@ -75,9 +75,10 @@ struct FoldQArgs {
   int B, Hq, Hkv, d, r_v, r_k;
 };
 cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl);
-// First launch of a fused decode step: the query fold and (when a.k_new is
-// set) the one-token append run side by side; n_counters ints at `counters`
-// are zeroed.
+// First launch of a fused decode step: the query fold, one block per 32
+// outputs of each (sequence, KV head), and (when a.k_new is set) the
+// one-token append, one more block per (sequence, KV head); n_counters ints
+// at `counters` are zeroed.
 cudaError_t launch_decode_prologue(const FoldQArgs& f, const AppendArgs& a, int* counters,
                                    int n_counters, cudaStream_t st, bool pdl);
 
@@ -159,6 +160,16 @@ bool attend_mma_fp8_supported(int G, int d, int r_v, int S);
 cudaError_t launch_attend_mma_fp8(const AttendArgs& a, cudaStream_t st, bool pdl);
 int attend_mma_slots(int B, int Hkv);
 cudaError_t launch_attend_mma(const AttendArgs& a, cudaStream_t st, bool pdl);
+// Selection and attention of a fused decode step in one launch, one cluster
+// of CTAs per (sequence, KV head) (select_attend.cuh).  The cluster size for
+// a step, or 0 when the step does not fit one wave (then the selection and
+// the attention launch separately).  s.sel, when set, receives the selection.
+int select_attend_cluster_size(int G, int d, int r_v, int S, int fp8, int B, int Hkv,
+                               int max_seq_len, int top_k);
+cudaError_t launch_select_attend(const SelectArgs& s, const AttendArgs& a, cudaStream_t st,
+                                 bool pdl);
+cudaError_t launch_select_attend_fp8(const SelectArgs& s, const AttendArgs& a, cudaStream_t st,
+                                     bool pdl);
 cudaError_t launch_attend(const AttendArgs& a, const CUtensorMap& tmK, const CUtensorMap& tmZ,
                           int wz, cudaStream_t st, bool pdl);
 

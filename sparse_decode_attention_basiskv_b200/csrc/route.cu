@@ -21,6 +21,7 @@
 #include "internal.h"
 #include "launch.cuh"
 #include "route_mma.cuh"
+#include "select_block.cuh"
 #include "step_blocks.cuh"
 
 namespace basiskv {
@@ -442,220 +443,13 @@ __global__ void __launch_bounds__(kRsThreads, kRsCtasPerSm)
   }
 }
 
-// -------------------------------------------------------- page selection
-// Per (sequence, KV head): the first n_sink and the last n_recent pages
-// always (by default the sink page 0 and the newest page P-1); the other
-// slots go to the best remaining pages by (score desc, index asc),
-// found exactly with an MSB-first radix select over order-preserving 32-bit
-// keys; ties at the threshold are taken in index order.  Output ascending.
-constexpr int kSelThreads = 512;
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-  if (f == 0.f) f = 0.f;  // -0 ranks as +0
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-struct SelShared {
-  int hist[2][256];  // radix histograms, alternating between passes
-  int sh[32];        // scan scratch
-  uint32_t digit;
-  int rem;
-  int done;  // the chosen bucket is taken whole: later digits are not needed
-};
-
-// Exclusive prefix sum over a block of NT threads; *total receives the sum.
-template <int NT>
-__device__ int block_excl_scan(int v, int* sh, int* total) {
-  constexpr int W = NT / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) sh[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < W ? sh[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    sh[lane] = w;
-  }
-  __syncthreads();
-  const int res = (warp ? sh[warp - 1] : 0) + x - v;
-  *total = sh[W - 1];
-  __syncthreads();
-  return res;
-}
-
-// Selection of one (sequence, KV head) by a block of NT threads.  keys and
-// tbl: shared arrays of at least ceil(max_seq_len / S) entries.
-template <int NT>
-__device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32_t* keys, int* tbl,
-                                          SelShared& ss) {
-  const int b = bg / a.Hkv, tid = threadIdx.x;
-  const int P_max = (a.max_seq_len + a.S - 1) / a.S;
-  int32_t* out = a.sel + (size_t)bg * a.top_k;
-  int32_t* outp = a.sel_phys ? a.sel_phys + (size_t)bg * a.top_k : nullptr;
-  const int32_t* bt = a.block_table + (size_t)b * a.max_pages;
-  const int ns = a.n_sink, nr = a.n_recent;  // forced leading / trailing pages
-  const float* sc = a.scores + (size_t)bg * a.max_pages + ns;  // candidate i = page ns + i
-  // The length, the first batch of scores and the block-table row are
-  // requested together (up to the longest possible context; what lies past
-  // this sequence's pages is dropped): one memory round trip, not two.
-  int T = a.seq_lens[b] + a.len_offset;
-  float v[8];
-  int t[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int i = u * NT + tid;
-    v[u] = i < P_max - ns ? __ldcg(sc + i) : 0.f;
-    t[u] = (outp && i < P_max) ? bt[i] : 0;
-  }
-  T = T < 0 ? 0 : (T > a.max_seq_len ? a.max_seq_len : T);
-  const int P = (T + a.S - 1) / a.S;
-  if (a.top_k >= P) {
-    for (int i = tid; i < a.top_k; i += NT) {
-      out[i] = i < P ? i : -1;
-      if (outp) outp[i] = i < P ? bt[i] : -1;
-    }
-    return;
-  }
-  const int n = P - ns - nr, need = a.top_k - ns - nr;  // n >= 1: P > top_k >= ns + nr
-  for (int base = 0; base < P; base += 8 * NT) {  // batches of eight loads a thread
-    if (base > 0) {
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = base + u * NT + tid;
-        v[u] = i < n ? __ldcg(sc + i) : 0.f;
-        t[u] = (outp && i < P) ? bt[i] : 0;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = base + u * NT + tid;
-      if (i < n) keys[i] = order_key(v[u]);
-      if (outp && i < P) tbl[i] = t[u];
-    }
-  }
-  for (int i = tid; i < 512; i += NT) (&ss.hist[0][0])[i] = 0;
-  __syncthreads();
-
-  // MSB-first radix select of the need-th largest key: two barriers a pass
-  // (the scanning warp clears the other histogram for the next pass).
-  uint32_t prefix = 0, pmask = 0;
-  int rem = need;
-  if (need > 0) {
-    int cur = 0;
-    for (int shift = 24; shift >= 0; shift -= 8, cur ^= 1) {
-      int* hist = ss.hist[cur];
-      // The leading digits of one context's scores are mostly the same (sign
-      // and exponent): lanes sharing lane 0's digit add through one atomic,
-      // the others individually, so same-address atomics do not serialise.
-      for (int base = 0; base < n; base += NT) {
-        const int i = base + tid;
-        int bin = -1;
-        if (i < n) {
-          const uint32_t k = keys[i];
-          if ((k & pmask) == prefix) bin = (int)((k >> shift) & 255);
-        }
-        const int b0 = __shfl_sync(0xffffffffu, bin, 0);
-        const unsigned same = __ballot_sync(0xffffffffu, bin == b0);
-        if (bin >= 0) {
-          if (bin != b0)
-            atomicAdd(&hist[bin], 1);
-          else if ((tid & 31) == __ffs(same) - 1)
-            atomicAdd(&hist[bin], __popc(same));
-        }
-      }
-      __syncthreads();
-      if (tid < 32) {  // lane l covers digits 255-8l .. 248-8l, high to low
-        int local = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) local += hist[255 - 8 * tid - j];
-        int cum = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, cum, o);
-          if (tid >= o) cum += y;
-        }
-        const unsigned hit = __ballot_sync(0xffffffffu, cum >= rem);
-        const int L = __ffs(hit) - 1;
-        if (tid == L) {
-          int start = cum - local;
-          for (int j = 0; j < 8; ++j) {
-            const int dg = 255 - 8 * L - j;
-            if (start + hist[dg] >= rem) {
-              ss.digit = (uint32_t)dg;
-              ss.rem = rem - start;
-              ss.done = hist[dg] == rem - start;
-              break;
-            }
-            start += hist[dg];
-          }
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) ss.hist[cur ^ 1][8 * tid + j] = 0;
-      }
-      __syncthreads();
-      prefix |= ss.digit << shift;
-      pmask |= 0xffu << shift;
-      rem = ss.rem;
-      // Every key of the bucket is taken: with the remaining digits zero the
-      // threshold is at or below all of them, so the keys above it plus all
-      // keys equal to it are exactly the bucket and everything above.
-      if (ss.done) {
-        rem = n;
-        break;
-      }
-    }
-  }
-  const uint32_t thr = prefix;
-  // Contiguous candidate chunk per thread, so prefix sums follow index order.
-  // One scan of packed counts (keys above the threshold << 16 | keys equal to
-  // it): the first `rem` equal keys in index order are taken.
-  const int E = (n + NT - 1) / NT;
-  const int i0 = min(tid * E, n), i1 = min(i0 + E, n);
-  int n_gt = 0, n_eq = 0;
-  if (need > 0)
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t k = keys[i];
-      n_gt += k > thr;
-      n_eq += k == thr;
-    }
-  int total;
-  const int before = block_excl_scan<NT>((n_gt << 16) | n_eq, ss.sh, &total);
-  if (need > 0) {
-    int r = before & 0xffff;
-    int pos = ns + (before >> 16) + min(r, rem);
-    for (int i = i0; i < i1; ++i) {
-      const uint32_t k = keys[i];
-      if ((k > thr) || (k == thr && r < rem)) {
-        if (outp) outp[pos] = tbl[i + ns];
-        out[pos++] = i + ns;
-      }
-      r += k == thr;
-    }
-  }
-  for (int i = tid; i < ns + nr; i += NT) {  // the forced pages, first and last
-    const int slot = i < ns ? i : a.top_k - nr + (i - ns);
-    const int page = i < ns ? i : P - nr + (i - ns);
-    out[slot] = page;
-    if (outp) outp[slot] = tbl[page];
-  }
-}
-
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   extern __shared__ uint32_t keys[];
   __shared__ SelShared ss;
   pdl_wait();
   int* tbl = reinterpret_cast<int*>(keys + (a.max_seq_len + a.S - 1) / a.S);
-  select_group<kSelThreads>(a, blockIdx.x, keys, tbl, ss);
+  select_group<kSelThreads>(a, blockIdx.x, keys, tbl, ss, a.sel + (size_t)blockIdx.x * a.top_k,
+                            a.sel_phys ? a.sel_phys + (size_t)blockIdx.x * a.top_k : nullptr);
 }
 
 RouteGeom route_geometry(int G, int r_v, int r_k, int S, int wz, int we) {
@@ -726,6 +520,24 @@ cudaError_t launch_route_rs(const RouteArgs& a, const CUtensorMap& tmZ, const CU
 
 // Narrow routers with an instance: (G, S) in {(4, 16), (8, 32)}, r_k 32,
 // r_v in {64, 96}, widths 16 or 32 each.
+// The full-width routers with a plain-load scoring instance (G, r_v, r_k, S).
+#define BKV_RM_FULL(X) \
+  X(4, 32, 32, 16)     \
+  X(4, 32, 32, 32)     \
+  X(8, 32, 32, 16)     \
+  X(8, 32, 32, 32)     \
+  X(4, 64, 32, 16)     \
+  X(4, 96, 32, 16)     \
+  X(4, 128, 32, 16)    \
+  X(4, 64, 32, 32)     \
+  X(4, 96, 32, 32)     \
+  X(8, 64, 32, 16)     \
+  X(8, 96, 32, 16)     \
+  X(8, 128, 32, 16)    \
+  X(8, 64, 32, 32)     \
+  X(8, 96, 32, 32)     \
+  X(8, 128, 32, 32)
+
 #define BKV_RM_NARROW(X)                                                            \
   X(4, 64, 32, 16, 16, 16) X(4, 64, 32, 16, 32, 16) X(4, 64, 32, 32, 16, 16)        \
   X(4, 64, 32, 32, 32, 16) X(4, 96, 32, 16, 16, 16) X(4, 96, 32, 16, 32, 16)        \
@@ -768,21 +580,7 @@ cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
 #define BKV_RM(GG, V, K, SS)                                     \
   if (a.G == GG && a.r_v == V && a.r_k == K && a.S == SS) \
     return launch_route_mma<GG, V, K, V, K, SS>(a, st, pdl);
-    BKV_RM(4, 32, 32, 16)
-    BKV_RM(4, 32, 32, 32)
-    BKV_RM(8, 32, 32, 16)
-    BKV_RM(8, 32, 32, 32)
-    BKV_RM(4, 64, 32, 16)
-    BKV_RM(4, 96, 32, 16)
-    BKV_RM(4, 128, 32, 16)
-    BKV_RM(4, 64, 32, 32)
-    BKV_RM(4, 96, 32, 32)
-    BKV_RM(8, 64, 32, 16)
-    BKV_RM(8, 96, 32, 16)
-    BKV_RM(8, 128, 32, 16)
-    BKV_RM(8, 64, 32, 32)
-    BKV_RM(8, 96, 32, 32)
-    BKV_RM(8, 128, 32, 32)
+    BKV_RM_FULL(BKV_RM)
 #undef BKV_RM
   }
   if (wz == rs_z_box_cols(a.r_v) && we == (a.r_k % 32 == 0 ? 32 : 16)) {
@@ -825,7 +623,9 @@ __global__ void __launch_bounds__(kSelThreads)
     pdl_wait();
     uint32_t* keys = reinterpret_cast<uint32_t*>(sa_dyn);
     select_group<kSelThreads>(s, blockIdx.x, keys,
-                              reinterpret_cast<int*>(keys + (s.max_seq_len + s.S - 1) / s.S), ss);
+                              reinterpret_cast<int*>(keys + (s.max_seq_len + s.S - 1) / s.S), ss,
+                              s.sel + (size_t)blockIdx.x * s.top_k,
+                              s.sel_phys ? s.sel_phys + (size_t)blockIdx.x * s.top_k : nullptr);
   } else if (threadIdx.x < kAppendThreads) {
     const int r = blockIdx.x - nsel;  // (sequence, KV head)
     append_block(a, r % a.Hkv, 0, r / a.Hkv, reinterpret_cast<uint16_t*>(sa_dyn), vs, ks, zs, rs,

@@ -129,6 +129,112 @@ __device__ __forceinline__ void append_block(const AppendArgs& a, int g, int j, 
     a.E_cache[tile * a.S * r_k + split_off(row, tid, a.S, r_k, a.esplit)] = f_to_bf16(ev);
 }
 
+// The same append without staging the factors in shared memory, for a block
+// that runs beside the query fold and the early page loads of the scoring
+// grid (a few KB of shared memory, like the fold's blocks, so the scoring
+// CTAs still fit beside it).  Each of the three products is split into
+// tasks of 8 outputs x 8 rows of the factor: a task's 8 16-byte row loads
+// are independent, so a product costs about one memory round trip; the
+// per-row-block partial sums meet in shared memory (red: at least
+// max(d/8 * r_v, r_v/8 * d, d/8 * r_k) floats).  Run by kAppendThreads
+// threads on named barrier bar.
+__device__ __forceinline__ void append_block_direct(const AppendArgs& a, int g, int b,
+                                                    float* vs, float* ks, float* zs, float* rs,
+                                                    float* red, int tid, int bar) {
+  const int d = a.d, r_v = a.r_v, r_k = a.r_k;
+  pdl_wait();
+  const size_t tok = ((size_t)b * a.n_new * a.Hkv + g) * d;  // token 0 of sequence b
+  uint16_t kb = 0;
+  if (tid < d) {
+    kb = a.k_new[tok + tid];
+    ks[tid] = bf16_to_f(kb);
+    vs[tid] = bf16_to_f(a.v_new[tok + tid]);
+  }
+  const int len = a.seq_lens[b];
+  const int cap = a.max_pages * a.S;
+  const bool fits = len >= 0 && len + 1 <= cap;
+  const int pp = fits ? a.block_table[(size_t)b * a.max_pages + len / a.S] : -1;
+  named_bar_sync(bar, kAppendThreads);
+  // y[o] = sum_i x[i] F[i][o] for a factor F [rows][outs] (row-major, bf16):
+  // task (row block rb, output group og) adds rows 8rb .. 8rb+7 for outputs
+  // 8og .. 8og+7 into red[rb][8og ..]; then y[o] = sum over row blocks.
+  auto product = [&](const uint16_t* F, const float* x, int rows, int outs, float* y) {
+    const int ngr = outs / 8, nrb = rows / 8;
+    for (int t = tid; t < ngr * nrb; t += kAppendThreads) {
+      const int og = t % ngr, rb = t / ngr;
+      uint4 w[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        w[r] = __ldg(reinterpret_cast<const uint4*>(F + (size_t)(8 * rb + r) * outs + 8 * og));
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const float xv = x[8 * rb + r];
+        const uint32_t u[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[2 * e] = fmaf(xv, bf16lo(u[e]), acc[2 * e]);
+          acc[2 * e + 1] = fmaf(xv, bf16hi(u[e]), acc[2 * e + 1]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[rb * outs + 8 * og + e] = acc[e];
+    }
+    named_bar_sync(bar, kAppendThreads);
+    for (int o = tid; o < outs; o += kAppendThreads) {
+      float v = 0.f;
+      for (int rb = 0; rb < nrb; ++rb) v += red[rb * outs + o];
+      y[o] = v;
+    }
+    named_bar_sync(bar, kAppendThreads);
+  };
+  // z = v A_V (A_V [d][r_v]); the residual k - z P_K (P_K [r_v][d]), with
+  // the unrounded z; e = residual U_K (U_K [d][r_k])
+  product(a.A_V + (size_t)g * d * r_v, vs, d, r_v, zs);
+  product(a.P_K + (size_t)g * r_v * d, zs, r_v, d, rs);
+  if (tid < d) rs[tid] = ks[tid] - rs[tid];
+  named_bar_sync(bar, kAppendThreads);
+  product(a.U_K + (size_t)g * d * r_k, rs, d, r_k, red + d / 8 * r_k);
+  const float* es = red + d / 8 * r_k;
+  if (!fits) {
+    if (tid == 0 && g == 0) raise_status(a.status, BASISKV_DEV_OVERFLOW);
+    return;
+  }
+  if (pp < 0 || pp >= a.num_phys) {
+    if (tid == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
+    return;
+  }
+  const size_t tile = (size_t)pp * a.Hkv + g;
+  const int row = len % a.S;
+  if (a.fp8) {  // E4M3 caches: one byte per value, rounded to nearest even, saturated
+    if (tid < d)
+      reinterpret_cast<uint8_t*>(a.K_cache)[(tile * a.S + row) * d + tid] =
+          (uint8_t)f_to_e4m3x2(bf16_to_f(kb), 0.f);
+    if (tid < r_v)
+      reinterpret_cast<uint8_t*>(a.Z_cache)[tile * a.S * r_v +
+                                            split_off(row, tid, a.S, r_v, a.zsplit)] =
+          (uint8_t)f_to_e4m3x2(zs[tid], 0.f);
+    if (tid < r_k)
+      reinterpret_cast<uint8_t*>(a.E_cache)[tile * a.S * r_k +
+                                            split_off(row, tid, a.S, r_k, a.esplit)] =
+          (uint8_t)f_to_e4m3x2(es[tid], 0.f);
+    return;
+  }
+  if (tid < d) a.K_cache[(tile * a.S + row) * d + tid] = kb;
+  if (tid < r_v)
+    a.Z_cache[tile * a.S * r_v + split_off(row, tid, a.S, r_v, a.zsplit)] = f_to_bf16(zs[tid]);
+  if (tid < r_k)
+    a.E_cache[tile * a.S * r_k + split_off(row, tid, a.S, r_k, a.esplit)] = f_to_bf16(es[tid]);
+}
+
+// Shared memory of append_block_direct's partial sums (floats).
+__host__ __device__ inline int append_direct_red_floats(int d, int r_v, int r_k) {
+  int n = d / 8 * r_v;
+  if (r_v / 8 * d > n) n = r_v / 8 * d;
+  if (d / 8 * r_k > n) n = d / 8 * r_k;
+  return n + d / 8 * r_k;  // + the residual code e, kept past the partials
+}
+
 // Folds the queries of (sequence, KV head) bg for outputs 32*yblk .. +31:
 //   qt[b][h][j]       = sum_i P_K[g][j][i] q[b][h][i]          j < r_v
 //   qt[b][h][r_v + c] = sum_i q[b][h][i] U_K[g][i][c]           c < r_k

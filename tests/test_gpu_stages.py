@@ -8,6 +8,7 @@ import torch
 import sparse_decode_attention_basiskv_b200 as bkv
 from oracle import basiskv_oracle as O
 from sparse_decode_attention_basiskv_b200 import synth
+from sparse_decode_attention_basiskv_b200.layer import DecodeLayer
 
 from harness import (A_REL, S_REL, Y_ABS, Y_REL, ZE_REL, assert_within, cache_row,
                      StepChecker,
@@ -297,3 +298,36 @@ def test_device_status_reports_bad_inputs():
     layer.decode(pb.q, k_new[:, 0].contiguous(), v_new[:, 0].contiguous(), max_seq_len=cap)
     assert bkv.read_device_status() & bkv.DEV_OVERFLOW
     assert layer.seq_lens.item() == cap
+
+
+@pytest.mark.parametrize("levels", [1, 3, 64])
+def test_selection_with_tied_scores(levels):
+    """Page scores with many exact ties: z is zero except column 0 of every
+    token, which holds one of `levels` values per page, and e is zero, so a
+    page's score is one product per head and pages with the same value tie
+    exactly (levels = 1: every score equal).  The threshold's bin then holds
+    hundreds of pages (1, 3 levels: the radix select decides) or a few (64
+    levels).  Ties rank by the lower page index on both sides, so the
+    selection must equal the oracle's bit for bit, through the selection
+    launch and through the fused decode step."""
+    wl = synth.with_sizes(synth.LLAMA8B_T32K_B16, B=2, T=16384, top_k=64)
+    pb = synth.make_problem(wl, device="cuda")
+    S, P = wl.page_size, wl.pages
+    lvl = torch.arange(P, device="cuda").remainder(levels).float() + 1.0
+    z = torch.zeros_like(pb.cache["Z"])
+    z[:, :, :P * S, 0] = lvl.repeat_interleave(S).bfloat16()
+    pb.cache["Z"] = z
+    pb.cache["E"] = torch.zeros_like(pb.cache["E"])
+    layer = DecodeLayer.from_problem(pb)
+    scores = torch.empty(wl.B, wl.Hkv, layer.dims.max_pages_per_seq, device="cuda")
+    sel_r = torch.empty(wl.B, wl.Hkv, wl.top_k, dtype=torch.int32, device="cuda")
+    bkv.basiskv_route(layer.dims, pb.q, layer.seq_lens, wl.T, layer.block_table, layer.P_K,
+                      layer.U_K, layer.Z, layer.E, wl.top_k, scores, sel_r, layer.workspace)
+    sel_d = torch.empty_like(sel_r)
+    layer.decode(pb.q, sel=sel_d, max_seq_len=wl.T)
+    status_clean()
+    for b in range(wl.B):
+        for g in range(wl.Hkv):
+            _, ref_sel, _ = oracle_route(pb, b, g, wl.T)
+            np.testing.assert_array_equal(sel_r[b, g].cpu().numpy(), ref_sel)
+            np.testing.assert_array_equal(sel_d[b, g].cpu().numpy(), ref_sel)
