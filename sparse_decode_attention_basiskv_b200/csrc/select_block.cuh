@@ -56,6 +56,9 @@ __device__ __forceinline__ int value_bin(uint32_t k, float vmin, float scale) {
 }
 
 // Exclusive prefix sum over a block of NT threads; *total receives the sum.
+// One barrier: each thread adds up the warp totals before its own warp
+// itself (at most 15 shared reads).  sh must not be written again until the
+// block has met at another barrier.
 template <int NT>
 __device__ int block_excl_scan(int v, int* sh, int* total) {
   constexpr int W = NT / 32;
@@ -68,20 +71,15 @@ __device__ int block_excl_scan(int v, int* sh, int* total) {
   }
   if (lane == 31) sh[warp] = x;
   __syncthreads();
-  if (warp == 0) {
-    int w = lane < W ? sh[lane] : 0;
+  int before = 0, all = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    sh[lane] = w;
+  for (int w = 0; w < W; ++w) {
+    const int t = sh[w];
+    before += w < warp ? t : 0;
+    all += t;
   }
-  __syncthreads();
-  const int res = (warp ? sh[warp - 1] : 0) + x - v;
-  *total = sh[W - 1];
-  __syncthreads();
-  return res;
+  *total = all;
+  return before + x - v;
 }
 
 // Selection of one (sequence, KV head) by a block of NT threads.  keys and
@@ -230,7 +228,6 @@ __device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32
         }
       }
       if (tid == 0) ss.radix = m > kSelMembers;
-      __syncthreads();
     } else if (tid == 0) {
       ss.radix = 1;
     }

@@ -238,11 +238,17 @@ __host__ __device__ inline int append_direct_red_floats(int d, int r_v, int r_k)
 // Folds the queries of (sequence, KV head) bg for outputs 32*yblk .. +31:
 //   qt[b][h][j]       = sum_i P_K[g][j][i] q[b][h][i]          j < r_v
 //   qt[b][h][r_v + c] = sum_i q[b][h][i] U_K[g][i][c]           c < r_k
-// Warp w sums the products over the w-th quarter of the head dimension for
-// every head of the group; the four partial sums meet in shared memory
-// (fsm: G*d + 4*G*32 floats).  All loads of a thread are independent, so the
-// block costs about one memory round trip.  Run by kFoldThreads threads
-// (tid = 0..kFoldThreads-1, whole warps) on named barrier bar.
+// Latent outputs (P_K, whose rows hold the head dimension contiguously):
+// warp w sums the products over the w-th quarter of the head dimension for
+// every head of the group, from 16-byte loads of its P_K rows; the four
+// partial sums meet in shared memory.  Residual-code outputs (U_K, whose
+// columns are strided): thread (row block rb, output group og) loads rows
+// 8rb .. 8rb+7 of U_K at columns 8og .. 8og+7 as one 16-byte load each and
+// sums them against every head; the row blocks' partial sums meet in shared
+// memory (fsm: G*d + max(4, d/8)*G*32 floats).  All loads of a thread are
+// independent, so the block costs about one memory round trip.  Run by
+// kFoldThreads threads (tid = 0..kFoldThreads-1, whole warps) on named
+// barrier bar.
 __device__ __forceinline__ void fold_query_block(const FoldQArgs& a, int bg, int yblk,
                                                  float* fsm, int tid, int bar) {
   const int b = bg / a.Hkv, g = bg % a.Hkv;
@@ -251,22 +257,62 @@ __device__ __forceinline__ void fold_query_block(const FoldQArgs& a, int bg, int
   const int j = yblk * 32 + lane;
   const int i0 = quarter * (d / 4), n = d / 4;
   float* qs = fsm;            // [G][d]
-  float* part = fsm + G * d;  // [4][G][32]
+  float* part = fsm + G * d;  // [4][G][32], or [d/8][G][32] for residual outputs
   pdl_wait();
-  // This thread's factor values go out first, all at once (they do not
-  // depend on the queries): a row quarter of P_K (n/8 <= 4 chunks of 16
-  // bytes) or a column quarter of U_K (n <= 32 values).
-  const bool is_p = j < a.r_v, is_u = !is_p && j < rq;
+  if (yblk * 32 >= a.r_v) {  // residual-code outputs: U_K columns cs .. cs + nout - 1
+    const int cs = yblk * 32 - a.r_v, nout = min(32, a.r_k - cs), ngr = nout / 8;
+    const int rb = tid / max(ngr, 1), og = tid - rb * max(ngr, 1);
+    const bool act = ngr > 0 && rb < d / 8;
+    uint4 w[8];
+    if (act) {
+      const uint16_t* src = a.U_K + ((size_t)g * d + 8 * rb) * a.r_k + cs + 8 * og;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        w[r] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * a.r_k));
+    }
+    const uint4* q8 = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + g * G) * d);
+    for (int i = tid; i < G * d / 8; i += kFoldThreads) {
+      const uint4 x = q8[i];
+      float4* dst = reinterpret_cast<float4*>(qs + 8 * i);
+      dst[0] = make_float4(bf16lo(x.x), bf16hi(x.x), bf16lo(x.y), bf16hi(x.y));
+      dst[1] = make_float4(bf16lo(x.z), bf16hi(x.z), bf16lo(x.w), bf16hi(x.w));
+    }
+    named_bar_sync(bar, kFoldThreads);
+    if (act) {
+      for (int h = 0; h < G; ++h) {
+        float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const float qv = qs[h * d + 8 * rb + r];
+          const uint32_t u[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc8[2 * e] = fmaf(qv, bf16lo(u[e]), acc8[2 * e]);
+            acc8[2 * e + 1] = fmaf(qv, bf16hi(u[e]), acc8[2 * e + 1]);
+          }
+        }
+        float4* dst = reinterpret_cast<float4*>(part + (rb * G + h) * 32 + 8 * og);
+        dst[0] = make_float4(acc8[0], acc8[1], acc8[2], acc8[3]);
+        dst[1] = make_float4(acc8[4], acc8[5], acc8[6], acc8[7]);
+      }
+    }
+    named_bar_sync(bar, kFoldThreads);
+    for (int o = tid; o < G * nout; o += kFoldThreads) {
+      const int h = o / nout, c = o - h * nout;
+      float v = 0.f;
+      for (int r8 = 0; r8 < d / 8; ++r8) v += part[(r8 * G + h) * 32 + c];
+      a.qt[((size_t)b * a.Hq + g * G + h) * rq + a.r_v + cs + c] = v;
+    }
+    return;
+  }
+  // Latent outputs.  This thread's factor values go out first, all at once
+  // (they do not depend on the queries): a row quarter of P_K (n/8 <= 4
+  // chunks of 16 bytes).
   uint4 prow[4];
-  float ucol[32];
-  if (is_p) {
+  {
     const uint4* row = reinterpret_cast<const uint4*>(a.P_K + ((size_t)g * a.r_v + j) * d + i0);
 #pragma unroll
     for (int c = 0; c < 4; ++c) prow[c] = c < n / 8 ? row[c] : make_uint4(0u, 0u, 0u, 0u);
-  } else if (is_u) {
-    const uint16_t* col = a.U_K + (size_t)g * d * a.r_k + (j - a.r_v) + (size_t)i0 * a.r_k;
-#pragma unroll
-    for (int k = 0; k < 32; ++k) ucol[k] = k < n ? bf16_to_f(col[(size_t)k * a.r_k]) : 0.f;
   }
   {  // the group's queries: 16-byte loads, all in flight together (G*d/8 <= 128)
     const uint4* q8 = reinterpret_cast<const uint4*>(a.q + ((size_t)b * a.Hq + g * G) * d);
@@ -281,7 +327,7 @@ __device__ __forceinline__ void fold_query_block(const FoldQArgs& a, int bg, int
   float acc[8];
 #pragma unroll
   for (int h = 0; h < 8; ++h) acc[h] = 0.f;
-  if (is_p) {
+  {
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       if (c >= n / 8) break;
@@ -297,18 +343,6 @@ __device__ __forceinline__ void fold_query_block(const FoldQArgs& a, int bg, int
             acc[h] = fmaf(p1, qv.y, fmaf(p0, qv.x, acc[h]));
           }
       }
-    }
-  } else if (is_u) {
-#pragma unroll
-    for (int k = 0; k < 32; k += 4) {
-      if (k >= n) break;
-#pragma unroll
-      for (int h = 0; h < 8; ++h)
-        if (h < G) {
-          const float4 qv = *reinterpret_cast<const float4*>(qs + h * d + i0 + k);
-          acc[h] = fmaf(ucol[k + 3], qv.w,
-                        fmaf(ucol[k + 2], qv.z, fmaf(ucol[k + 1], qv.y, fmaf(ucol[k], qv.x, acc[h]))));
-        }
     }
   }
 #pragma unroll
@@ -329,7 +363,7 @@ __host__ __device__ inline size_t append_block_smem(int d, int r_v, int r_k) {
   return (size_t)(2 * d * r_v + d * r_k) * sizeof(uint16_t);
 }
 __host__ __device__ inline size_t fold_block_smem(int G, int d) {
-  return (size_t)(G * d + 4 * G * 32) * sizeof(float);
+  return (size_t)(G * d + (d / 8 > 4 ? d / 8 : 4) * G * 32) * sizeof(float);
 }
 static_assert(kAppendThreads == kFoldThreads, "the prologue's groups share one size");
 
