@@ -63,7 +63,7 @@ N_TOKENS = 8   # distinct appended tokens per layer cycled over the steps (--sta
 
 def algorithmic_bytes(wl, T: int, append: bool = True) -> dict:
     """Bytes one decode step must move at context length T (after append)."""
-    S = wl.page_size
+    S = wl.sel_page  # tokens per selected (routing) page
     P = -(-T // S)
     sel = min(wl.top_k, P)
     r = wl.router  # the router reads z[:, :r_b] and e[:, :r_q]

@@ -128,6 +128,20 @@ typedef struct basiskv_dims {
    *      is divided out of the scores, so queries of any fp32 magnitude
    *      keep about 22 (routing) or all 8 (attention) significant bits. */
   int32_t cache_fp8;
+  /* Routing page (Table 10's adopted Page4: pages of 4 tokens are scored and
+   * selected; Table 9's budget counts tokens):
+   *   0 = page_size (a routing page is a cache page)
+   *   4 or 8 with page_size 16 or 32: the cache keeps its page_size pages
+   *     (one block-table entry per page_size tokens), while the router
+   *     scores every route_page tokens, and top_k, sink_pages,
+   *     recent_pages, the selection and page_scores count routing pages.
+   *     Needs the bf16 caches, a router with a plain-load instance for it
+   *     (listed with basiskv_route), and, for basiskv_decode /
+   *     basiskv_decode_latents, a batch whose (sequence, KV head) groups
+   *     fit one wave of the fused selection + attention launch
+   *     (basiskv_workspace_size returns 0 otherwise); basiskv_attend does
+   *     not take it (BASISKV_ERR_UNSUPPORTED_SHAPE). */
+  int32_t route_page;
 } basiskv_dims;
 
 enum basiskv_status {

@@ -40,7 +40,7 @@ class Dims(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "B", "Hq", "Hkv", "d", "hidden", "r_v", "r_k", "page_size",
         "max_pages_per_seq", "num_phys_pages",
-        "route_r_v", "route_r_k", "sink_pages", "recent_pages", "cache_fp8")]
+        "route_r_v", "route_r_k", "sink_pages", "recent_pages", "cache_fp8", "route_page")]
 
     @classmethod
     def of(cls, B, Hq, Hkv, d, hidden, r_v, r_k, page_size, max_pages_per_seq,

@@ -132,6 +132,10 @@ int route_rv(const basiskv_dims* d) { return d->route_r_v ? d->route_r_v : d->r_
 int route_rk(const basiskv_dims* d) { return d->route_r_k ? d->route_r_k : d->r_k; }
 int sink_pages(const basiskv_dims* d) { return d->sink_pages == 0 ? 1 : (d->sink_pages < 0 ? 0 : d->sink_pages); }
 int recent_pages(const basiskv_dims* d) { return d->recent_pages == 0 ? 1 : d->recent_pages; }
+// Routing page: tokens per score and per selected page (the cache page by default).
+int route_page(const basiskv_dims* d) { return d->route_page ? d->route_page : d->page_size; }
+// Scores per cache page.
+int route_spp(const basiskv_dims* d) { return d->page_size / route_page(d); }
 
 int check_dims(const basiskv_dims* d) {
   if (!d) return BASISKV_ERR_INVALID_ARG;
@@ -162,6 +166,14 @@ int check_dims(const basiskv_dims* d) {
   if ((route_rv(d) < d->r_v || route_rk(d) < d->r_k) &&
       !route_narrow_supported(G, d->r_v, d->r_k, route_rv(d), route_rk(d), d->page_size))
     return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  // routing page
+  if (d->route_page != 0 && d->route_page != d->page_size) {
+    if (d->route_page != 4 && d->route_page != 8) return BASISKV_ERR_INVALID_ARG;
+    if (d->route_page > d->page_size || d->cache_fp8 ||
+        !route_subpage_supported(G, d->r_v, d->r_k, route_rv(d), route_rk(d), d->page_size,
+                                 d->route_page))
+      return BASISKV_ERR_UNSUPPORTED_SHAPE;
+  }
   // cache element type
   if (d->cache_fp8 != 0 && d->cache_fp8 != 1) return BASISKV_ERR_INVALID_ARG;
   if (d->cache_fp8 &&
@@ -177,7 +189,7 @@ int check_len_topk(const basiskv_dims* d, int top_k, int max_seq_len) {
     return BASISKV_ERR_INVALID_ARG;
   // Page selection keeps a 32-bit key and a block-table entry per page in
   // shared memory.
-  const long long P = (max_seq_len + d->page_size - 1) / d->page_size;
+  const long long P = (max_seq_len + route_page(d) - 1) / route_page(d);
   if (P * 8 > 200 * 1024) return BASISKV_ERR_UNSUPPORTED_SHAPE;
   return BASISKV_OK;
 }
@@ -205,7 +217,7 @@ WsLayout ws_layout(const basiskv_dims* d, int top_k) {
   w.qt = off;
   off += align256((size_t)d->B * d->Hq * (d->r_v + d->r_k) * 4);
   w.scores = off;
-  off += align256((size_t)d->B * d->Hkv * d->max_pages_per_seq * 4);
+  off += align256((size_t)d->B * d->Hkv * d->max_pages_per_seq * route_spp(d) * 4);
   w.sel = off;
   off += align256((size_t)d->B * d->Hkv * top_k * 4);
   w.selp = off;  // physical pages of the selection
@@ -367,11 +379,13 @@ int run_route(const basiskv_dims* d, const basiskv_bf16* q, const int32_t* seq_l
   r.rb = route_rv(d);
   r.rq = route_rk(d);
   r.fp8 = d->cache_fp8;
+  r.rp = route_page(d);
   rc = launch_status(launch_route_scores(r, tmZ, tmE, wz, we, st, pdl));
   if (rc || !sel) return rc;  // no selection requested: scores only
-  SelectArgs s{scores, seq_lens, sel, d->B, d->Hkv, d->page_size, d->max_pages_per_seq, top_k,
+  SelectArgs s{scores, seq_lens, sel, d->B, d->Hkv, route_page(d), d->max_pages_per_seq, top_k,
                max_seq_len, len_offset, block_table,
-               reinterpret_cast<int32_t*>(ws + L.selp), sink_pages(d), recent_pages(d)};
+               route_spp(d) > 1 ? nullptr : reinterpret_cast<int32_t*>(ws + L.selp),
+               sink_pages(d), recent_pages(d), route_spp(d)};
   if (with_append) return launch_status(launch_select_append(s, *with_append, st, pdl));
   return launch_status(launch_select(s, st, pdl));
 }
@@ -413,8 +427,8 @@ AttendArgs make_attend_args(const basiskv_dims* d, const basiskv_bf16* q, const 
 // The cluster size of the fused selection + attention launch for this step
 // (0: the step takes the separate selection and attention launches).
 int fused_cluster(const basiskv_dims* d, int top_k, int max_seq_len) {
-  return select_attend_cluster_size(d->Hq / d->Hkv, d->d, d->r_v, d->page_size, d->cache_fp8,
-                                    d->B, d->Hkv, max_seq_len, top_k);
+  return select_attend_cluster_size(d->Hq / d->Hkv, d->d, d->r_v, d->page_size, route_page(d),
+                                    d->cache_fp8, d->B, d->Hkv, max_seq_len, top_k);
 }
 
 // Selection and attention of a fused step in one launch (after the scores):
@@ -426,11 +440,12 @@ int run_select_attend(const basiskv_dims* d, const basiskv_bf16* q, const int32_
   unsigned int* status = device_status_ptr();
   if (!status) return BASISKV_ERR_CUDA;
   SelectArgs s{reinterpret_cast<float*>(ws + L.scores), seq_lens, sel, d->B, d->Hkv,
-               d->page_size, d->max_pages_per_seq, top_k, max_seq_len, len_offset, block_table,
-               nullptr, sink_pages(d), recent_pages(d)};
+               route_page(d), d->max_pages_per_seq, top_k, max_seq_len, len_offset,
+               block_table, nullptr, sink_pages(d), recent_pages(d), route_spp(d)};
   AttendArgs a = make_attend_args(d, q, seq_lens, block_table, K_cache, Z_cache, nullptr, nullptr,
                                   top_k, ws, L, len_offset, status);
   a.early_inputs = 1;
+  a.rp = route_page(d);
   a.a_bf16 = a_bf16;
   return launch_status(launch_select_attend(s, a, st, pdl));
 }
@@ -635,6 +650,7 @@ int basiskv_attend(const basiskv_dims* dims, const basiskv_bf16* q, const int32_
   if (rc) return rc;
   rc = check_len_topk(dims, top_k, max_seq_len);
   if (rc) return rc;
+  if (route_spp(dims) > 1) return BASISKV_ERR_UNSUPPORTED_SHAPE;  // takes cache pages only
   BKV_REQUIRE(q);
   BKV_REQUIRE4(seq_lens);
   BKV_REQUIRE4(block_table);
@@ -722,6 +738,7 @@ int basiskv_decode(const basiskv_dims* dims, const basiskv_bf16* q, const basisk
                                     block_table, A_V, P_K, U_K, K_cache, Z_cache, E_cache);
   if (!app.status) return BASISKV_ERR_CUDA;
   const bool fused = fused_cluster(dims, top_k, max_seq_len) > 0;
+  if (route_spp(dims) > 1 && !fused) return BASISKV_ERR_UNSUPPORTED_SHAPE;  // routing pages
   {
     FoldQArgs f{q, P_K, U_K, reinterpret_cast<float*>(ws + L.qt), dims->B, dims->Hq, dims->Hkv,
                 dims->d, dims->r_v, dims->r_k};
@@ -793,6 +810,7 @@ int basiskv_decode_latents(const basiskv_dims* dims, const basiskv_bf16* q,
                                     block_table, A_V, P_K, U_K, K_cache, Z_cache, E_cache);
   if (!app.status) return BASISKV_ERR_CUDA;
   const bool fused = fused_cluster(dims, top_k, max_seq_len) > 0;  // as in basiskv_decode
+  if (route_spp(dims) > 1 && !fused) return BASISKV_ERR_UNSUPPORTED_SHAPE;
   {
     FoldQArgs f{q, P_K, U_K, reinterpret_cast<float*>(ws + L.qt), dims->B, dims->Hq, dims->Hkv,
                 dims->d, dims->r_v, dims->r_k};

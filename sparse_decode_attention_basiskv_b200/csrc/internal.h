@@ -94,7 +94,11 @@ struct RouteArgs {
   unsigned int* status;
   int rb, rq;  // widths the router reads: z[:, :rb], e[:, :rq]
   int fp8;     // Z and E hold E4M3 bytes
+  int rp;      // routing page (tokens per score); S: one score per cache page
 };
+// Whether the plain-load scoring kernel has an instance for routing pages
+// of rp < S tokens with this router.
+bool route_subpage_supported(int G, int r_v, int r_k, int rb, int rq, int S, int rp);
 // Whether the plain-load scoring kernel has an instance for a router
 // narrower than the cached widths.
 bool route_narrow_supported(int G, int r_v, int r_k, int rb, int rq, int S);
@@ -106,7 +110,7 @@ cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
                                 bool pdl);
 
 struct SelectArgs {
-  const float* scores;
+  const float* scores;  // [B][Hkv][max_pages * spp]
   const int32_t* seq_lens;
   int32_t* sel;  // [B][Hkv][top_k]
   int B, Hkv, S, max_pages, top_k, max_seq_len;
@@ -116,6 +120,9 @@ struct SelectArgs {
   const int32_t* block_table;
   int32_t* sel_phys;  // [B][Hkv][top_k] or null
   int n_sink, n_recent;  // leading / trailing pages always kept
+  // Scores per cache page (routing pages of S tokens each, S above being
+  // the routing page): 1, or page_size / route_page (sel_phys then null).
+  int spp;
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st, bool pdl);
 // The selection together with a one-token append (a.n_new == 1), whose
@@ -149,6 +156,7 @@ struct AttendArgs {
   int early_inputs;
   int zsplit;  // Z tiles store their first zsplit columns first
   int fp8;     // K and Z hold E4M3 bytes
+  int rp;      // routing page: sel holds routing pages of rp tokens (rp <= S)
 };
 int attend_pages_per_split(int S);
 // Plain-load tensor-core attention with its own merge (needs a.cnt zeroed,
@@ -164,7 +172,7 @@ cudaError_t launch_attend_mma(const AttendArgs& a, cudaStream_t st, bool pdl);
 // of CTAs per (sequence, KV head) (select_attend.cuh).  The cluster size for
 // a step, or 0 when the step does not fit one wave (then the selection and
 // the attention launch separately).  s.sel, when set, receives the selection.
-int select_attend_cluster_size(int G, int d, int r_v, int S, int fp8, int B, int Hkv,
+int select_attend_cluster_size(int G, int d, int r_v, int S, int rp, int fp8, int B, int Hkv,
                                int max_seq_len, int top_k);
 cudaError_t launch_select_attend(const SelectArgs& s, const AttendArgs& a, cudaStream_t st,
                                  bool pdl);

@@ -563,9 +563,35 @@ cudaError_t launch_fold_query(const FoldQArgs& a, cudaStream_t st, bool pdl) {
   return launch_k(fold_query_kernel, grid, dim3(kFoldThreads), smem, st, pdl, a);
 }
 
+// Routers with routing pages smaller than the cache page (G, r_v, r_k, rb,
+// rq, S, rp): the pages' B16R16 router and the full-width router at the
+// Llama-3.1-8B (page 16) and Qwen3-32B (page 32) shapes.
+#define BKV_RM_SUBPAGE(X)                                                             \
+  X(4, 64, 32, 16, 16, 16, 4) X(4, 64, 32, 16, 16, 16, 8) X(4, 96, 32, 16, 16, 16, 4) \
+  X(4, 64, 32, 64, 32, 16, 4) X(4, 96, 32, 96, 32, 16, 4) X(8, 96, 32, 16, 16, 32, 4) \
+  X(8, 96, 32, 96, 32, 32, 4)
+
+bool route_subpage_supported(int G, int r_v, int r_k, int rb, int rq, int S, int rp) {
+#define BKV_RMP(GG, V, K, RB_, RQ_, SS, RP_) \
+  if (G == GG && r_v == V && r_k == K && rb == RB_ && rq == RQ_ && S == SS && rp == RP_) return true;
+  BKV_RM_SUBPAGE(BKV_RMP)
+#undef BKV_RMP
+  return false;
+}
+
 cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
                                 const CUtensorMap& tmE, int wz, int we, cudaStream_t st,
                                 bool pdl) {
+  if (a.rp && a.rp != a.S) {  // routing pages smaller than the cache page
+    if (a.fp8 || !(a.Z && a.E)) return cudaErrorNotSupported;
+#define BKV_RMP(GG, V, K, RB_, RQ_, SS, RP_)                                              \
+  if (a.G == GG && a.r_v == V && a.r_k == K && a.rb == RB_ && a.rq == RQ_ && a.S == SS && \
+      a.rp == RP_)                                                                       \
+    return launch_route_mma<GG, V, K, RB_, RQ_, SS, RP_>(a, st, pdl);
+    BKV_RM_SUBPAGE(BKV_RMP)
+#undef BKV_RMP
+    return cudaErrorNotSupported;
+  }
   if (a.fp8) return launch_route_scores_fp8(a, st, pdl);
   if ((a.rb != a.r_v || a.rq != a.r_k) && !(a.Z && a.E)) return cudaErrorNotSupported;
   if (a.Z && a.E) {

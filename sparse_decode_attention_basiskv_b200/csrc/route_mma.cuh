@@ -173,9 +173,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // (lane c loads columns 8c .. 8c+7, 16 bytes: two k-steps of the MMA) and at
 // most one 16-column tail chunk (lane c loads columns 4c .. 4c+3, 8 bytes:
 // one k-step), so every lane loads and every loaded byte is used.
-template <int G, int RV, int RK, int RB, int RQ, int S, int PW>
+// RP: the routing page (RP = S: one score per cache page; RP = 4 or 8: the
+// router scores every RP tokens of a cache page, S / RP scores a page, the
+// scores row of a group holding max_pages * S / RP entries).
+template <int G, int RV, int RK, int RB, int RQ, int S, int PW, int RP = S>
 __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S>()))
     route_mma_kernel(RouteArgs a) {
+  static_assert(RP == S || RP == 4 || RP == 8, "routing pages of 4 or 8 tokens, or the page");
+  constexpr int NR = S / RP;  // routing pages per cache page
   extern __shared__ uint4 rm_frags[];
   constexpr int NZF = RB / 32, NZH = (RB % 32) / 16, NEF = RQ / 32, NEH = (RQ % 32) / 16;
   constexpr int NCZ = NZF + NZH, NC = NCZ + NEF + NEH, NT = S / 8, RQ_ = RV + RK;
@@ -277,7 +282,9 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S>()))
       }
     }
     // This lane's maximum over page k's live tokens and the group's heads
-    // (the warp reduction follows).
+    // (the warp reduction follows); with routing pages smaller than 8
+    // tokens, per 8-token tile instead (tbest[t]).
+    float tbest[NT];
     auto page_best = [&](int k) -> float {
       float acc[NT][SETS][4];
 #pragma unroll
@@ -313,15 +320,47 @@ __global__ void __launch_bounds__(kRmThreads, (rm_ctas_per_sm<G, RB, RQ, S>()))
           s1 = lr < G ? acc[t][0][1] + (acc[t][0][3] + lo1) : -INFINITY;
         }
         const int tok = ulp[k] * S + t * 8 + 2 * lc;
-        if (tok < uT[k]) best = fmaxf(best, s0);
-        if (tok + 1 < uT[k]) best = fmaxf(best, s1);
+        float tb = -INFINITY;
+        if (tok < uT[k]) tb = s0;
+        if (tok + 1 < uT[k]) tb = fmaxf(tb, s1);
+        tbest[t] = tb;
+        best = fmaxf(best, tb);
       }
       return best;
+    };
+    // The scores of the routing pages of page k (RP < S): tile t's maximum
+    // over the lanes that hold tokens of the same routing page (RP = 4:
+    // lanes with equal c >> 1; RP = 8: the whole warp), written by one lane
+    // per routing page.
+    auto routing_scores = [&](int k) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        float v = tbest[t];
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+        if (RP == 8) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        const int sub = RP == 8 ? t : 2 * t + (lc >> 1);
+        if (lr == 0 && (RP == 8 ? lc == 0 : (lc & 1) == 0))
+          a.scores[(size_t)ubg[k] * a.max_pages * NR + (size_t)ulp[k] * NR + sub] = v;
+      }
     };
     bool one_group = true;
 #pragma unroll
     for (int k = 1; k < PW; ++k) one_group = one_group && (!uok[k] || ubg[k] == ubg[0]);
-    if (one_group) {  // the common case: the batch's pages are scored side by side
+    if (NR > 1) {  // routing pages smaller than the cache page: scored one page at a time
+#pragma unroll
+      for (int k = 0; k < PW; ++k) {
+        if (!uok[k]) continue;
+        if (ubg[k] != frag_bg) {
+          load_frags(ub[k], ug[k]);
+          frag_bg = ubg[k];
+        }
+        (void)page_best(k);
+        routing_scores(k);
+      }
+    } else if (one_group) {  // the common case: the batch's pages are scored side by side
       if (ubg[0] != frag_bg) {
         load_frags(ub[0], ug[0]);
         frag_bg = ubg[0];
@@ -366,7 +405,7 @@ constexpr int rm_pages_per_batch() {
                     : 1);
 }
 
-template <int G, int RV, int RK, int RB, int RQ, int S>
+template <int G, int RV, int RK, int RB, int RQ, int S, int RP = S>
 cudaError_t launch_route_mma(const RouteArgs& a, cudaStream_t st, bool pdl) {
   constexpr int PW = rm_pages_per_batch<RB, RQ, S>();
   constexpr int NC = (RB + 31) / 32 + (RQ + 31) / 32;
@@ -378,11 +417,11 @@ cudaError_t launch_route_mma(const RouteArgs& a, cudaStream_t st, bool pdl) {
   if (grid < 1) grid = 1;
   const size_t smem = (size_t)kRmWarps * (G == 8 ? 2 : 1) * NC * 2 * 32 * 16;
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(route_mma_kernel<G, RV, RK, RB, RQ, S, PW>,
+    cudaError_t e = cudaFuncSetAttribute(route_mma_kernel<G, RV, RK, RB, RQ, S, PW, RP>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  return launch_k(route_mma_kernel<G, RV, RK, RB, RQ, S, PW>, dim3((unsigned)grid),
+  return launch_k(route_mma_kernel<G, RV, RK, RB, RQ, S, PW, RP>, dim3((unsigned)grid),
                   dim3(kRmThreads), smem, st, pdl, a);
 }
 

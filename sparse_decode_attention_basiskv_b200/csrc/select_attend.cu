@@ -4,11 +4,11 @@
 
 namespace basiskv {
 
-int select_attend_cluster_size(int G, int d, int r_v, int S, int fp8, int B, int Hkv,
+int select_attend_cluster_size(int G, int d, int r_v, int S, int rp, int fp8, int B, int Hkv,
                                int max_seq_len, int top_k) {
   if (fp8 ? !attend_mma_fp8_supported(G, d, r_v, S) : !attend_mma_supported(G, d, r_v, S))
     return 0;
-  const int P_max = (max_seq_len + S - 1) / S;
+  const int P_max = (max_seq_len + rp - 1) / rp;  // routing pages
   return select_attend_cluster(G, d, r_v, fp8 != 0, B, Hkv, P_max, top_k, num_sms());
 }
 

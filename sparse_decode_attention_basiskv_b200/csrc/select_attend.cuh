@@ -28,6 +28,7 @@
 // CTAs); larger batches keep the two-launch path.
 #pragma once
 
+#include <climits>
 #include <cooperative_groups.h>
 
 #include "attend_mma.cuh"
@@ -112,6 +113,11 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
   const int rank = C > 1 ? (int)cg::this_cluster().block_rank() : 0;
   const int bg = blockIdx.x / C, b = bg / a.Hkv, g = bg - b * a.Hkv;
   const int S = a.S, TP = S >> 4, logS = 31 - __clz(S);
+  // Routing pages of RPG tokens (the selection's unit); NR per cache page.
+  // A 16-token unit is 1 / TP of a routing page of S tokens, or QP routing
+  // pages of 4 or 8 tokens.
+  const int RPG = a.rp ? a.rp : S, NR = S / RPG, QP = RPG < 16 ? 16 / RPG : 0;
+  const int P_phys = (s.max_seq_len + S - 1) / S;  // block-table entries read
 
   // The out-projection may take SMs as this grid's CTAs retire; it requests
   // only its weight tiles before its own wait.
@@ -130,7 +136,7 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
   }
   {
     const int32_t* row = a.block_table + (size_t)b * a.max_pages;
-    for (int i = tid; i < P_max; i += kAmThreads) cp_async4(tbl + i, row + i);
+    for (int i = tid; i < P_phys; i += kAmThreads) cp_async4(tbl + i, row + i);
   }
   cp_async_commit();
   pdl_wait();  // the page scores are the previous launch's output
@@ -138,8 +144,8 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
   cp_async_wait_all();
   __syncthreads();  // the page list, queries and block-table row are in; region A is free
   T = T < 0 ? 0 : (T > s.max_seq_len ? s.max_seq_len : T);
-  const int nsel = min(a.top_k, (T + S - 1) / S);
-  const int U = nsel * TP;  // units with a page
+  const int nsel = min(a.top_k, (T + RPG - 1) / RPG);
+  const int U = QP ? (nsel + QP - 1) / QP : nsel * TP;  // units with a page
   const int u0 = (int)((long)U * rank / C), u1 = (int)((long)U * (rank + 1) / C);
   const int count = u0 + warp < u1 ? (u1 - u0 - warp + kAmWarps - 1) / kAmWarps : 0;
 
@@ -189,84 +195,108 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
 #pragma unroll
     for (int e = 0; e < 2; ++e) acc[c][e][0] = acc[c][e][1] = acc[c][e][2] = acc[c][e][3] = 0.f;
 
-  // Unit nn of this warp is unit u0 + warp + 8 nn of the group: slot / TP of
-  // the page list, 16-token part % TP of that page.  A bad block-table entry
-  // is flagged and read as page 0.
-  auto unit_ids = [&](int nn, int& lp, int& pp) {
-    const int idx = u0 + warp + kAmWarps * nn;
-    lp = list[idx / TP];
-    pp = lp >= 0 && lp < P_max ? tbl[lp] : -1;
+  // Unit nn of this warp is unit u0 + warp + 8 nn of the group.  This lane
+  // holds tokens lr and lr + 8 of it: their cache rows (global row index in
+  // the [page][KV head][S] row space) and their positions in the sequence
+  // (past the length when there is no page).  Routing pages of S tokens:
+  // the unit is part idx % TP of list entry idx / TP.  Smaller routing
+  // pages: token x is row x % RPG of list entry idx * QP + x / RPG, which
+  // sits at row (page % NR) * RPG of cache page page / NR.  A bad
+  // block-table entry is flagged and read as page 0.
+  struct Rows {
+    size_t r0, r1;
+    int p0, p1;
+  };
+  auto cache_page = [&](int lp) -> int {
+    int pp = lp >= 0 && lp / NR < P_phys ? tbl[lp / NR] : -1;
     if (lp < 0) {
       pp = 0;
     } else if (pp < 0 || pp >= a.num_phys) {
       if (lane == 0) raise_status(a.status, BASISKV_DEV_BAD_PAGE);
       pp = 0;
     }
+    return pp;
   };
-  auto unit_row = [&](int nn, int pp) -> size_t {
-    const int tau = (u0 + warp + kAmWarps * nn) % TP;
-    return ((size_t)pp * a.Hkv + g) * S + 16 * tau + lr;
+  auto unit_rows = [&](int nn) -> Rows {
+    const int idx = u0 + warp + kAmWarps * nn;
+    Rows u;
+    if (QP == 0) {
+      const int lp = list[idx / TP], tau = idx % TP;
+      u.r0 = ((size_t)cache_page(lp) * a.Hkv + g) * S + 16 * tau + lr;
+      u.r1 = u.r0 + 8;
+      u.p0 = lp >= 0 ? lp * S + 16 * tau + lr : INT_MAX;
+      u.p1 = lp >= 0 ? u.p0 + 8 : INT_MAX;
+    } else {
+      const int x0 = lr, x1 = lr + 8;
+      const int s0 = idx * QP + x0 / RPG, s1 = idx * QP + x1 / RPG;
+      const int lp0 = s0 < nsel ? list[s0] : -1, lp1 = s1 < nsel ? list[s1] : -1;
+      u.r0 = ((size_t)cache_page(lp0) * a.Hkv + g) * S + (lp0 >= 0 ? lp0 % NR : 0) * RPG +
+             x0 % RPG;
+      u.r1 = ((size_t)cache_page(lp1) * a.Hkv + g) * S + (lp1 >= 0 ? lp1 % NR : 0) * RPG +
+             x1 % RPG;
+      u.p0 = lp0 >= 0 ? lp0 * RPG + x0 % RPG : INT_MAX;
+      u.p1 = lp1 >= 0 ? lp1 * RPG + x1 % RPG : INT_MAX;
+    }
+    return u;
   };
   uint4 kx[NKC][2], zx[NZC][2];
-  auto load_k = [&](size_t row) {
+  auto load_k = [&](const Rows& u) {
     if constexpr (F8) {
       const uint8_t* K8 = reinterpret_cast<const uint8_t*>(a.K);
 #pragma unroll
       for (int c = 0; c < NKC; ++c) {
-        ldg_stream8(kx[c][0], K8 + row * D + 32 * c + 8 * lc);
-        ldg_stream8(kx[c][1], K8 + (row + 8) * D + 32 * c + 8 * lc);
+        ldg_stream8(kx[c][0], K8 + u.r0 * D + 32 * c + 8 * lc);
+        ldg_stream8(kx[c][1], K8 + u.r1 * D + 32 * c + 8 * lc);
       }
     } else {
 #pragma unroll
       for (int c = 0; c < NKC; ++c) {
-        kx[c][0] = ldg_stream(a.K + row * D + 32 * c + 8 * lc);
-        kx[c][1] = ldg_stream(a.K + (row + 8) * D + 32 * c + 8 * lc);
+        kx[c][0] = ldg_stream(a.K + u.r0 * D + 32 * c + 8 * lc);
+        kx[c][1] = ldg_stream(a.K + u.r1 * D + 32 * c + 8 * lc);
       }
     }
   };
-  auto load_z = [&](size_t row, int slot) {  // asynchronous, into the warp's ring
-    const size_t tile = row >> logS;
-    const int trow = (int)(row & (S - 1));
+  auto load_z = [&](const Rows& u, int slot) {  // asynchronous, into the warp's ring
+    const size_t tile0 = u.r0 >> logS, tile1 = u.r1 >> logS;
+    const int trow0 = (int)(u.r0 & (S - 1)), trow1 = (int)(u.r1 & (S - 1));
     if constexpr (F8) {
-      const uint8_t* zt8 = reinterpret_cast<const uint8_t*>(a.Z) + tile * S * RV;
+      const uint8_t* z8 = reinterpret_cast<const uint8_t*>(a.Z);
 #pragma unroll
       for (int c = 0; c < NZC; ++c) {
         const int col = 32 * c + 8 * lc;
         cp_async8(zring8 + ((slot * NZC + c) * 2 + 0) * 32 + lane,
-                  zt8 + split_off(trow, col, S, RV, a.zsplit));
+                  z8 + tile0 * S * RV + split_off(trow0, col, S, RV, a.zsplit));
         cp_async8(zring8 + ((slot * NZC + c) * 2 + 1) * 32 + lane,
-                  zt8 + split_off(trow + 8, col, S, RV, a.zsplit));
+                  z8 + tile1 * S * RV + split_off(trow1, col, S, RV, a.zsplit));
       }
       return;
     }
-    const uint16_t* zt = a.Z + tile * S * RV;
 #pragma unroll
     for (int c = 0; c < NZC; ++c) {
       const int col = 32 * c + 8 * lc;
       cp_async16(zring + ((slot * NZC + c) * 2 + 0) * 32 + lane,
-                 zt + split_off(trow, col, S, RV, a.zsplit));
+                 a.Z + tile0 * S * RV + split_off(trow0, col, S, RV, a.zsplit));
       cp_async16(zring + ((slot * NZC + c) * 2 + 1) * 32 + lane,
-                 zt + split_off(trow + 8, col, S, RV, a.zsplit));
+                 a.Z + tile1 * S * RV + split_off(trow1, col, S, RV, a.zsplit));
     }
   };
-  int lp_c = -1, pp_c = 0;
+  Rows cur{0, 8, INT_MAX, INT_MAX};
   if (count > 0) {
-    unit_ids(0, lp_c, pp_c);
-    const size_t row0 = unit_row(0, pp_c);
-    load_k(row0);
-    load_z(row0, 0);
+    cur = unit_rows(0);
+    load_k(cur);
+    load_z(cur, 0);
   }
   cp_async_commit();
   // Unit n computes while unit n + 1 loads: its latents are requested (into
   // shared memory) before unit n starts, its Keys (into registers) as soon
   // as QK has consumed the current ones.
   for (int n = 0; n < count; ++n) {
-    const int tau = (u0 + warp + kAmWarps * n) % TP;
     const bool more = n + 1 < count;
-    int lp_n = -1, pp_n = 0;
-    if (more) unit_ids(n + 1, lp_n, pp_n);
-    const size_t row_n = more ? unit_row(n + 1, pp_n) : 0;
-    if (more) load_z(row_n, (n + 1) & 1);
+    Rows nxt{0, 8, INT_MAX, INT_MAX};
+    if (more) {
+      nxt = unit_rows(n + 1);
+      load_z(nxt, (n + 1) & 1);
+    }
     cp_async_commit();
     float sc4[4] = {0.f, 0.f, 0.f, 0.f};  // [tokens r, r + 8] x [heads 2c, 2c + 1]
 #pragma unroll
@@ -285,9 +315,8 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
         mma_bf16_16816(sc4, kx[c][0].z, kx[c][1].z, kx[c][0].w, kx[c][1].w, qf.z, qf.w);
       }
     }
-    if (more) load_k(row_n);
-    const int pos = lp_c * S + 16 * tau + lr;
-    const bool v0 = lp_c >= 0 && pos < T, v1 = lp_c >= 0 && pos + 8 < T;
+    if (more) load_k(nxt);
+    const bool v0 = cur.p0 < T, v1 = cur.p1 < T;
     const float x00 = v0 ? sc4[0] * sl0 : -INFINITY;
     const float x01 = v0 ? sc4[1] * sl1 : -INFINITY;
     const float x10 = v1 ? sc4[2] * sl0 : -INFINITY;
@@ -367,11 +396,9 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
         }
       }
     }
-    lp_c = lp_n;
-    pp_c = pp_n;
+    cur = nxt;
   }
   cp_async_wait_all();
-  (void)pp_c;
 
   // ---- the CTA's warps meet: per-warp state to shared memory, one partial
 #pragma unroll

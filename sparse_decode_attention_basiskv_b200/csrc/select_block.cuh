@@ -94,7 +94,8 @@ __device__ __forceinline__ void select_group(const SelectArgs& a, int bg, uint32
   const int P_max = (a.max_seq_len + a.S - 1) / a.S;
   const int32_t* bt = a.block_table + (size_t)b * a.max_pages;
   const int ns = a.n_sink, nr = a.n_recent;  // forced leading / trailing pages
-  const float* sc = a.scores + (size_t)bg * a.max_pages + ns;  // candidate i = page ns + i
+  // candidate i = page ns + i (routing pages when spp > 1)
+  const float* sc = a.scores + (size_t)bg * a.max_pages * (a.spp > 1 ? a.spp : 1) + ns;
   // The length, the first batch of scores and the block-table row are
   // requested together (up to the longest possible context; what lies past
   // this sequence's pages is dropped): one memory round trip, not two.

@@ -74,10 +74,16 @@ class Workload:
     sink_pages: int = 0
     recent_pages: int = 0
     cache_fp8: int = 0  # 1: the K, Z and E caches hold FP8 E4M3 values
+    route_page: int = 0  # tokens per routing page (0 = page_size)
 
     @property
     def G(self) -> int:
         return self.Hq // self.Hkv
+
+    @property
+    def sel_page(self) -> int:
+        """Tokens per selected (routing) page: the oracle's page size."""
+        return self.route_page or self.page_size
 
     @property
     def pages(self) -> int:
@@ -110,6 +116,8 @@ class Workload:
             "steps")}
         if (self.route_r_v, self.route_r_k, self.sink_pages, self.recent_pages) != (0, 0, 0, 0):
             out["router"] = self.router
+        if self.route_page:
+            out["route_page"] = self.route_page
         out["cache"] = "e4m3" if self.cache_fp8 else "bf16"
         return out
 
@@ -135,6 +143,13 @@ LLAMA8B_T32K_B16_B16R16 = replace(
 # The headline shape with FP8 E4M3 caches (Table 13's KV format).
 LLAMA8B_T32K_B16_FP8 = replace(LLAMA8B_T32K_B16, name="llama8b_layer_b16_t32k_v64_append1_e4m3",
                                cache_fp8=1)
+# The pages' adopted router configuration (Table 10's Page4; Table 9's
+# budget of 2048 routed tokens plus a 64-token recent window; Table 13's
+# B16R16): 4-token routing pages over the cache's 16-token pages, 512 routed
+# pages + a 16-page recent window, no sink page.
+LLAMA8B_T32K_B16_B16R16_PAGE4 = replace(
+    LLAMA8B_T32K_B16, name="llama8b_layer_b16_t32k_v64_router_b16r16_page4_recent64",
+    top_k=528, route_r_v=16, route_r_k=16, sink_pages=-1, recent_pages=16, route_page=4)
 QWEN32B_T64K_B8 = Workload("qwen32b_layer_b8_t64k_v96_prefill4k", B=8, Hq=64,
                            Hkv=8, d=128, hidden=5120, T=65536, page_size=32,
                            r_v=96, r_k=32, top_k=64, n_planted=8, seed=3,

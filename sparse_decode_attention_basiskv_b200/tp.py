@@ -119,7 +119,7 @@ class TPDecodeLayer:
                     r_k=wl.r_k, page_size=wl.page_size, max_pages_per_seq=pc,
                     num_phys_pages=wl.B * pc, route_r_v=wl.route_r_v, route_r_k=wl.route_r_k,
                     sink_pages=wl.sink_pages, recent_pages=wl.recent_pages,
-                    cache_fp8=wl.cache_fp8)
+                    cache_fp8=wl.cache_fp8, route_page=wl.route_page)
         g0, g1, _, _ = head_shard(wl.Hq, wl.Hkv, world, rank)
         fl = {k: v.to(device).contiguous()
               for k, v in shard_factors(pb.factors, wl.Hq, wl.Hkv, wl.d, world, rank).items()}

@@ -70,7 +70,7 @@ def oracle_route(pb, b: int, g: int, T: int, cache=None) -> tuple:
     qg = np64(pb.q[b, g * wl.G:(g + 1) * wl.G])
     r = wl.router
     sc = O.page_scores(qg, np64(c["Z"][b, g]), np64(c["E"][b, g]), f["P_K"][g], f["U_K"][g], T,
-                       wl.page_size, r["r_b"], r["r_q"])
+                       wl.sel_page, r["r_b"], r["r_q"])
     sel, tie = O.select_pages(sc, wl.top_k, r["n_sink"], r["n_recent"])
     return sc, sel, tie
 
@@ -140,7 +140,7 @@ class StepChecker:
         """(a_ref, y_ref) of one sequence on the GPU's selection."""
         if not other:
             return out["a"], out["y"]
-        G, S = self.wl.G, self.wl.page_size
+        G, S = self.wl.G, self.wl.sel_page
         a = out["a"].copy()
         for g in other:
             a[g * G:(g + 1) * G], _ = O.attend(q_b[g * G:(g + 1) * G], out["K"][g], out["Z"][g],

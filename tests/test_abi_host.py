@@ -247,3 +247,30 @@ def test_noalloc_reports_the_validation_status(lib):
                 num_phys_pages=256 * 25000 // 8)
     assert lib.basiskv_workspace_size(ctypes.byref(big), 64, 400000) > bkv.NOALLOC_SCRATCH_BYTES
     assert _noalloc(lib, big, 64, 400000) == bkv.ERR_SCRATCH_LIMIT
+
+
+def test_route_page_validation(lib):
+    """Routing pages of 4 or 8 tokens (Table 10's Page4) over cache pages of
+    16 or 32: accepted for routers with such an instance and bf16 caches;
+    other values, E4M3 caches and routers without an instance are refused;
+    the standalone attention takes cache pages only."""
+    nar = dict(Hq=8, Hkv=2, r_v=64, r_k=32, route_r_v=16, route_r_k=16, sink_pages=-1,
+               recent_pages=4)
+    ok = _dims(**nar, route_page=4)
+    assert lib.basiskv_workspace_size(ctypes.byref(ok), 64, 1024) > 0
+    assert lib.basiskv_workspace_size(ctypes.byref(_dims(**nar, route_page=8)), 64, 1024) > 0
+    assert lib.basiskv_workspace_size(ctypes.byref(_dims(**nar, route_page=16)), 64, 1024) > 0
+    # the scores hold one entry per routing page
+    plain = lib.basiskv_workspace_size(ctypes.byref(_dims(**nar)), 64, 1024)
+    assert lib.basiskv_workspace_size(ctypes.byref(ok), 64, 1024) > plain
+    for bad, status in ((3, bkv.ERR_INVALID_ARG), (2, bkv.ERR_INVALID_ARG)):
+        d = _dims(**nar, route_page=bad)
+        assert lib.basiskv_route(ctypes.byref(d), FAKE, FAKE, 256, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                 64, None, FAKE, FAKE, 1 << 20, None) == status
+    for d in (_dims(**nar, route_page=4, cache_fp8=1),  # E4M3 caches
+              _dims(route_page=4, r_v=32, r_k=16),      # no routing-page instance
+              _dims(**nar, route_page=8, page_size=8)):  # not smaller than the page
+        assert lib.basiskv_workspace_size(ctypes.byref(d), 64, 1024) == 0
+    a = lib.basiskv_attend(ctypes.byref(ok), FAKE, FAKE, 1024, FAKE, FAKE, FAKE, FAKE, 64, FAKE,
+                           FAKE, 1 << 20, None)
+    assert a == bkv.ERR_UNSUPPORTED_SHAPE

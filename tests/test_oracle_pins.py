@@ -162,7 +162,7 @@ def test_narrow_router_ignores_unread_dimensions():
     sc = O.page_scores(rng.standard_normal((2, d)), z, e, rng.standard_normal((r_v, d)),
                        _orth(rng, d, r_k), T, S, 4, 2)
     np.testing.assert_array_equal(sc, np.zeros_like(sc))
-@pytest.mark.parametrize("T,S", [(37, 8), (32, 8), (5, 16), (64, 16)])
+@pytest.mark.parametrize("T,S", [(37, 8), (32, 8), (5, 16), (64, 16), (39, 4), (3, 4)])
 def test_page_scores_closed_form(T, S):
     """khat_t = c_t u and q_h = alpha_h u  =>  score(p) = max_{t,h} alpha_h c_t.
 
@@ -198,7 +198,7 @@ def _sdpa_gqa(q, K, V):
     return o[0, :, 0].numpy()
 
 
-@pytest.mark.parametrize("T,S", [(40, 8), (48, 16), (7, 8)])
+@pytest.mark.parametrize("T,S", [(40, 8), (48, 16), (7, 8), (22, 4)])
 def test_attend_all_pages_equals_sdpa(T, S):
     rng = np.random.default_rng(T + S)
     G, d, r_v = 4, 16, 6
