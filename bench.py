@@ -462,7 +462,9 @@ def run_gpu(args) -> None:
     # scores-only call: two launches, the scoring kernel is ~98% of them.
     T_r = T_after(W + K - 1)
     layer.seq_lens.fill_(T_r)
-    scores = torch.empty(wl.B, wl.Hkv, layer.dims.max_pages_per_seq, device="cuda")
+    scores = torch.empty(wl.B, wl.Hkv,
+                         layer.dims.max_pages_per_seq * (wl.page_size // wl.sel_page),
+                         device="cuda")
     reps = max(20, min(200, K))
 
     def route():
@@ -1067,9 +1069,11 @@ def main():
                     help="override the batch (smaller cases for profiling)")
     ap.add_argument("--context", type=int, default=0,
                     help="override the context length (smaller cases for profiling)")
-    ap.add_argument("--router", default="full", choices=["full", "b16r16"],
+    ap.add_argument("--router", default="full", choices=["full", "b16r16", "b16r16_page4"],
                     help="full: the default router (all latent and residual dims, sink + "
-                         "newest page); b16r16: the pages' narrow router and budget")
+                         "newest page); b16r16: the pages' narrow router and budget at the "
+                         "cache's 16-token pages; b16r16_page4: the same at 4-token routing "
+                         "pages (2048 routed + 64 recent tokens)")
     ap.add_argument("--cache", default="bf16", choices=["bf16", "e4m3"],
                     help="element type of the K, Z and E caches")
     ap.add_argument("--prefill", action="store_true",
@@ -1088,6 +1092,8 @@ def main():
     WL = DECODE_WORKLOADS[args.workload]
     if args.router == "b16r16":
         WL = synth.LLAMA8B_T32K_B16_B16R16
+    elif args.router == "b16r16_page4":
+        WL = synth.LLAMA8B_T32K_B16_B16R16_PAGE4
     if args.cache == "e4m3":
         WL = synth.with_sizes(WL, cache_fp8=1, name=WL.name + "_e4m3")
     if args.warmup < 3:

@@ -112,9 +112,14 @@ def strerror(status: int) -> str:
 
 
 def _ptr(t) -> int | None:
-    """Device (or host) address of a tensor, None for None."""
+    """Device (or host) address of a tensor, None for None.  The library
+    reads every array as dense row-major memory, so a strided view is
+    refused rather than read in the wrong order."""
     if t is None:
         return None
+    if not t.is_contiguous():
+        raise ValueError(f"tensor of shape {tuple(t.shape)} is not contiguous "
+                         "(call .contiguous() first)")
     return t.data_ptr()
 
 

@@ -8,14 +8,14 @@
 // with W_app,g of shape (r_v + r_k) x 2d.  fold_append_kernel builds W_app
 // (fp32 products, stored bf16) and append_tc_kernel runs the product:
 // 128-token M tiles, N = r_v + r_k, K = 2d, operands staged by TMA in
-// 128-byte-swizzled K-major tiles through a two-slot ring (so two or three
-// CTAs share an SM and one CTA's loads overlap another's epilogue), a
-// single thread issuing tcgen05.mma
+// 128-byte-swizzled K-major tiles, a single thread issuing tcgen05.mma
 // (kind::f16, bf16 inputs, fp32 accumulator in tensor memory), and four
-// epilogue warps that read the accumulator with tcgen05.ld and scatter the
-// bf16 z / e rows, and the exact Key, into the paged caches.  The folded
-// factor is rounded to bf16 once; the decode-time append (append.cu) keeps
-// the two-step form with an unrounded z.
+// epilogue warps that read the accumulator with tcgen05.ld and write the
+// z / e rows, and the exact Key, into the paged caches.  The folded factor
+// is rounded to bf16 once; the decode-time append (append.cu) keeps the
+// two-step form with an unrounded z.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "launch.cuh"
@@ -108,9 +108,27 @@ __global__ void __launch_bounds__(kFoldAppThreads) fold_append_kernel(FoldAppArg
 }
 
 // ------------------------------------------------------------------- GEMM
-constexpr int kTcThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
+// One persistent CTA per SM walks a contiguous range of work items (KV head
+// g, 128-row M tile), head-major, so W_app,g is staged once per head and
+// stays resident while the v/k tiles stream through a ring of 16 KB slots.
+// The accumulator is double-buffered in tensor memory: the MMA of tile i+1
+// runs while the epilogue drains tile i.  The epilogue moves no cache bytes
+// through registers one lane per row: each lane converts its row into a
+// shared-memory staging row and hands it to the copy engine (one bulk copy
+// per cache part).  A seventh warp copies the exact Key out of each k slot
+// as soon as it lands: 8-row TMA tensor stores wherever 8 rows land on 8
+// consecutive cache rows (every group of an aligned chunk; a ragged group
+// falls back to plain stores), so a slot returns to the producer once its
+// MMAs are done and the copy engine has read it, and the ring keeps
+// streaming while the epilogue works.
+// warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue, warp 6 Key copy
+constexpr int kTcThreads = 224;
+constexpr int kTcEpiWarps = 4;
+constexpr int kTcKeyWarp = 6;
 constexpr int kTcBM = 128, kTcBK = 64;
-constexpr int kTcSlots = 2;  // k-block ring
+constexpr int kTcABytes = kTcBM * kTcBK * 2;  // one ring slot: 128 rows x 128 bytes
+constexpr int kTcMaxSlots = 12;
+constexpr unsigned long long kTcDrainNs = 10000000ull;  // waits for copies in flight at exit
 
 __host__ __device__ constexpr uint32_t tc_idesc(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
@@ -127,29 +145,107 @@ __device__ __forceinline__ uint64_t tc_sdesc(uint32_t saddr) {
   return d;
 }
 
+// Staging row: z | e in the cache element type.  Its stride in 16-byte
+// chunks is rounded up to an odd count, so that eight consecutive rows start
+// in eight different bank groups (one row per lane writes without
+// conflicts).
+__host__ __device__ constexpr int tc_stage_stride(int N, int fp8) {
+  return ((fp8 ? N : 2 * N) / 16) | 1;
+}
+
+struct TcSmem {
+  size_t w, ring, stage, ktab, bars, total;
+};
+
+__host__ __device__ inline TcSmem tc_smem(int N, int d, int fp8, int slots) {
+  TcSmem L;
+  L.w = 0;                                           // nkb tiles of N x 128 bytes
+  L.ring = (size_t)N * 2 * d * 2;                    // a multiple of 2 KB
+  L.stage = L.ring + (size_t)slots * kTcABytes;
+  L.ktab = L.stage + (size_t)kTcEpiWarps * 32 * tc_stage_stride(N, fp8) * 16;
+  L.bars = L.ktab + kTcBM * 8;  // the Key warp's cache row per tile row
+  L.total = L.bars + (2 * (size_t)slots + 7) * 8 + 16;
+  return L;
+}
+
+// shared -> global bulk copy (16-byte aligned ends, size % 16 == 0)
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+
+// 2-D tiled store of one box from shared memory (bulk group)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int32_t x,
+                                             int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// this thread's bulk copies have read their shared-memory sources
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// this thread's bulk copies are complete
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1)
     append_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmW, AppendArgs a, int N, int tmem_cols) {
+                     const __grid_constant__ CUtensorMap tmW,
+                     const __grid_constant__ CUtensorMap tmKc, AppendArgs a, int N, int tmem_cols,
+                     int slots, int n_mt) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1k(smem_raw);
   const int d = a.d, nkb = 2 * d / kTcBK;  // k-blocks: first d/64 from v, then from k
-  const int a_bytes = kTcBM * kTcBK * 2, b_bytes = N * kTcBK * 2;
-  uint8_t* a_tiles = smem;                           // kTcSlots x 16 KB
-  uint8_t* b_tiles = smem + kTcSlots * a_bytes;      // kTcSlots x N*128 B
-  uint64_t* full = reinterpret_cast<uint64_t*>(b_tiles + kTcSlots * b_bytes);
-  uint64_t* empty = full + kTcSlots;
-  uint64_t* accum = empty + kTcSlots;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  const int cb = a.fp8 ? 1 : 2;            // cache bytes per element
+  const TcSmem L = tc_smem(N, d, a.fp8, slots);
+  uint8_t* w_tiles = smem + L.w;
+  uint8_t* ring = smem + L.ring;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* empty = full + slots;
+  uint64_t* tfull = empty + slots;  // [2] accumulator buffer written
+  uint64_t* tempty = tfull + 2;     // [2] accumulator buffer drained
+  uint64_t* wfull = tempty + 2;
+  uint64_t* wempty = wfull + 1;
+  uint64_t* drain = wempty + 1;  // the MMA thread's last commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = blockIdx.y, m0 = blockIdx.x * kTcBM;
   const int rows = a.B * a.n_new;
+  const int n_items = n_mt * a.Hkv;
+  const int i0 = (int)((long long)blockIdx.x * n_items / gridDim.x);
+  const int i1 = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
+  const int acc_cols = tmem_cols / 2;
 
   if (tid == 0) {
-    for (int s = 0; s < kTcSlots; ++s) {
+    for (int s = 0; s < slots; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 2);  // the MMAs' commit + the Key warp's release (v slots: a stand-in)
     }
-    mbar_init(accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kTcEpiWarps);
+    }
+    mbar_init(wfull, 1);
+    mbar_init(wempty, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -169,155 +265,242 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmW);
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % kTcSlots;
-      // the slot is free once the MMAs that read its previous k-block are done
-      if (kb >= kTcSlots && !mbar_wait(&empty[s], ((kb / kTcSlots) - 1) & 1, a.status)) break;
-      mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
-      const bool from_v = kb < nkb / 2;
-      const int col = (from_v ? kb : kb - nkb / 2) * kTcBK;
-      // 3-D maps over [rows][Hkv][d]: coordinates (column, head, row)
-      tma_load_3d(a_tiles + s * a_bytes, from_v ? &tmV : &tmK, col, g, m0, &full[s]);
-      tma_load_2d(b_tiles + s * b_bytes, &tmW, kb * kTcBK, g * N, &full[s]);
+    if (!a.fp8) prefetch_tmap(&tmKc);
+    int it = 0, wl = 0, cur_g = -1;
+    bool ok = true;
+    for (int item = i0; item < i1 && ok; ++item) {
+      const int g = item / n_mt, m0 = (item % n_mt) * kTcBM;
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % slots;
+        // the slot is free once its previous k-block has been consumed
+        if (it >= slots && !(ok = mbar_wait_or_abort(&empty[s], ((it / slots) - 1) & 1,
+                                                     a.status, abort_flag)))
+          break;
+        mbar_arrive_expect_tx(&full[s], kTcABytes);
+        const bool from_v = kb < nkb / 2;
+        const int col = (from_v ? kb : kb - nkb / 2) * kTcBK;
+        // 3-D maps over [rows][Hkv][d]: coordinates (column, head, row)
+        tma_load_3d(ring + s * kTcABytes, from_v ? &tmV : &tmK, col, g, m0, &full[s]);
+      }
+      if (ok && g != cur_g) {  // a new head: its factor, once the last MMA on the old one is done
+        if (wl > 0 && !(ok = mbar_wait_or_abort(wempty, (wl - 1) & 1, a.status, abort_flag)))
+          break;
+        mbar_arrive_expect_tx(wfull, (uint32_t)N * 2 * d * 2);
+        for (int kb = 0; kb < nkb; ++kb)
+          tma_load_2d(w_tiles + kb * N * 128, &tmW, kb * kTcBK, g * N, wfull);
+        ++wl;
+        cur_g = g;
+      }
     }
+    // drain: every copy issued must have landed before the CTA exits
+    for (int u = it - 1; u >= 0 && u >= it - slots; --u)
+      mbar_wait(&full[u % slots], (u / slots) & 1, a.status, kTcDrainNs);
+    if (wl > 0) mbar_wait(wfull, (wl - 1) & 1, a.status, kTcDrainNs);
   } else if (warp == 1 && lane == 0) {  // ------------------------------ MMA
     const uint32_t idesc = tc_idesc(kTcBM, N);
+    int it = 0, wl = 0, cur_g = -1, lt = 0;
     bool ok = true;
-    for (int kb = 0; kb < nkb && ok; ++kb) {
-      const int s = kb % kTcSlots;
-      ok = mbar_wait(&full[s], (kb / kTcSlots) & 1, a.status);
-      if (!ok) break;
+    for (int item = i0; item < i1 && ok; ++item, ++lt) {
+      const int g = item / n_mt;
+      if (g != cur_g) {
+        if (!(ok = mbar_wait_or_abort(wfull, wl & 1, a.status, abort_flag))) break;
+        ++wl;
+        cur_g = g;
+      }
+      const int buf = lt & 1;
+      if (lt >= 2 && !(ok = mbar_wait_or_abort(&tempty[buf], ((lt >> 1) - 1) & 1, a.status,
+                                               abort_flag)))
+        break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint64_t da = tc_sdesc(smem_u32(a_tiles + s * a_bytes));
-      const uint64_t db = tc_sdesc(smem_u32(b_tiles + s * b_bytes));
+      const uint32_t dt = tmem + (uint32_t)(buf * acc_cols);
+      for (int kb = 0; kb < nkb; ++kb, ++it) {
+        const int s = it % slots;
+        if (!(ok = mbar_wait_or_abort(&full[s], (it / slots) & 1, a.status, abort_flag))) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint64_t da = tc_sdesc(smem_u32(ring + s * kTcABytes));
+        const uint64_t db = tc_sdesc(smem_u32(w_tiles + kb * N * 128));
 #pragma unroll
-      for (int k = 0; k < kTcBK / 16; ++k) {
-        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-        asm volatile(
-            "{ .reg .pred p; setp.ne.b32 p, %4, 0;"
-            " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem),
-            "l"(da + 2 * k), "l"(db + 2 * k), "r"(idesc), "r"(acc)
-            : "memory");
+        for (int k = 0; k < kTcBK / 16; ++k) {
+          const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+          asm volatile(
+              "{ .reg .pred p; setp.ne.b32 p, %4, 0;"
+              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(dt),
+              "l"(da + 2 * k), "l"(db + 2 * k), "r"(idesc), "r"(acc)
+              : "memory");
+        }
+        // slot s is released when these MMAs complete (and, for a k slot,
+        // once the Key warp has copied it out)
+        tc_commit(&empty[s]);
+        if (kb < nkb / 2) mbar_arrive(&empty[s]);
       }
-      // slot s is released when these MMAs complete
-      asm volatile(
-          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-              smem_u32(&empty[s]))
-          : "memory");
+      if (!ok) break;
+      tc_commit(&tfull[buf]);
+      if (item + 1 < i1 && (item + 1) / n_mt != g) tc_commit(wempty);
     }
-    if (ok)
-      asm volatile(
-          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-              smem_u32(accum))
-          : "memory");
-  } else if (warp >= 2) {  // ---------------------------------------- epilogue
-    const int quarter = warp & 3;
-    const int r = m0 + quarter * 32 + lane;  // token row of the chunk
-    bool ok = mbar_wait(accum, 0, a.status);
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    size_t slot = 0;
-    bool live = false;
-    if (r < rows) {
-      const int b = r / a.n_new, j = r % a.n_new;
-      const int len = a.seq_lens[b];
-      const int cap = a.max_pages * a.S;
-      if (len < 0 || len + a.n_new > cap) {
-        if (j == 0 && g == 0) raise_status(a.status, BASISKV_DEV_OVERFLOW);
-      } else {
-        const int pos = len + j;
-        const int pp = a.block_table[(size_t)b * a.max_pages + pos / a.S];
-        if (pp < 0 || pp >= a.num_phys) {
-          raise_status(a.status, BASISKV_DEV_BAD_PAGE);
+    // drain: one more commit tracks every MMA this thread issued
+    tc_commit(drain);
+    mbar_wait(drain, 0, a.status, kTcDrainNs);
+  } else if (warp >= 2 && warp < 2 + kTcEpiWarps) {  // ------------------- epilogue
+    const int quarter = warp & 3;  // this warp's 32 TMEM lanes = tile rows
+    uint4* my = reinterpret_cast<uint4*>(smem + L.stage) +
+                ((size_t)(warp - 2) * 32 + lane) * tc_stage_stride(N, a.fp8);  // this lane's row
+    const int zs = a.zsplit, es = a.esplit;
+    uint8_t* const zc = reinterpret_cast<uint8_t*>(a.Z_cache);
+    uint8_t* const ec = reinterpret_cast<uint8_t*>(a.E_cache);
+    int lt = 0;
+    for (int item = i0; item < i1; ++item, ++lt) {
+      const int g = item / n_mt, m0 = (item % n_mt) * kTcBM;
+      // this lane's row: its cache tile (physical page x KV head) and row
+      // within the tile, or dead
+      const int r = m0 + quarter * 32 + lane;
+      long long tile = 0;
+      int trow = 0, live = 0;
+      if (r < rows) {
+        const int b = r / a.n_new, j = r % a.n_new;
+        const int len = a.seq_lens[b];
+        const int cap = a.max_pages * a.S;
+        if (len < 0 || len + a.n_new > cap) {
+          if (j == 0 && g == 0) raise_status(a.status, BASISKV_DEV_OVERFLOW);
         } else {
-          slot = ((size_t)pp * a.Hkv + g) * a.S + pos % a.S;
-          live = true;
-        }
-      }
-    }
-    // every lane of the warp joins the tcgen05.ld; only live rows store
-    for (int c0 = 0; c0 < N; c0 += 16) {
-      float v[16];
-      uint32_t rr[16];
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-          "%11, %12, %13, %14, %15}, [%16];"
-          : "=r"(rr[0]), "=r"(rr[1]), "=r"(rr[2]), "=r"(rr[3]), "=r"(rr[4]), "=r"(rr[5]),
-            "=r"(rr[6]), "=r"(rr[7]), "=r"(rr[8]), "=r"(rr[9]), "=r"(rr[10]), "=r"(rr[11]),
-            "=r"(rr[12]), "=r"(rr[13]), "=r"(rr[14]), "=r"(rr[15])
-          : "r"(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c0));
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-      if (!(ok && live)) continue;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(rr[i]);
-      const size_t tile = slot / a.S;
-      const int trow = (int)(slot - tile * a.S);
-      if (a.fp8) {  // E4M3 caches: 16 bytes per 16 columns
-        uint32_t pb[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          pb[i] = f_to_e4m3x2(v[4 * i], v[4 * i + 1]) |
-                  (f_to_e4m3x2(v[4 * i + 2], v[4 * i + 3]) << 16);
-        uint8_t* dst8 =
-            c0 < a.r_v
-                ? reinterpret_cast<uint8_t*>(a.Z_cache) + tile * a.S * a.r_v +
-                      split_off(trow, c0, a.S, a.r_v, a.zsplit)
-                : reinterpret_cast<uint8_t*>(a.E_cache) + tile * a.S * a.r_k +
-                      split_off(trow, c0 - a.r_v, a.S, a.r_k, a.esplit);
-        *reinterpret_cast<uint4*>(dst8) = make_uint4(pb[0], pb[1], pb[2], pb[3]);
-        continue;
-      }
-      uint32_t pk[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        pk[i] = (uint32_t)f_to_bf16(v[2 * i]) | ((uint32_t)f_to_bf16(v[2 * i + 1]) << 16);
-      // columns c0..c0+15 are z (c < r_v) or e (c >= r_v); r_v, r_k are multiples of 16
-      uint16_t* dst =
-          c0 < a.r_v
-              ? a.Z_cache + tile * a.S * a.r_v + split_off(trow, c0, a.S, a.r_v, a.zsplit)
-              : a.E_cache + tile * a.S * a.r_k +
-                    split_off(trow, c0 - a.r_v, a.S, a.r_k, a.esplit);
-      uint4* d4 = reinterpret_cast<uint4*>(dst);
-      d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-    }
-    if (ok && live) {  // the exact Key, copied as is (E4M3: rounded)
-      // The row is still in shared memory: the last d/64 k-blocks staged for
-      // the product are the Key's columns (128-byte rows, 16-byte chunk j of
-      // row t stored at chunk j ^ (t & 7)).
-      const int t = quarter * 32 + lane;
-      // acquire the staged tiles' TMA writes (their last phases are complete)
-      bool kok = true;
-      for (int kb = nkb / 2; kb < nkb; ++kb)
-        kok = kok && mbar_wait(&full[kb % kTcSlots], (kb / kTcSlots) & 1, a.status);
-      uint4 kr[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        if (i < d / 8) {
-          const int kb = nkb / 2 + i / 8;  // the k-block of columns 8i .. 8i + 7
-          const uint8_t* tile = a_tiles + (kb % kTcSlots) * a_bytes;
-          kr[i] = *reinterpret_cast<const uint4*>(tile + t * 128 + (((i & 7) ^ (t & 7)) << 4));
-        }
-      }
-      if (!kok) {
-      } else if (a.fp8) {
-        uint2* dstk = reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(a.K_cache) + slot * d);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (i < d / 8) {
-            const uint4 x = kr[i];
-            const float2 f0 = bf16x2_to_f2(x.x), f1 = bf16x2_to_f2(x.y), f2 = bf16x2_to_f2(x.z),
-                         f3 = bf16x2_to_f2(x.w);
-            dstk[i] = make_uint2(f_to_e4m3x2(f0.x, f0.y) | (f_to_e4m3x2(f1.x, f1.y) << 16),
-                                 f_to_e4m3x2(f2.x, f2.y) | (f_to_e4m3x2(f3.x, f3.y) << 16));
+          const int pos = len + j;
+          const int pp = a.block_table[(size_t)b * a.max_pages + pos / a.S];
+          if (pp < 0 || pp >= a.num_phys) {
+            raise_status(a.status, BASISKV_DEV_BAD_PAGE);
+          } else {
+            tile = (long long)pp * a.Hkv + g;
+            trow = pos % a.S;
+            live = 1;
           }
         }
-      } else {
-        uint4* dstk = reinterpret_cast<uint4*>(a.K_cache + slot * d);
+      }
+      const int buf = lt & 1;
+      bool ok = mbar_wait_or_abort(&tfull[buf], (lt >> 1) & 1, a.status, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      // accumulator -> cache element type -> this lane's staging row
+      const uint32_t ta = tmem + (uint32_t)(buf * acc_cols) + ((uint32_t)(quarter * 32) << 16);
+      for (int c0 = 0; c0 < N; c0 += 16) {
+        uint32_t rr[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
+            "%10, %11, %12, %13, %14, %15}, [%16];"
+            : "=r"(rr[0]), "=r"(rr[1]), "=r"(rr[2]), "=r"(rr[3]), "=r"(rr[4]), "=r"(rr[5]),
+              "=r"(rr[6]), "=r"(rr[7]), "=r"(rr[8]), "=r"(rr[9]), "=r"(rr[10]), "=r"(rr[11]),
+              "=r"(rr[12]), "=r"(rr[13]), "=r"(rr[14]), "=r"(rr[15])
+            : "r"(ta + (uint32_t)c0));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        float v[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (i < d / 8) dstk[i] = kr[i];
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(rr[i]);
+        if (a.fp8) {  // E4M3: 16 columns are one chunk
+          uint32_t pb[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            pb[i] = f_to_e4m3x2(v[4 * i], v[4 * i + 1]) |
+                    (f_to_e4m3x2(v[4 * i + 2], v[4 * i + 3]) << 16);
+          my[c0 / 16] = make_uint4(pb[0], pb[1], pb[2], pb[3]);
+        } else {
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            pk[i] = (uint32_t)f_to_bf16(v[2 * i]) | ((uint32_t)f_to_bf16(v[2 * i + 1]) << 16);
+          my[c0 / 8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          my[c0 / 8 + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+      // the accumulator buffer is free for the MMA two tiles on
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (live) {
+        // the staging row's parts go to their caches (Z and E tiles store
+        // the first zsplit / esplit columns of every row first)
+        fence_proxy_async();
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(my);
+        const size_t zt = (size_t)tile * a.S * a.r_v * cb, et = (size_t)tile * a.S * a.r_k * cb;
+        bulk_store(zc + zt + (size_t)trow * zs * cb, src, zs * cb);
+        if (zs < a.r_v)
+          bulk_store(zc + zt + ((size_t)a.S * zs + (size_t)trow * (a.r_v - zs)) * cb,
+                     src + zs * cb, (a.r_v - zs) * cb);
+        bulk_store(ec + et + (size_t)trow * es * cb, src + a.r_v * cb, es * cb);
+        if (es < a.r_k)
+          bulk_store(ec + et + ((size_t)a.S * es + (size_t)trow * (a.r_k - es)) * cb,
+                     src + (a.r_v + es) * cb, (a.r_k - es) * cb);
+      }
+      // the staging row is rewritten next tile, once the copy engine has read it
+      bulk_commit();
+      bulk_wait_read();
+    }
+    bulk_wait_all();
+  } else if (warp == kTcKeyWarp) {  // --------------------------------- Key copy
+    // The exact Key, straight from each k slot (16-byte chunk j of tile row t
+    // sits at chunk j ^ (t & 7) of its 128-byte row).  tab[t] = the Key
+    // cache row of tile row t, or -1 for a dead row.
+    long long* tab = reinterpret_cast<long long*>(smem + L.ktab);
+    uint8_t* const kc = reinterpret_cast<uint8_t*>(a.K_cache);
+    int lt = 0;
+    bool ok = true;
+    for (int item = i0; item < i1 && ok; ++item, ++lt) {
+      const int g = item / n_mt, m0 = (item % n_mt) * kTcBM;
+      __syncwarp();  // the previous tile's reads of tab are done
+      for (int i = 0; i < kTcBM / 32; ++i) {
+        const int t = lane + 32 * i, r = m0 + t;
+        long long sl = -1;
+        if (r < rows) {
+          const int b = r / a.n_new, j = r % a.n_new;
+          const int len = a.seq_lens[b];
+          if (len >= 0 && len + a.n_new <= a.max_pages * a.S) {
+            const int pos = len + j;
+            const int pp = a.block_table[(size_t)b * a.max_pages + pos / a.S];
+            if (pp >= 0 && pp < a.num_phys) sl = ((long long)pp * a.Hkv + g) * a.S + pos % a.S;
+          }
+        }
+        tab[t] = sl;
+      }
+      __syncwarp();
+      // lane j < 16: do the 8 rows of group j land on 8 consecutive cache rows?
+      bool boxed = false;
+      if (!a.fp8 && lane < kTcBM / 8) {
+        const long long s0 = tab[8 * lane];
+        boxed = s0 >= 0;
+        for (int i = 1; i < 8; ++i) boxed = boxed && tab[8 * lane + i] == s0 + i;
+      }
+      const unsigned bmask = __ballot_sync(0xffffffffu, boxed);
+      for (int kb = 0; kb < nkb / 2; ++kb) {
+        const int u = lt * nkb + nkb / 2 + kb, s = u % slots;
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait_or_abort(&full[s], (u / slots) & 1, a.status, abort_flag));
+        if (!ok) break;
+        const uint8_t* stage = ring + (size_t)s * kTcABytes;
+        if (boxed) tma_store_2d(&tmKc, stage + lane * 8 * 128, kb * kTcBK, (int32_t)tab[8 * lane]);
+        if (bmask != (1u << (kTcBM / 8)) - 1) {
+          // the other rows, four per pass, eight lanes on a row's chunks
+          for (int p = 0; p < kTcBM / 4; ++p) {
+            const int t = p * 4 + (lane >> 3), ch = lane & 7;
+            const long long sl = tab[t];
+            if (((bmask >> (t >> 3)) & 1u) || sl < 0) continue;
+            const uint4 x =
+                *reinterpret_cast<const uint4*>(stage + t * 128 + ((ch ^ (t & 7)) << 4));
+            if (a.fp8) {
+              const float2 f0 = bf16x2_to_f2(x.x), f1 = bf16x2_to_f2(x.y),
+                           f2 = bf16x2_to_f2(x.z), f3 = bf16x2_to_f2(x.w);
+              *reinterpret_cast<uint2*>(kc + sl * d + kb * kTcBK + ch * 8) =
+                  make_uint2(f_to_e4m3x2(f0.x, f0.y) | (f_to_e4m3x2(f1.x, f1.y) << 16),
+                             f_to_e4m3x2(f2.x, f2.y) | (f_to_e4m3x2(f3.x, f3.y) << 16));
+            } else {
+              *reinterpret_cast<uint4*>(kc + (sl * d + kb * kTcBK + ch * 8) * 2) = x;
+            }
+          }
+        }
+        // the slot goes back to the producer once the copy engine has read it
+        bulk_commit();
+        bulk_wait_read();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
       }
     }
+    bulk_wait_all();
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -349,20 +532,25 @@ cudaError_t launch_fold_append(const FoldAppArgs& a, cudaStream_t st, bool pdl) 
 }
 
 cudaError_t launch_append_tc(const AppendArgs& a, const CUtensorMap& tmV, const CUtensorMap& tmK,
-                             const CUtensorMap& tmW, cudaStream_t st, bool pdl) {
+                             const CUtensorMap& tmW, const CUtensorMap& tmKc, cudaStream_t st,
+                             bool pdl) {
   const int N = a.r_v + a.r_k;
-  const int tmem_cols = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
-  size_t smem = (size_t)kTcSlots * (kTcBM * kTcBK * 2 + N * kTcBK * 2) + 64 + 1024;
-  // At most 512 / tmem_cols CTAs per SM may hold tensor memory at once: with
-  // 256 columns keep it to two by shared memory (three would need <= 75 KB).
-  if (tmem_cols > 128 && smem < 76 * 1024) smem = 76 * 1024;
+  const int acc = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
+  const int tmem_cols = 2 * acc;  // two accumulator buffers
+  const int nkb = 2 * a.d / kTcBK;
+  const size_t cap = 227 * 1024 - 1024;  // the 1 KB alignment pad comes off the top
+  const size_t fixed = tc_smem(N, a.d, a.fp8, 0).total;
+  if (fixed + (size_t)nkb * kTcABytes > cap) return cudaErrorInvalidConfiguration;
+  const int slots = (int)std::min<size_t>(kTcMaxSlots, (cap - fixed) / kTcABytes);
+  const size_t smem = tc_smem(N, a.d, a.fp8, slots).total + 1024;
   cudaError_t e = cudaFuncSetAttribute(append_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int rows = a.B * a.n_new;
-  dim3 grid((rows + kTcBM - 1) / kTcBM, a.Hkv);
-  return launch_k(append_tc_kernel, grid, dim3(kTcThreads), smem, st, pdl, tmV, tmK, tmW, a, N,
-                  tmem_cols);
+  const int n_mt = (rows + kTcBM - 1) / kTcBM;
+  const int grid = std::min(n_mt * a.Hkv, num_sms());
+  return launch_k(append_tc_kernel, dim3(grid), dim3(kTcThreads), smem, st, pdl, tmV, tmK, tmW,
+                  tmKc, a, N, tmem_cols, slots, n_mt);
 }
 
 }  // namespace basiskv

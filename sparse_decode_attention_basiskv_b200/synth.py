@@ -371,7 +371,7 @@ def make_tokens(wl: Workload, factors: dict, n: int, device="cpu",
     lat = torch.einsum("bnhd,hdr->bnhr", v.float(), A_V)
     k = (torch.einsum("bnhr,hrd->bnhd", lat, P_K)
          + torch.einsum("bnhr,hdr->bnhd", ep, U_K) + noise)
-    return k.bfloat16(), v
+    return k.bfloat16().contiguous(), v
 
 
 def block_table(wl: Workload, device="cpu") -> torch.Tensor:

@@ -274,3 +274,14 @@ def test_route_page_validation(lib):
     a = lib.basiskv_attend(ctypes.byref(ok), FAKE, FAKE, 1024, FAKE, FAKE, FAKE, FAKE, 64, FAKE,
                            FAKE, 1 << 20, None)
     assert a == bkv.ERR_UNSUPPORTED_SHAPE
+
+
+def test_binding_refuses_strided_tensors():
+    """The library reads every array as dense row-major memory: the binding
+    refuses a strided view instead of passing its base address."""
+    import torch
+    strided = torch.zeros(4, 6)[:, ::2]
+    with pytest.raises(ValueError, match="not contiguous"):
+        bkv._ptr(strided)
+    dense = torch.zeros(4, 6)
+    assert bkv._ptr(dense) == dense.data_ptr() and bkv._ptr(None) is None

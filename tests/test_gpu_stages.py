@@ -10,7 +10,8 @@ from oracle import basiskv_oracle as O
 from sparse_decode_attention_basiskv_b200 import synth
 from sparse_decode_attention_basiskv_b200.layer import DecodeLayer
 
-from harness import (A_REL, S_REL, Y_ABS, Y_REL, ZE_REL, assert_within, cache_row,
+from harness import (A_REL, S_REL, Y_ABS, Y_REL, ZE_REL, assert_e4m3_bracket, assert_within,
+                     cache_row,
                      StepChecker,
                      factors_np, gpu_layer, np64, oracle_route, status_clean)
 
@@ -278,6 +279,69 @@ def test_prefill_chunk_append(prefolded):
         assert_within(np64(cache_row(layer.Z, wl, "Z", phys, g, rows)), z_ref, ZE_REL, what="prefill z")
         assert_within(np64(cache_row(layer.E, wl, "E", phys, g, rows)), e_ref, ZE_REL, what="prefill e")
         assert torch.equal(layer.K[phys, g, rows], k[b, :, g])
+
+
+# Sequences of different lengths take one chunk each in one call:
+# (workload, starting lengths).
+RAGGED_PREFILL = {
+    "qwen": (synth.with_sizes(synth.QWEN32B_T64K_B8, B=3, T=160, prefill_tokens=200),
+             [5, 37, 131]),
+    # the narrow router's split tiles (16 latent + 16 residual columns first)
+    "llama_b16r16": (synth.with_sizes(synth.LLAMA8B_T32K_B16_B16R16, B=3, T=160, top_k=8,
+                                      prefill_tokens=200), [5, 37, 131]),
+    "qwen_e4m3": (synth.with_sizes(synth.QWEN32B_T64K_B8, B=3, T=160, prefill_tokens=200,
+                                   cache_fp8=1), [5, 37, 131]),
+    # the benchmarked launch: eight 4096-token chunks, 2048 (head, M tile)
+    # items over the SMs, so every CTA runs many items and reloads W_app
+    "qwen_b8_4096": (synth.with_sizes(synth.QWEN32B_T64K_B8, B=8, T=160, prefill_tokens=4096),
+                     [96, 101, 3, 64, 77, 32, 0, 159]),
+}
+
+
+@pytest.mark.parametrize("name", list(RAGGED_PREFILL))
+def test_prefill_append_ragged_rows(name):
+    """Sequences at ragged lengths (5, 37 and 131, say) take a chunk each
+    in one tensor-core call (200 tokens: 600 token rows), so M tiles
+    straddle sequences and start pages at odd offsets, and the last tile is
+    partial.  Every appended row matches the oracle, and no other cache row
+    changes."""
+    wl, lens0 = RAGGED_PREFILL[name]
+    n = wl.prefill_tokens
+    pb, layer = gpu_layer(wl, seq_lens=lens0)
+    f = factors_np(pb)
+    k, v = synth.make_tokens(wl, pb.factors, n, device="cuda", stream_id=7)
+    before = {nm: t.clone() for nm, t in (("K", layer.K), ("Z", layer.Z), ("E", layer.E))}
+    layer.append(k, v, n)
+    status_clean()
+    assert layer.seq_lens.tolist() == [x + n for x in lens0]
+    fp8 = bool(wl.cache_fp8)
+    touched = torch.zeros(layer.K.shape[:3], dtype=torch.bool)  # [phys][Hkv][page row]
+    for b, L0 in enumerate(lens0):
+        toks = np.arange(L0, L0 + n)
+        phys = layer.block_table[b, toks // wl.page_size].long().cpu()
+        rows = torch.as_tensor(toks % wl.page_size)
+        touched[phys, :, rows] = True
+        for g in range(wl.Hkv):
+            z_ref, e_ref = O.append_latents(np64(k[b, :, g]), np64(v[b, :, g]), f["A_V"][g],
+                                            f["P_K"][g], f["U_K"][g])
+            z = np64(cache_row(layer.Z, wl, "Z", phys, g, rows))
+            e = np64(cache_row(layer.E, wl, "E", phys, g, rows))
+            if fp8:
+                assert_e4m3_bracket(z, z_ref, ZE_REL * np.abs(z_ref).max(), what=f"z b{b} g{g}")
+                assert_e4m3_bracket(e, e_ref, ZE_REL * np.abs(e_ref).max(), what=f"e b{b} g{g}")
+                kb = layer.K.view(torch.uint8)[phys, g, rows].view(torch.float8_e4m3fn).float()
+                np.testing.assert_array_equal(np64(kb), O.to_e4m3(np64(k[b, :, g])))
+            else:
+                assert_within(z, z_ref, ZE_REL, what=f"z b{b} g{g}")
+                assert_within(e, e_ref, ZE_REL, what=f"e b{b} g{g}")
+                assert torch.equal(layer.K[phys, g, rows], k[b, :, g])
+    keep = ~touched.to(layer.K.device)
+    lead = wl.tile_lead()
+    for nm, t in (("K", layer.K), ("Z", layer.Z), ("E", layer.E)):
+        now, old = t.view(torch.uint8) if fp8 else t, before[nm].view(torch.uint8) if fp8 else before[nm]
+        if nm != "K":
+            now, old = synth.unsplit_tiles(now, lead[nm]), synth.unsplit_tiles(old, lead[nm])
+        assert torch.equal(now[keep], old[keep]), f"{nm}: a row outside the appended tokens changed"
 
 
 def test_device_status_reports_bad_inputs():
