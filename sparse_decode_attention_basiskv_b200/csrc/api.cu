@@ -324,11 +324,13 @@ int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_b
     const uint64_t dims3[3] = {(uint64_t)d->d, (uint64_t)d->Hkv, rows};
     const uint64_t str3[2] = {(uint64_t)d->d * 2, (uint64_t)d->Hkv * d->d * 2};
     const uint32_t box3[3] = {64, 1, 128};
-    CUtensorMap tmV, tmK, tmW, tmKc;
+    CUtensorMap tmV, tmK, tmW, tmWk, tmKc;
     if (!make_tmap_3d(&tmV, v_new, dims3, str3, box3, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_3d(&tmK, k_new, dims3, str3, box3, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tmap_2d(&tmW, w_app, (uint64_t)d->Hkv * N, 2 * d->d, (uint64_t)4 * d->d, N, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
+                      CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tmap_2d(&tmWk, w_app, (uint64_t)d->Hkv * N, 2 * d->d, (uint64_t)4 * d->d, d->r_k,
+                      64, CU_TENSOR_MAP_SWIZZLE_128B))
       return BASISKV_ERR_CUDA;
     if (d->cache_fp8) {
       tmKc = tmK;  // not read: E4M3 Key rows leave through the staging rows
@@ -337,7 +339,7 @@ int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_b
                              (uint64_t)d->d * 2, 8, 64, CU_TENSOR_MAP_SWIZZLE_128B)) {
       return BASISKV_ERR_CUDA;
     }
-    rc = launch_status(launch_append_tc(a, tmV, tmK, tmW, tmKc, st, pdl));
+    rc = launch_status(launch_append_tc(a, tmV, tmK, tmW, tmWk, tmKc, st, pdl));
   } else {
     rc = launch_status(launch_append_small(a, st, pdl));
   }

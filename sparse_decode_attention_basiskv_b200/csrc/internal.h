@@ -62,11 +62,13 @@ size_t append_factor_bytes(int Hkv, int d, int r_v, int r_k);
 cudaError_t launch_fold_append(const FoldAppArgs& a, cudaStream_t st, bool pdl);
 // tmV, tmK: 3-D maps over [rows][Hkv][d] (box 64 x 1 x 128); tmW: 2-D map over
 // [Hkv*(r_v+r_k)][2d] (box (r_v+r_k) x 64); all with 128-byte swizzle.
-// tmKc: the bf16 Key cache as [num_phys * Hkv * S][d] (box 8 x 64, 128-byte
-// swizzle), the target of the Key's TMA stores (unused for E4M3 caches).
+// tmWk: the same W_app map with a box of r_k rows (the residual rows of the
+// k k-blocks).  tmKc: the bf16 Key cache as [num_phys * Hkv * S][d] (box
+// 8 x 64, 128-byte swizzle), the target of the Key's TMA stores (unused for
+// E4M3 caches).
 cudaError_t launch_append_tc(const AppendArgs& a, const CUtensorMap& tmV, const CUtensorMap& tmK,
-                             const CUtensorMap& tmW, const CUtensorMap& tmKc, cudaStream_t st,
-                             bool pdl);
+                             const CUtensorMap& tmW, const CUtensorMap& tmWk,
+                             const CUtensorMap& tmKc, cudaStream_t st, bool pdl);
 cudaError_t launch_bump_lengths(const AppendArgs& a, cudaStream_t st, bool pdl);
 
 // ------------------------------------------------------------------- route

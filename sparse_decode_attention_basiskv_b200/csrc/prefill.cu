@@ -111,20 +111,22 @@ __global__ void __launch_bounds__(kFoldAppThreads) fold_append_kernel(FoldAppArg
 // One persistent CTA per SM walks a contiguous range of work items (KV head
 // g, 128-row M tile), head-major, so W_app,g is staged once per head and
 // stays resident while the v/k tiles stream through a ring of 16 KB slots.
-// The accumulator is double-buffered in tensor memory: the MMA of tile i+1
-// runs while the epilogue drains tile i.  The epilogue moves no cache bytes
-// through registers one lane per row: each lane converts its row into a
-// shared-memory staging row and hands it to the copy engine (one bulk copy
-// per cache part).  A seventh warp copies the exact Key out of each k slot
-// as soon as it lands: 8-row TMA tensor stores wherever 8 rows land on 8
-// consecutive cache rows (every group of an aligned chunk; a ragged group
-// falls back to plain stores), so a slot returns to the producer once its
-// MMAs are done and the copy engine has read it, and the ring keeps
-// streaming while the epilogue works.
-// warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue, warp 6 Key copy
-constexpr int kTcThreads = 224;
-constexpr int kTcEpiWarps = 4;
-constexpr int kTcKeyWarp = 6;
+// Only W_app's nonzero blocks are staged: the v k-blocks multiply all N
+// rows, the k k-blocks only the r_k residual rows (N = r_k, into the
+// accumulator's e columns).  The accumulator is double-buffered in tensor
+// memory: the MMA of tile i+1 runs while the epilogue drains tile i.  The
+// epilogue converts each lane's row into dense per-part staging blocks and
+// hands every run of consecutive cache rows to the copy engine as one bulk
+// copy per cache part.  Four more warps copy the exact Key out of each k
+// slot as soon as it lands: 8-row TMA tensor stores wherever 8 rows land on
+// 8 consecutive cache rows (every group of an aligned chunk; a ragged group,
+// and E4M3 rounding, fall back to plain stores), so a slot returns to the
+// producer once its MMAs are done and the copy engine has read it, and the
+// ring keeps streaming while the epilogue works.
+// warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue, warps 6-9 Key copy
+constexpr int kTcEpiWarps = 4, kTcKeyWarps = 4;
+constexpr int kTcKeyWarp0 = 2 + kTcEpiWarps;
+constexpr int kTcThreads = 32 * (kTcKeyWarp0 + kTcKeyWarps);
 constexpr int kTcBM = 128, kTcBK = 64;
 constexpr int kTcABytes = kTcBM * kTcBK * 2;  // one ring slot: 128 rows x 128 bytes
 constexpr int kTcMaxSlots = 12;
@@ -145,27 +147,30 @@ __device__ __forceinline__ uint64_t tc_sdesc(uint32_t saddr) {
   return d;
 }
 
-// Staging row: z | e in the cache element type.  Its stride in 16-byte
-// chunks is rounded up to an odd count, so that eight consecutive rows start
-// in eight different bank groups (one row per lane writes without
-// conflicts).
-__host__ __device__ constexpr int tc_stage_stride(int N, int fp8) {
-  return ((fp8 ? N : 2 * N) / 16) | 1;
-}
-
+// Shared memory: W_app's v k-blocks (d/64 tiles of N x 128 bytes), its k
+// k-blocks (d/64 tiles of r_k x 128 bytes), the ring, the epilogue's
+// staging (per warp: 32 dense rows of each cache part, z | e in the cache
+// element type), then the barriers.
 struct TcSmem {
-  size_t w, ring, stage, ktab, bars, total;
+  size_t wk, ring, stage, bars, total;
 };
 
-__host__ __device__ inline TcSmem tc_smem(int N, int d, int fp8, int slots) {
+__host__ __device__ inline TcSmem tc_smem(int r_v, int r_k, int d, int fp8, int slots) {
+  const int N = r_v + r_k;
   TcSmem L;
-  L.w = 0;                                           // nkb tiles of N x 128 bytes
-  L.ring = (size_t)N * 2 * d * 2;                    // a multiple of 2 KB
+  L.wk = (size_t)(d / 64) * N * 128;                 // multiples of 2 KB
+  L.ring = L.wk + (size_t)(d / 64) * r_k * 128;
   L.stage = L.ring + (size_t)slots * kTcABytes;
-  L.ktab = L.stage + (size_t)kTcEpiWarps * 32 * tc_stage_stride(N, fp8) * 16;
-  L.bars = L.ktab + kTcBM * 8;  // the Key warp's cache row per tile row
+  L.bars = L.stage + (size_t)kTcEpiWarps * 32 * N * (fp8 ? 1 : 2);
   L.total = L.bars + (2 * (size_t)slots + 7) * 8 + 16;
   return L;
+}
+
+__device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
+  asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0], %1; }" ::"r"(
+                   smem_u32(bar)),
+               "r"(n)
+               : "memory");
 }
 
 // shared -> global bulk copy (16-byte aligned ends, size % 16 == 0)
@@ -208,14 +213,16 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 __global__ void __launch_bounds__(kTcThreads, 1)
     append_tc_kernel(const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmW,
+                     const __grid_constant__ CUtensorMap tmWk,
                      const __grid_constant__ CUtensorMap tmKc, AppendArgs a, int N, int tmem_cols,
                      int slots, int n_mt) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1k(smem_raw);
   const int d = a.d, nkb = 2 * d / kTcBK;  // k-blocks: first d/64 from v, then from k
   const int cb = a.fp8 ? 1 : 2;            // cache bytes per element
-  const TcSmem L = tc_smem(N, d, a.fp8, slots);
-  uint8_t* w_tiles = smem + L.w;
+  const TcSmem L = tc_smem(a.r_v, a.r_k, d, a.fp8, slots);
+  uint8_t* w_tiles = smem;            // v k-blocks: N rows each
+  uint8_t* wk_tiles = smem + L.wk;    // k k-blocks: the r_k residual rows
   uint8_t* ring = smem + L.ring;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + slots;
@@ -236,7 +243,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < slots; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 2);  // the MMAs' commit + the Key warp's release (v slots: a stand-in)
+      // the MMAs' commit + the Key warps' releases (v slots: a stand-in)
+      mbar_init(&empty[s], 1 + kTcKeyWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
@@ -265,6 +273,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     prefetch_tmap(&tmV);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmW);
+    prefetch_tmap(&tmWk);
     if (!a.fp8) prefetch_tmap(&tmKc);
     int it = 0, wl = 0, cur_g = -1;
     bool ok = true;
@@ -285,9 +294,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (ok && g != cur_g) {  // a new head: its factor, once the last MMA on the old one is done
         if (wl > 0 && !(ok = mbar_wait_or_abort(wempty, (wl - 1) & 1, a.status, abort_flag)))
           break;
-        mbar_arrive_expect_tx(wfull, (uint32_t)N * 2 * d * 2);
-        for (int kb = 0; kb < nkb; ++kb)
+        mbar_arrive_expect_tx(wfull, (uint32_t)(N + a.r_k) * d * 2);
+        for (int kb = 0; kb < nkb / 2; ++kb) {
           tma_load_2d(w_tiles + kb * N * 128, &tmW, kb * kTcBK, g * N, wfull);
+          tma_load_2d(wk_tiles + kb * a.r_k * 128, &tmWk, d + kb * kTcBK, g * N + a.r_v, wfull);
+        }
         ++wl;
         cur_g = g;
       }
@@ -297,7 +308,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_wait(&full[u % slots], (u / slots) & 1, a.status, kTcDrainNs);
     if (wl > 0) mbar_wait(wfull, (wl - 1) & 1, a.status, kTcDrainNs);
   } else if (warp == 1 && lane == 0) {  // ------------------------------ MMA
-    const uint32_t idesc = tc_idesc(kTcBM, N);
+    const uint32_t idesc = tc_idesc(kTcBM, N), idesc_e = tc_idesc(kTcBM, a.r_k);
     int it = 0, wl = 0, cur_g = -1, lt = 0;
     bool ok = true;
     for (int item = i0; item < i1 && ok; ++item, ++lt) {
@@ -317,21 +328,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int s = it % slots;
         if (!(ok = mbar_wait_or_abort(&full[s], (it / slots) & 1, a.status, abort_flag))) break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        // a v k-block feeds all N columns; a k k-block only the e columns
+        const bool from_v = kb < nkb / 2;
         const uint64_t da = tc_sdesc(smem_u32(ring + s * kTcABytes));
-        const uint64_t db = tc_sdesc(smem_u32(w_tiles + kb * N * 128));
+        const uint64_t db = tc_sdesc(smem_u32(
+            from_v ? w_tiles + kb * N * 128 : wk_tiles + (kb - nkb / 2) * a.r_k * 128));
+        const uint32_t dk = from_v ? dt : dt + (uint32_t)a.r_v;
+        const uint32_t ik = from_v ? idesc : idesc_e;
 #pragma unroll
         for (int k = 0; k < kTcBK / 16; ++k) {
           const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
           asm volatile(
               "{ .reg .pred p; setp.ne.b32 p, %4, 0;"
-              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(dt),
-              "l"(da + 2 * k), "l"(db + 2 * k), "r"(idesc), "r"(acc)
+              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(dk),
+              "l"(da + 2 * k), "l"(db + 2 * k), "r"(ik), "r"(acc)
               : "memory");
         }
         // slot s is released when these MMAs complete (and, for a k slot,
-        // once the Key warp has copied it out)
+        // once the Key warps have copied it out)
         tc_commit(&empty[s]);
-        if (kb < nkb / 2) mbar_arrive(&empty[s]);
+        if (from_v) mbar_arrive_n(&empty[s], kTcKeyWarps);
       }
       if (!ok) break;
       tc_commit(&tfull[buf]);
@@ -340,11 +356,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // drain: one more commit tracks every MMA this thread issued
     tc_commit(drain);
     mbar_wait(drain, 0, a.status, kTcDrainNs);
-  } else if (warp >= 2 && warp < 2 + kTcEpiWarps) {  // ------------------- epilogue
+  } else if (warp >= 2 && warp < kTcKeyWarp0) {  // ----------------------- epilogue
     const int quarter = warp & 3;  // this warp's 32 TMEM lanes = tile rows
-    uint4* my = reinterpret_cast<uint4*>(smem + L.stage) +
-                ((size_t)(warp - 2) * 32 + lane) * tc_stage_stride(N, a.fp8);  // this lane's row
     const int zs = a.zsplit, es = a.esplit;
+    // this warp's staging: 32 dense rows of each part (Z's first zs
+    // columns, the rest of Z, E's first es columns, the rest of E)
+    uint8_t* const zA = smem + L.stage + (size_t)(warp - 2) * 32 * N * cb;
+    uint8_t* const zB = zA + 32 * zs * cb;
+    uint8_t* const eA = zA + 32 * a.r_v * cb;
+    uint8_t* const eB = eA + 32 * es * cb;
     uint8_t* const zc = reinterpret_cast<uint8_t*>(a.Z_cache);
     uint8_t* const ec = reinterpret_cast<uint8_t*>(a.E_cache);
     int lt = 0;
@@ -373,12 +393,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
+      // runs: consecutive live lanes on consecutive rows of one cache tile
+      const long long ptile = __shfl_up_sync(0xffffffffu, tile, 1);
+      const int ptrow = __shfl_up_sync(0xffffffffu, trow, 1);
+      const int plive = __shfl_up_sync(0xffffffffu, live, 1);
+      const bool lead =
+          live && (lane == 0 || !plive || ptile != tile || ptrow + 1 != trow);
+      const unsigned stops = __ballot_sync(0xffffffffu, lead || !live);
+      const unsigned after = stops & ~((2u << lane) - 1u);  // stops above this lane
+      const int run = (after ? __ffs(after) - 1 : 32) - lane;
       const int buf = lt & 1;
       bool ok = mbar_wait_or_abort(&tfull[buf], (lt >> 1) & 1, a.status, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      // accumulator -> cache element type -> this lane's staging row
+      // accumulator -> cache element type -> this lane's rows of the parts
       const uint32_t ta = tmem + (uint32_t)(buf * acc_cols) + ((uint32_t)(quarter * 32) << 16);
       for (int c0 = 0; c0 < N; c0 += 16) {
         uint32_t rr[16];
@@ -390,98 +419,95 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               "=r"(rr[12]), "=r"(rr[13]), "=r"(rr[14]), "=r"(rr[15])
             : "r"(ta + (uint32_t)c0));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        // the part holding columns c0 .. c0 + 15 (zs, es are multiples of 16)
+        uint8_t* dst;
+        if (c0 < zs)
+          dst = zA + (lane * zs + c0) * cb;
+        else if (c0 < a.r_v)
+          dst = zB + (lane * (a.r_v - zs) + c0 - zs) * cb;
+        else if (c0 < a.r_v + es)
+          dst = eA + (lane * es + c0 - a.r_v) * cb;
+        else
+          dst = eB + (lane * (a.r_k - es) + c0 - a.r_v - es) * cb;
         float v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(rr[i]);
-        if (a.fp8) {  // E4M3: 16 columns are one chunk
+        if (a.fp8) {  // E4M3: 16 columns are one 16-byte chunk
           uint32_t pb[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             pb[i] = f_to_e4m3x2(v[4 * i], v[4 * i + 1]) |
                     (f_to_e4m3x2(v[4 * i + 2], v[4 * i + 3]) << 16);
-          my[c0 / 16] = make_uint4(pb[0], pb[1], pb[2], pb[3]);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(pb[0], pb[1], pb[2], pb[3]);
         } else {
           uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             pk[i] = (uint32_t)f_to_bf16(v[2 * i]) | ((uint32_t)f_to_bf16(v[2 * i + 1]) << 16);
-          my[c0 / 8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          my[c0 / 8 + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          reinterpret_cast<uint4*>(dst)[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          reinterpret_cast<uint4*>(dst)[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
       // the accumulator buffer is free for the MMA two tiles on
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      // the staged rows are visible to the copy engine once every lane is here
+      fence_proxy_async();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
-      if (live) {
-        // the staging row's parts go to their caches (Z and E tiles store
-        // the first zsplit / esplit columns of every row first)
-        fence_proxy_async();
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(my);
+      if (lead) {
+        // one bulk copy per part for the run's rows (Z and E tiles store the
+        // first zs / es columns of every row first)
         const size_t zt = (size_t)tile * a.S * a.r_v * cb, et = (size_t)tile * a.S * a.r_k * cb;
-        bulk_store(zc + zt + (size_t)trow * zs * cb, src, zs * cb);
+        bulk_store(zc + zt + (size_t)trow * zs * cb, zA + lane * zs * cb, run * zs * cb);
         if (zs < a.r_v)
           bulk_store(zc + zt + ((size_t)a.S * zs + (size_t)trow * (a.r_v - zs)) * cb,
-                     src + zs * cb, (a.r_v - zs) * cb);
-        bulk_store(ec + et + (size_t)trow * es * cb, src + a.r_v * cb, es * cb);
+                     zB + lane * (a.r_v - zs) * cb, run * (a.r_v - zs) * cb);
+        bulk_store(ec + et + (size_t)trow * es * cb, eA + lane * es * cb, run * es * cb);
         if (es < a.r_k)
           bulk_store(ec + et + ((size_t)a.S * es + (size_t)trow * (a.r_k - es)) * cb,
-                     src + (a.r_v + es) * cb, (a.r_k - es) * cb);
+                     eB + lane * (a.r_k - es) * cb, run * (a.r_k - es) * cb);
       }
-      // the staging row is rewritten next tile, once the copy engine has read it
+      // the staging is rewritten next tile, once the copy engine has read it
       bulk_commit();
       bulk_wait_read();
+      __syncwarp();
     }
     bulk_wait_all();
-  } else if (warp == kTcKeyWarp) {  // --------------------------------- Key copy
-    // The exact Key, straight from each k slot (16-byte chunk j of tile row t
-    // sits at chunk j ^ (t & 7) of its 128-byte row).  tab[t] = the Key
-    // cache row of tile row t, or -1 for a dead row.
-    long long* tab = reinterpret_cast<long long*>(smem + L.ktab);
+  } else if (warp >= kTcKeyWarp0) {  // ---------------------------------- Key copy
+    // The exact Key of tile rows 32w .. 32w + 31 (w = this Key warp), straight
+    // from each k slot (16-byte chunk j of tile row t sits at chunk
+    // j ^ (t & 7) of its 128-byte row).
+    const int t = (warp - kTcKeyWarp0) * 32 + lane;  // this lane's tile row
     uint8_t* const kc = reinterpret_cast<uint8_t*>(a.K_cache);
     int lt = 0;
     bool ok = true;
     for (int item = i0; item < i1 && ok; ++item, ++lt) {
-      const int g = item / n_mt, m0 = (item % n_mt) * kTcBM;
-      __syncwarp();  // the previous tile's reads of tab are done
-      for (int i = 0; i < kTcBM / 32; ++i) {
-        const int t = lane + 32 * i, r = m0 + t;
-        long long sl = -1;
-        if (r < rows) {
-          const int b = r / a.n_new, j = r % a.n_new;
-          const int len = a.seq_lens[b];
-          if (len >= 0 && len + a.n_new <= a.max_pages * a.S) {
-            const int pos = len + j;
-            const int pp = a.block_table[(size_t)b * a.max_pages + pos / a.S];
-            if (pp >= 0 && pp < a.num_phys) sl = ((long long)pp * a.Hkv + g) * a.S + pos % a.S;
-          }
+      const int g = item / n_mt, r = (item % n_mt) * kTcBM + t;
+      long long sl = -1;  // this row's Key cache row, or -1 (dead)
+      if (r < rows) {
+        const int b = r / a.n_new, j = r % a.n_new;
+        const int len = a.seq_lens[b];
+        if (len >= 0 && len + a.n_new <= a.max_pages * a.S) {
+          const int pos = len + j;
+          const int pp = a.block_table[(size_t)b * a.max_pages + pos / a.S];
+          if (pp >= 0 && pp < a.num_phys) sl = ((long long)pp * a.Hkv + g) * a.S + pos % a.S;
         }
-        tab[t] = sl;
       }
-      __syncwarp();
-      // lane j < 16: do the 8 rows of group j land on 8 consecutive cache rows?
-      bool boxed = false;
-      if (!a.fp8 && lane < kTcBM / 8) {
-        const long long s0 = tab[8 * lane];
-        boxed = s0 >= 0;
-        for (int i = 1; i < 8; ++i) boxed = boxed && tab[8 * lane + i] == s0 + i;
-      }
-      const unsigned bmask = __ballot_sync(0xffffffffu, boxed);
+      // do the 8 rows of this lane's group land on 8 consecutive cache rows?
+      const long long s0 = __shfl_sync(0xffffffffu, sl, lane & ~7);
+      const unsigned seq = __ballot_sync(0xffffffffu, sl >= 0 && sl == s0 + (lane & 7));
+      const bool boxed = !a.fp8 && ((seq >> (lane & ~7)) & 0xffu) == 0xffu;
       for (int kb = 0; kb < nkb / 2; ++kb) {
         const int u = lt * nkb + nkb / 2 + kb, s = u % slots;
         ok = __all_sync(0xffffffffu,
                         mbar_wait_or_abort(&full[s], (u / slots) & 1, a.status, abort_flag));
         if (!ok) break;
-        const uint8_t* stage = ring + (size_t)s * kTcABytes;
-        if (boxed) tma_store_2d(&tmKc, stage + lane * 8 * 128, kb * kTcBK, (int32_t)tab[8 * lane]);
-        if (bmask != (1u << (kTcBM / 8)) - 1) {
-          // the other rows, four per pass, eight lanes on a row's chunks
-          for (int p = 0; p < kTcBM / 4; ++p) {
-            const int t = p * 4 + (lane >> 3), ch = lane & 7;
-            const long long sl = tab[t];
-            if (((bmask >> (t >> 3)) & 1u) || sl < 0) continue;
-            const uint4 x =
-                *reinterpret_cast<const uint4*>(stage + t * 128 + ((ch ^ (t & 7)) << 4));
+        const uint8_t* row = ring + (size_t)s * kTcABytes + t * 128;
+        if (boxed) {
+          if ((lane & 7) == 0) tma_store_2d(&tmKc, row, kb * kTcBK, (int32_t)sl);
+        } else if (sl >= 0) {
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint4 x = *reinterpret_cast<const uint4*>(row + ((ch ^ (t & 7)) << 4));
             if (a.fp8) {
               const float2 f0 = bf16x2_to_f2(x.x), f1 = bf16x2_to_f2(x.y),
                            f2 = bf16x2_to_f2(x.z), f3 = bf16x2_to_f2(x.w);
@@ -532,17 +558,17 @@ cudaError_t launch_fold_append(const FoldAppArgs& a, cudaStream_t st, bool pdl) 
 }
 
 cudaError_t launch_append_tc(const AppendArgs& a, const CUtensorMap& tmV, const CUtensorMap& tmK,
-                             const CUtensorMap& tmW, const CUtensorMap& tmKc, cudaStream_t st,
-                             bool pdl) {
+                             const CUtensorMap& tmW, const CUtensorMap& tmWk,
+                             const CUtensorMap& tmKc, cudaStream_t st, bool pdl) {
   const int N = a.r_v + a.r_k;
   const int acc = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
   const int tmem_cols = 2 * acc;  // two accumulator buffers
   const int nkb = 2 * a.d / kTcBK;
   const size_t cap = 227 * 1024 - 1024;  // the 1 KB alignment pad comes off the top
-  const size_t fixed = tc_smem(N, a.d, a.fp8, 0).total;
+  const size_t fixed = tc_smem(a.r_v, a.r_k, a.d, a.fp8, 0).total;
   if (fixed + (size_t)nkb * kTcABytes > cap) return cudaErrorInvalidConfiguration;
   const int slots = (int)std::min<size_t>(kTcMaxSlots, (cap - fixed) / kTcABytes);
-  const size_t smem = tc_smem(N, a.d, a.fp8, slots).total + 1024;
+  const size_t smem = tc_smem(a.r_v, a.r_k, a.d, a.fp8, slots).total + 1024;
   cudaError_t e = cudaFuncSetAttribute(append_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -550,7 +576,7 @@ cudaError_t launch_append_tc(const AppendArgs& a, const CUtensorMap& tmV, const 
   const int n_mt = (rows + kTcBM - 1) / kTcBM;
   const int grid = std::min(n_mt * a.Hkv, num_sms());
   return launch_k(append_tc_kernel, dim3(grid), dim3(kTcThreads), smem, st, pdl, tmV, tmK, tmW,
-                  tmKc, a, N, tmem_cols, slots, n_mt);
+                  tmWk, tmKc, a, N, tmem_cols, slots, n_mt);
 }
 
 }  // namespace basiskv
