@@ -321,25 +321,51 @@ int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_b
     }
     const int N = d->r_v + d->r_k;
     const uint64_t rows = (uint64_t)d->B * n_new;
-    const uint64_t dims3[3] = {(uint64_t)d->d, (uint64_t)d->Hkv, rows};
-    const uint64_t str3[2] = {(uint64_t)d->d * 2, (uint64_t)d->Hkv * d->d * 2};
-    const uint32_t box3[3] = {64, 1, 128};
-    CUtensorMap tmV, tmK, tmW, tmWk, tmKc;
-    if (!make_tmap_3d(&tmV, v_new, dims3, str3, box3, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_3d(&tmK, k_new, dims3, str3, box3, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_2d(&tmW, w_app, (uint64_t)d->Hkv * N, 2 * d->d, (uint64_t)4 * d->d, N, 64,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_2d(&tmWk, w_app, (uint64_t)d->Hkv * N, 2 * d->d, (uint64_t)4 * d->d, d->r_k,
-                      64, CU_TENSOR_MAP_SWIZZLE_128B))
-      return BASISKV_ERR_CUDA;
-    if (d->cache_fp8) {
-      tmKc = tmK;  // not read: E4M3 Key rows leave through the staging rows
-    } else if (!make_tmap_2d(&tmKc, K_cache,
-                             (uint64_t)d->num_phys_pages * d->Hkv * d->page_size, d->d,
-                             (uint64_t)d->d * 2, 8, 64, CU_TENSOR_MAP_SWIZZLE_128B)) {
-      return BASISKV_ERR_CUDA;
+    // The five tensor maps depend only on these addresses and sizes; a
+    // caller that appends chunk after chunk from the same buffers (a prefill
+    // loop) reuses the previous call's maps instead of encoding them again.
+    struct MapKey {
+      const void *v, *k, *w, *kc;
+      uint64_t rows;
+      int d, Hkv, N, r_k, slots_rows, fp8;
+      bool operator==(const MapKey& o) const {
+        return v == o.v && k == o.k && w == o.w && kc == o.kc && rows == o.rows && d == o.d &&
+               Hkv == o.Hkv && N == o.N && r_k == o.r_k && slots_rows == o.slots_rows &&
+               fp8 == o.fp8;
+      }
+    };
+    struct MapSet {
+      bool valid = false;
+      MapKey key;
+      CUtensorMap v, k, w, wk, kc;
+    };
+    thread_local MapSet cache;
+    const MapKey key{v_new, k_new, w_app, K_cache, rows, d->d, d->Hkv, N, d->r_k,
+                     d->num_phys_pages * d->Hkv * d->page_size, d->cache_fp8};
+    if (!(cache.valid && cache.key == key)) {
+      cache.valid = false;
+      const uint64_t dims3[3] = {(uint64_t)d->d, (uint64_t)d->Hkv, rows};
+      const uint64_t str3[2] = {(uint64_t)d->d * 2, (uint64_t)d->Hkv * d->d * 2};
+      const uint32_t box3[3] = {64, 1, 128};
+      if (!make_tmap_3d(&cache.v, v_new, dims3, str3, box3, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !make_tmap_3d(&cache.k, k_new, dims3, str3, box3, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !make_tmap_2d(&cache.w, w_app, (uint64_t)d->Hkv * N, 2 * d->d, (uint64_t)4 * d->d, N,
+                        64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !make_tmap_2d(&cache.wk, w_app, (uint64_t)d->Hkv * N, 2 * d->d, (uint64_t)4 * d->d,
+                        d->r_k, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return BASISKV_ERR_CUDA;
+      if (d->cache_fp8) {
+        cache.kc = cache.k;  // not read: E4M3 Key rows are rounded lane by lane
+      } else if (!make_tmap_2d(&cache.kc, K_cache,
+                               (uint64_t)d->num_phys_pages * d->Hkv * d->page_size, d->d,
+                               (uint64_t)d->d * 2, 8, 64, CU_TENSOR_MAP_SWIZZLE_128B)) {
+        return BASISKV_ERR_CUDA;
+      }
+      cache.key = key;
+      cache.valid = true;
     }
-    rc = launch_status(launch_append_tc(a, tmV, tmK, tmW, tmWk, tmKc, st, pdl));
+    rc = launch_status(
+        launch_append_tc(a, cache.v, cache.k, cache.w, cache.wk, cache.kc, st, pdl));
   } else {
     rc = launch_status(launch_append_small(a, st, pdl));
   }

@@ -59,6 +59,9 @@ __global__ void __launch_bounds__(kFoldThreads)
 // kernel skipped the sequence for the same reason.
 __global__ void bump_lengths_kernel(const int32_t* seq_lens, int32_t* out, int B, int n_new,
                                     int cap, unsigned int* status) {
+  // the next launch may be scheduled at once: it waits for this grid to
+  // complete before it touches the lengths
+  pdl_launch_dependents();
   pdl_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= B) return;

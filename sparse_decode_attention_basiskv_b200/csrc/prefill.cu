@@ -15,6 +15,7 @@
 // is rounded to bf16 once; the decode-time append (append.cu) keeps the
 // two-step form with an unrounded z.
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "internal.h"
@@ -152,7 +153,7 @@ __device__ __forceinline__ uint64_t tc_sdesc(uint32_t saddr) {
 // staging (per warp: 32 dense rows of each cache part, z | e in the cache
 // element type), then the barriers.
 struct TcSmem {
-  size_t wk, ring, stage, bars, total;
+  size_t wk, ring, stage, bars, lens, total;
 };
 
 __host__ __device__ inline TcSmem tc_smem(int r_v, int r_k, int d, int fp8, int slots) {
@@ -162,8 +163,31 @@ __host__ __device__ inline TcSmem tc_smem(int r_v, int r_k, int d, int fp8, int 
   L.ring = L.wk + (size_t)(d / 64) * r_k * 128;
   L.stage = L.ring + (size_t)slots * kTcABytes;
   L.bars = L.stage + (size_t)kTcEpiWarps * 32 * N * (fp8 ? 1 : 2);
-  L.total = L.bars + (2 * (size_t)slots + 7) * 8 + 16;
+  L.lens = L.bars + (2 * (size_t)slots + 7) * 8 + 16;
+  L.total = L.lens + 256 * 4;  // the sequences' lengths (B <= 256)
   return L;
+}
+
+// Cache position of token row r of the chunk (pos = -1: no such row, or its
+// sequence would overflow) and the block-table entry of that position's
+// page, loaded here and checked where it is used, a tile later.
+struct RowRef {
+  int pos, pp;
+};
+
+__device__ __forceinline__ RowRef row_ref(const AppendArgs& a, const int* lens, int rows, int r,
+                                          int g, bool report) {
+  RowRef x{-1, -1};
+  if (r >= rows) return x;
+  const int b = r / a.n_new, j = r - b * a.n_new;
+  const int len = lens[b];
+  if (len < 0 || len + a.n_new > a.max_pages * a.S) {
+    if (report && j == 0 && g == 0) raise_status(a.status, BASISKV_DEV_OVERFLOW);
+    return x;
+  }
+  x.pos = len + j;
+  x.pp = a.block_table[(size_t)b * a.max_pages + x.pos / a.S];
+  return x;
 }
 
 __device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
@@ -268,6 +292,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
   pdl_wait();
+  // The next launch (the length update) may be scheduled now: it waits for
+  // this grid to complete before it reads or writes anything.
+  pdl_launch_dependents();
+  // the epilogue and Key warps read the lengths from shared memory
+  int* lens = reinterpret_cast<int*>(smem + L.lens);
+  if (warp >= 2) {
+    for (int i = tid - 64; i < a.B; i += kTcThreads - 64) lens[i] = a.seq_lens[i];
+    asm volatile("bar.sync 1, %0;" ::"r"(kTcThreads - 64) : "memory");
+  }
 
   if (warp == 0 && lane == 0) {  // ------------------------------------- TMA
     prefetch_tmap(&tmV);
@@ -279,6 +312,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     for (int item = i0; item < i1 && ok; ++item) {
       const int g = item / n_mt, m0 = (item % n_mt) * kTcBM;
+      if (item == i0) {  // the first head's factor goes first: every MMA needs it
+        mbar_arrive_expect_tx(wfull, (uint32_t)(N + a.r_k) * d * 2);
+        for (int kb = 0; kb < nkb / 2; ++kb) {
+          tma_load_2d(w_tiles + kb * N * 128, &tmW, kb * kTcBK, g * N, wfull);
+          tma_load_2d(wk_tiles + kb * a.r_k * 128, &tmWk, d + kb * kTcBK, g * N + a.r_v, wfull);
+        }
+        wl = 1;
+        cur_g = g;
+      }
       for (int kb = 0; kb < nkb; ++kb, ++it) {
         const int s = it % slots;
         // the slot is free once its previous k-block has been consumed
@@ -368,31 +410,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t* const zc = reinterpret_cast<uint8_t*>(a.Z_cache);
     uint8_t* const ec = reinterpret_cast<uint8_t*>(a.E_cache);
     int lt = 0;
+    RowRef cur = i0 < i1 ? row_ref(a, lens, rows, (i0 % n_mt) * kTcBM + quarter * 32 + lane,
+                                   i0 / n_mt, true)
+                         : RowRef{-1, -1};
     for (int item = i0; item < i1; ++item, ++lt) {
-      const int g = item / n_mt, m0 = (item % n_mt) * kTcBM;
+      const int g = item / n_mt;
+      // the next tile's block-table entry is in flight while this tile drains
+      const RowRef nxt =
+          item + 1 < i1 ? row_ref(a, lens, rows, ((item + 1) % n_mt) * kTcBM + quarter * 32 + lane,
+                                  (item + 1) / n_mt, true)
+                        : RowRef{-1, -1};
       // this lane's row: its cache tile (physical page x KV head) and row
       // within the tile, or dead
-      const int r = m0 + quarter * 32 + lane;
       long long tile = 0;
       int trow = 0, live = 0;
-      if (r < rows) {
-        const int b = r / a.n_new, j = r % a.n_new;
-        const int len = a.seq_lens[b];
-        const int cap = a.max_pages * a.S;
-        if (len < 0 || len + a.n_new > cap) {
-          if (j == 0 && g == 0) raise_status(a.status, BASISKV_DEV_OVERFLOW);
+      if (cur.pos >= 0) {
+        if (cur.pp < 0 || cur.pp >= a.num_phys) {
+          raise_status(a.status, BASISKV_DEV_BAD_PAGE);
         } else {
-          const int pos = len + j;
-          const int pp = a.block_table[(size_t)b * a.max_pages + pos / a.S];
-          if (pp < 0 || pp >= a.num_phys) {
-            raise_status(a.status, BASISKV_DEV_BAD_PAGE);
-          } else {
-            tile = (long long)pp * a.Hkv + g;
-            trow = pos % a.S;
-            live = 1;
-          }
+          tile = (long long)cur.pp * a.Hkv + g;
+          trow = cur.pos % a.S;
+          live = 1;
         }
       }
+      cur = nxt;
       // runs: consecutive live lanes on consecutive rows of one cache tile
       const long long ptile = __shfl_up_sync(0xffffffffu, tile, 1);
       const int ptrow = __shfl_up_sync(0xffffffffu, trow, 1);
@@ -481,18 +522,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint8_t* const kc = reinterpret_cast<uint8_t*>(a.K_cache);
     int lt = 0;
     bool ok = true;
+    RowRef cur = i0 < i1 ? row_ref(a, lens, rows, (i0 % n_mt) * kTcBM + t, i0 / n_mt, false)
+                         : RowRef{-1, -1};
     for (int item = i0; item < i1 && ok; ++item, ++lt) {
-      const int g = item / n_mt, r = (item % n_mt) * kTcBM + t;
+      const int g = item / n_mt;
+      // the next tile's block-table entry is in flight while this tile's slots drain
+      const RowRef nxt = item + 1 < i1 ? row_ref(a, lens, rows, ((item + 1) % n_mt) * kTcBM + t,
+                                                 (item + 1) / n_mt, false)
+                                       : RowRef{-1, -1};
       long long sl = -1;  // this row's Key cache row, or -1 (dead)
-      if (r < rows) {
-        const int b = r / a.n_new, j = r % a.n_new;
-        const int len = a.seq_lens[b];
-        if (len >= 0 && len + a.n_new <= a.max_pages * a.S) {
-          const int pos = len + j;
-          const int pp = a.block_table[(size_t)b * a.max_pages + pos / a.S];
-          if (pp >= 0 && pp < a.num_phys) sl = ((long long)pp * a.Hkv + g) * a.S + pos % a.S;
-        }
-      }
+      if (cur.pos >= 0 && cur.pp >= 0 && cur.pp < a.num_phys)
+        sl = ((long long)cur.pp * a.Hkv + g) * a.S + cur.pos % a.S;
+      cur = nxt;
       // do the 8 rows of this lane's group land on 8 consecutive cache rows?
       const long long s0 = __shfl_sync(0xffffffffu, sl, lane & ~7);
       const unsigned seq = __ballot_sync(0xffffffffu, sl >= 0 && sl == s0 + (lane & 7));
@@ -569,9 +610,22 @@ cudaError_t launch_append_tc(const AppendArgs& a, const CUtensorMap& tmV, const 
   if (fixed + (size_t)nkb * kTcABytes > cap) return cudaErrorInvalidConfiguration;
   const int slots = (int)std::min<size_t>(kTcMaxSlots, (cap - fixed) / kTcABytes);
   const size_t smem = tc_smem(a.r_v, a.r_k, a.d, a.fp8, slots).total + 1024;
-  cudaError_t e = cudaFuncSetAttribute(append_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the kernel's shared-memory limit, raised once per device to the largest
+  // size asked for so far
+  static std::atomic<int> raised[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || raised[dev].load(std::memory_order_relaxed) < (int)smem) {
+    e = cudaFuncSetAttribute(append_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) {
+      int cur = raised[dev].load();
+      while (cur < (int)smem && !raised[dev].compare_exchange_weak(cur, (int)smem)) {
+      }
+    }
+  }
   const int rows = a.B * a.n_new;
   const int n_mt = (rows + kTcBM - 1) / kTcBM;
   const int grid = std::min(n_mt * a.Hkv, num_sms());
