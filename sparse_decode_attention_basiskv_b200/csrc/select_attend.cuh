@@ -117,6 +117,9 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
   // A 16-token unit is 1 / TP of a routing page of S tokens, or QP routing
   // pages of 4 or 8 tokens.
   const int RPG = a.rp ? a.rp : S, NR = S / RPG, QP = RPG < 16 ? 16 / RPG : 0;
+  // every one of these is a power of two: the unit addressing below shifts
+  // and masks (TP is 1 or 2 wherever it is used)
+  const int logTP = TP >> 1, logNR = 31 - __clz(NR), logRPG = 31 - __clz(RPG);
   const int P_phys = (s.max_seq_len + S - 1) / S;  // block-table entries read
 
   // The out-projection may take SMs as this grid's CTAs retire; it requests
@@ -208,7 +211,8 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
     int p0, p1;
   };
   auto cache_page = [&](int lp) -> int {
-    int pp = lp >= 0 && lp / NR < P_phys ? tbl[lp / NR] : -1;
+    const int cp = lp >> logNR;
+    int pp = lp >= 0 && cp < P_phys ? tbl[cp] : -1;
     if (lp < 0) {
       pp = 0;
     } else if (pp < 0 || pp >= a.num_phys) {
@@ -221,21 +225,21 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
     const int idx = u0 + warp + kAmWarps * nn;
     Rows u;
     if (QP == 0) {
-      const int lp = list[idx / TP], tau = idx % TP;
+      const int lp = list[idx >> logTP], tau = idx & (TP - 1);
       u.r0 = ((size_t)cache_page(lp) * a.Hkv + g) * S + 16 * tau + lr;
       u.r1 = u.r0 + 8;
       u.p0 = lp >= 0 ? lp * S + 16 * tau + lr : INT_MAX;
       u.p1 = lp >= 0 ? u.p0 + 8 : INT_MAX;
     } else {
-      const int x0 = lr, x1 = lr + 8;
-      const int s0 = idx * QP + x0 / RPG, s1 = idx * QP + x1 / RPG;
+      const int x0 = lr, x1 = lr + 8, m = RPG - 1;
+      const int s0 = idx * QP + (x0 >> logRPG), s1 = idx * QP + (x1 >> logRPG);
       const int lp0 = s0 < nsel ? list[s0] : -1, lp1 = s1 < nsel ? list[s1] : -1;
-      u.r0 = ((size_t)cache_page(lp0) * a.Hkv + g) * S + (lp0 >= 0 ? lp0 % NR : 0) * RPG +
-             x0 % RPG;
-      u.r1 = ((size_t)cache_page(lp1) * a.Hkv + g) * S + (lp1 >= 0 ? lp1 % NR : 0) * RPG +
-             x1 % RPG;
-      u.p0 = lp0 >= 0 ? lp0 * RPG + x0 % RPG : INT_MAX;
-      u.p1 = lp1 >= 0 ? lp1 * RPG + x1 % RPG : INT_MAX;
+      u.r0 = ((size_t)cache_page(lp0) * a.Hkv + g) * S +
+             (lp0 >= 0 ? (lp0 & (NR - 1)) << logRPG : 0) + (x0 & m);
+      u.r1 = ((size_t)cache_page(lp1) * a.Hkv + g) * S +
+             (lp1 >= 0 ? (lp1 & (NR - 1)) << logRPG : 0) + (x1 & m);
+      u.p0 = lp0 >= 0 ? (lp0 << logRPG) + (x0 & m) : INT_MAX;
+      u.p1 = lp1 >= 0 ? (lp1 << logRPG) + (x1 & m) : INT_MAX;
     }
     return u;
   };
@@ -257,17 +261,19 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
     }
   };
   auto load_z = [&](const Rows& u, int slot) {  // asynchronous, into the warp's ring
-    const size_t tile0 = u.r0 >> logS, tile1 = u.r1 >> logS;
-    const int trow0 = (int)(u.r0 & (S - 1)), trow1 = (int)(u.r1 & (S - 1));
+    // rows r0 and r1 = r0 + 8 share one tile unless routing pages split the unit
+    const size_t tile0 = u.r0 >> logS, tile1 = QP == 0 ? tile0 : u.r1 >> logS;
+    const int trow0 = (int)(u.r0 & (S - 1)), trow1 = QP == 0 ? trow0 + 8 : (int)(u.r1 & (S - 1));
+    const size_t zt0 = tile0 * S * RV, zt1 = QP == 0 ? zt0 : tile1 * S * RV;
     if constexpr (F8) {
       const uint8_t* z8 = reinterpret_cast<const uint8_t*>(a.Z);
 #pragma unroll
       for (int c = 0; c < NZC; ++c) {
         const int col = 32 * c + 8 * lc;
         cp_async8(zring8 + ((slot * NZC + c) * 2 + 0) * 32 + lane,
-                  z8 + tile0 * S * RV + split_off(trow0, col, S, RV, a.zsplit));
+                  z8 + zt0 + split_off(trow0, col, S, RV, a.zsplit));
         cp_async8(zring8 + ((slot * NZC + c) * 2 + 1) * 32 + lane,
-                  z8 + tile1 * S * RV + split_off(trow1, col, S, RV, a.zsplit));
+                  z8 + zt1 + split_off(trow1, col, S, RV, a.zsplit));
       }
       return;
     }
@@ -275,9 +281,9 @@ __global__ void __launch_bounds__(kAmThreads, kAmCtasPerSm)
     for (int c = 0; c < NZC; ++c) {
       const int col = 32 * c + 8 * lc;
       cp_async16(zring + ((slot * NZC + c) * 2 + 0) * 32 + lane,
-                 a.Z + tile0 * S * RV + split_off(trow0, col, S, RV, a.zsplit));
+                 a.Z + zt0 + split_off(trow0, col, S, RV, a.zsplit));
       cp_async16(zring + ((slot * NZC + c) * 2 + 1) * 32 + lane,
-                 a.Z + tile1 * S * RV + split_off(trow1, col, S, RV, a.zsplit));
+                 a.Z + zt1 + split_off(trow1, col, S, RV, a.zsplit));
     }
   };
   Rows cur{0, 8, INT_MAX, INT_MAX};

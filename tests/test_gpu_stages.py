@@ -295,6 +295,13 @@ RAGGED_PREFILL = {
     # items over the SMs, so every CTA runs many items and reloads W_app
     "qwen_b8_4096": (synth.with_sizes(synth.QWEN32B_T64K_B8, B=8, T=160, prefill_tokens=4096),
                      [96, 101, 3, 64, 77, 32, 0, 159]),
+    # other product shapes: d 64 (one k-block per operand, N = 48), r_k 64
+    # with N = 160 and 192 (the fewest ring slots), pages of 8 and 32 tokens
+    "tiny_d64": (synth.with_sizes(synth.TINY, B=3, T=160, prefill_tokens=200), [5, 37, 131]),
+    "llama_v96_k64_p8": (synth.with_sizes(synth.LLAMA8B_T4K, B=2, T=160, r_k=64, page_size=8,
+                                          prefill_tokens=700), [13, 150]),
+    "llama_v128_k64_p32": (synth.with_sizes(synth.LLAMA8B_T4K, B=2, T=160, r_v=128, r_k=64,
+                                            page_size=32, prefill_tokens=700), [0, 77]),
 }
 
 
@@ -364,17 +371,19 @@ def test_device_status_reports_bad_inputs():
     assert layer.seq_lens.item() == cap
 
 
+@pytest.mark.parametrize("T", [16384, 2048], ids=["p1024", "p128"])
 @pytest.mark.parametrize("levels", [1, 3, 64])
-def test_selection_with_tied_scores(levels):
+def test_selection_with_tied_scores(levels, T):
     """Page scores with many exact ties: z is zero except column 0 of every
     token, which holds one of `levels` values per page, and e is zero, so a
     page's score is one product per head and pages with the same value tie
-    exactly (levels = 1: every score equal).  The threshold's bin then holds
-    hundreds of pages (1, 3 levels: the radix select decides) or a few (64
-    levels).  Ties rank by the lower page index on both sides, so the
-    selection must equal the oracle's bit for bit, through the selection
-    launch and through the fused decode step."""
-    wl = synth.with_sizes(synth.LLAMA8B_T32K_B16, B=2, T=16384, top_k=64)
+    exactly (levels = 1: every score equal).  At 1024 pages the threshold's
+    bin then holds hundreds of pages (1, 3 levels: the radix select decides)
+    or a few (64 levels); at 128 pages every candidate is ranked directly.
+    Ties rank by the lower page index on both sides, so the selection must
+    equal the oracle's bit for bit, through the selection launch and through
+    the fused decode step."""
+    wl = synth.with_sizes(synth.LLAMA8B_T32K_B16, B=2, T=T, top_k=64)
     pb = synth.make_problem(wl, device="cuda")
     S, P = wl.page_size, wl.pages
     lvl = torch.arange(P, device="cuda").remainder(levels).float() + 1.0
