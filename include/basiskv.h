@@ -319,7 +319,7 @@ BASISKV_API int basiskv_outproj_sources(const basiskv_dims* dims, const basiskv_
 /* Size of the static device scratch array behind basiskv_decode_noalloc. */
 #define BASISKV_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 
-/* basiskv_decode for callers that cannot allocate device memory.  The paper
+/* basiskv_decode for callers that cannot allocate device memory.  The method
  * has no counterpart: this is a deployment variant of the fused decode step.
  *
  * Some callers cannot call cudaMalloc when they run a step: a runtime that
@@ -357,7 +357,7 @@ BASISKV_API int basiskv_decode_noalloc(const basiskv_dims* dims, const basiskv_b
  * itself reported an error. */
 BASISKV_API int basiskv_read_device_status(void* stream, uint32_t* flags);
 
-/* Self-test of the library's bounded waits.  The paper has no counterpart:
+/* Self-test of the library's bounded waits.  The method has no counterpart:
  * this checks the failure path every kernel relies on.  Every wait of a
  * kernel here on an mbarrier gives up after a time limit, records
  * BASISKV_DEV_TIMEOUT in the device status word and lets the kernel return,

@@ -153,7 +153,7 @@ __device__ __forceinline__ uint64_t tc_sdesc(uint32_t saddr) {
 // staging (per warp: 32 dense rows of each cache part, z | e in the cache
 // element type), then the barriers.
 struct TcSmem {
-  size_t wk, ring, stage, bars, lens, total;
+  size_t wk, ring, stage, kstage, bars, lens, total;
 };
 
 __host__ __device__ inline TcSmem tc_smem(int r_v, int r_k, int d, int fp8, int slots) {
@@ -162,7 +162,9 @@ __host__ __device__ inline TcSmem tc_smem(int r_v, int r_k, int d, int fp8, int 
   L.wk = (size_t)(d / 64) * N * 128;                 // multiples of 2 KB
   L.ring = L.wk + (size_t)(d / 64) * r_k * 128;
   L.stage = L.ring + (size_t)slots * kTcABytes;
-  L.bars = L.stage + (size_t)kTcEpiWarps * 32 * N * (fp8 ? 1 : 2);
+  L.kstage = L.stage + (size_t)kTcEpiWarps * 32 * N * (fp8 ? 1 : 2);
+  // E4M3 caches: each Key warp's 32 rounded Key rows (d bytes each)
+  L.bars = L.kstage + (fp8 ? (size_t)kTcKeyWarps * 32 * d : 0);
   L.lens = L.bars + (2 * (size_t)slots + 7) * 8 + 16;
   L.total = L.lens + 256 * 4;  // the sequences' lengths (B <= 256)
   return L;
@@ -517,9 +519,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp >= kTcKeyWarp0) {  // ---------------------------------- Key copy
     // The exact Key of tile rows 32w .. 32w + 31 (w = this Key warp), straight
     // from each k slot (16-byte chunk j of tile row t sits at chunk
-    // j ^ (t & 7) of its 128-byte row).
+    // j ^ (t & 7) of its 128-byte row).  E4M3 caches: each lane rounds its
+    // row into the warp's staging rows, and every run of consecutive cache
+    // rows leaves as one bulk copy.
     const int t = (warp - kTcKeyWarp0) * 32 + lane;  // this lane's tile row
     uint8_t* const kc = reinterpret_cast<uint8_t*>(a.K_cache);
+    uint8_t* const k8 = smem + L.kstage + (size_t)(warp - kTcKeyWarp0) * 32 * d;  // [32][d]
+    // Lane-dependent chunk order for the rounding: chunk c = ch ^ A(l) of
+    // row l in step ch, A(l) = 2l over GF(8) (x^3 + x + 1).  A and A + 1 are
+    // both one-to-one, so in every step eight consecutive lanes read eight
+    // different 16-byte chunk positions of the swizzled slot (c ^ l) and
+    // write eight different 8-byte columns of their staging rows (c).
+    const int gl = lane & 7, gfa = ((gl << 1) ^ ((gl >> 2) * 3)) & 7;
     int lt = 0;
     bool ok = true;
     RowRef cur = i0 < i1 ? row_ref(a, lens, rows, (i0 % n_mt) * kTcBM + t, i0 / n_mt, false)
@@ -544,27 +555,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         mbar_wait_or_abort(&full[s], (u / slots) & 1, a.status, abort_flag));
         if (!ok) break;
         const uint8_t* row = ring + (size_t)s * kTcABytes + t * 128;
-        if (boxed) {
-          if ((lane & 7) == 0) tma_store_2d(&tmKc, row, kb * kTcBK, (int32_t)sl);
-        } else if (sl >= 0) {
-          for (int ch = 0; ch < 8; ++ch) {
-            const uint4 x = *reinterpret_cast<const uint4*>(row + ((ch ^ (t & 7)) << 4));
-            if (a.fp8) {
+        if (a.fp8) {
+          if (sl >= 0)
+            for (int ch = 0; ch < 8; ++ch) {
+              const int c = ch ^ gfa;
+              const uint4 x = *reinterpret_cast<const uint4*>(row + ((c ^ (t & 7)) << 4));
               const float2 f0 = bf16x2_to_f2(x.x), f1 = bf16x2_to_f2(x.y),
                            f2 = bf16x2_to_f2(x.z), f3 = bf16x2_to_f2(x.w);
-              *reinterpret_cast<uint2*>(kc + sl * d + kb * kTcBK + ch * 8) =
+              *reinterpret_cast<uint2*>(k8 + lane * d + kb * kTcBK + c * 8) =
                   make_uint2(f_to_e4m3x2(f0.x, f0.y) | (f_to_e4m3x2(f1.x, f1.y) << 16),
                              f_to_e4m3x2(f2.x, f2.y) | (f_to_e4m3x2(f3.x, f3.y) << 16));
-            } else {
-              *reinterpret_cast<uint4*>(kc + (sl * d + kb * kTcBK + ch * 8) * 2) = x;
             }
-          }
+        } else if (boxed) {
+          if ((lane & 7) == 0) tma_store_2d(&tmKc, row, kb * kTcBK, (int32_t)sl);
+        } else if (sl >= 0) {
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(kc + (sl * d + kb * kTcBK + ch * 8) * 2) =
+                *reinterpret_cast<const uint4*>(row + ((ch ^ (t & 7)) << 4));
         }
         // the slot goes back to the producer once the copy engine has read it
         bulk_commit();
         bulk_wait_read();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
+      }
+      if (a.fp8 && ok) {
+        // runs: consecutive lanes on consecutive Key cache rows
+        const long long psl = __shfl_up_sync(0xffffffffu, sl, 1);
+        const bool lead = sl >= 0 && (lane == 0 || psl < 0 || psl + 1 != sl);
+        const unsigned stops = __ballot_sync(0xffffffffu, lead || sl < 0);
+        const unsigned after = stops & ~((2u << lane) - 1u);
+        const int run = (after ? __ffs(after) - 1 : 32) - lane;
+        fence_proxy_async();  // the rounded rows are visible to the copy engine
+        __syncwarp();
+        if (lead) bulk_store(kc + sl * d, k8 + lane * d, (uint32_t)(run * d));
+        bulk_commit();
+        bulk_wait_read();  // the staging rows are rewritten next tile
+        __syncwarp();
       }
     }
     bulk_wait_all();

@@ -371,6 +371,44 @@ def test_device_status_reports_bad_inputs():
     assert layer.seq_lens.item() == cap
 
 
+def test_prefill_append_reports_bad_pages_and_overflow():
+    """The tensor-core append's own checks.  A block-table entry outside
+    the cache: that page's rows are skipped (the bad-page bit is set) and
+    every other row lands.  A chunk that would pass the end of a sequence's
+    block-table row: that sequence is skipped whole (the overflow bit) and
+    its length is left as it was, while the other sequence appends."""
+    wl = synth.with_sizes(synth.QWEN32B_T64K_B8, B=2, T=160, prefill_tokens=400)
+    n, S = 200, wl.page_size
+    pb, layer = gpu_layer(wl, seq_lens=[5, 37])
+    k, v = synth.make_tokens(wl, pb.factors, n, device="cuda", stream_id=5)
+    status_clean()
+    lp_bad = (5 + 60) // S  # a page inside sequence 0's chunk
+    good = int(layer.block_table[0, lp_bad])
+    K0 = layer.K[good].clone()
+    layer.block_table[0, lp_bad] = layer.dims.num_phys_pages + 7
+    layer.append(k, v, n)
+    assert bkv.read_device_status() & bkv.DEV_BAD_PAGE
+    assert bkv.read_device_status() == 0  # cleared
+    layer.block_table[0, lp_bad] = good
+    assert torch.equal(layer.K[good], K0), "rows of the bad page were written"
+    for b, L0 in enumerate([5, 37]):
+        toks = np.arange(L0, L0 + n)
+        keep = toks // S != lp_bad if b == 0 else np.ones(n, dtype=bool)
+        phys = layer.block_table[b, toks[keep] // S].long().cpu()
+        rows = torch.as_tensor(toks[keep] % S)
+        assert torch.equal(layer.K[phys, :, rows], k[b, torch.as_tensor(np.nonzero(keep)[0])])
+    assert layer.seq_lens.tolist() == [5 + n, 37 + n]
+    # sequence 0 now ends 10 tokens before its block-table row does
+    cap = layer.dims.max_pages_per_seq * S
+    layer.seq_lens[0] = cap - 10
+    layer.append(k, v, n)
+    assert bkv.read_device_status() & bkv.DEV_OVERFLOW
+    assert layer.seq_lens.tolist() == [cap - 10, 37 + 2 * n]
+    toks = np.arange(37 + n, 37 + 2 * n)
+    phys = layer.block_table[1, toks // S].long().cpu()
+    assert torch.equal(layer.K[phys, :, torch.as_tensor(toks % S)], k[1])
+
+
 @pytest.mark.parametrize("T", [16384, 2048], ids=["p1024", "p128"])
 @pytest.mark.parametrize("levels", [1, 3, 64])
 def test_selection_with_tied_scores(levels, T):
