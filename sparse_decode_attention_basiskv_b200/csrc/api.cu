@@ -364,8 +364,9 @@ int run_append(const basiskv_dims* d, const basiskv_bf16* k_new, const basiskv_b
       cache.key = key;
       cache.valid = true;
     }
-    rc = launch_status(
-        launch_append_tc(a, cache.v, cache.k, cache.w, cache.wk, cache.kc, st, pdl));
+    // the tensor-core kernel advances the lengths itself
+    return launch_status(
+        launch_append_tc(a, cache.v, cache.k, cache.w, cache.wk, cache.kc, bump, st, pdl));
   } else {
     rc = launch_status(launch_append_small(a, st, pdl));
   }

@@ -66,9 +66,12 @@ cudaError_t launch_fold_append(const FoldAppArgs& a, cudaStream_t st, bool pdl);
 // k k-blocks).  tmKc: the bf16 Key cache as [num_phys * Hkv * S][d] (box
 // 8 x 64, 128-byte swizzle), the target of the Key's TMA stores (unused for
 // E4M3 caches).
+// bump: the kernel also advances seq_lens by n_new (its last CTA to read
+// them does it); calls whose launches overlap on the device (other streams)
+// use different arrival slots, up to 64 at once.
 cudaError_t launch_append_tc(const AppendArgs& a, const CUtensorMap& tmV, const CUtensorMap& tmK,
                              const CUtensorMap& tmW, const CUtensorMap& tmWk,
-                             const CUtensorMap& tmKc, cudaStream_t st, bool pdl);
+                             const CUtensorMap& tmKc, bool bump, cudaStream_t st, bool pdl);
 cudaError_t launch_bump_lengths(const AppendArgs& a, cudaStream_t st, bool pdl);
 
 // ------------------------------------------------------------------- route

@@ -133,6 +133,12 @@ constexpr int kTcABytes = kTcBM * kTcBK * 2;  // one ring slot: 128 rows x 128 b
 constexpr int kTcMaxSlots = 12;
 constexpr unsigned long long kTcDrainNs = 10000000ull;  // waits for copies in flight at exit
 
+// Arrival counts for the in-kernel length update, one slot per call in
+// flight (the host hands slots out round-robin): zero when the library
+// loads, and reset by the CTA that completes a call's count.
+constexpr int kTcArriveSlots = 64;
+__device__ unsigned int g_tc_arrive[kTcArriveSlots];
+
 __host__ __device__ constexpr uint32_t tc_idesc(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
@@ -241,7 +247,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      const __grid_constant__ CUtensorMap tmW,
                      const __grid_constant__ CUtensorMap tmWk,
                      const __grid_constant__ CUtensorMap tmKc, AppendArgs a, int N, int tmem_cols,
-                     int slots, int n_mt) {
+                     int slots, int n_mt, int bump_slot) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1k(smem_raw);
   const int d = a.d, nkb = 2 * d / kTcBK;  // k-blocks: first d/64 from v, then from k
@@ -302,6 +308,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp >= 2) {
     for (int i = tid - 64; i < a.B; i += kTcThreads - 64) lens[i] = a.seq_lens[i];
     asm volatile("bar.sync 1, %0;" ::"r"(kTcThreads - 64) : "memory");
+    // The lengths advance once every CTA holds its copy: each CTA arrives
+    // after reading them, and the last to arrive advances them (skipping,
+    // with the overflow bit, a sequence whose chunk does not fit its
+    // block-table row) and resets the count.  Nothing waits here.
+    if (bump_slot >= 0 && tid == 64) {
+      __threadfence();
+      if (atomicAdd(&g_tc_arrive[bump_slot], 1u) == gridDim.x - 1) {
+        __threadfence();
+        const int cap = a.max_pages * a.S;
+        for (int b = 0; b < a.B; ++b) {
+          const int len = lens[b];
+          if (len < 0 || len + a.n_new > cap)
+            raise_status(a.status, BASISKV_DEV_OVERFLOW);
+          else
+            a.seq_lens_out[b] = len + a.n_new;
+        }
+        g_tc_arrive[bump_slot] = 0;
+      }
+    }
   }
 
   if (warp == 0 && lane == 0) {  // ------------------------------------- TMA
@@ -627,7 +652,7 @@ cudaError_t launch_fold_append(const FoldAppArgs& a, cudaStream_t st, bool pdl) 
 
 cudaError_t launch_append_tc(const AppendArgs& a, const CUtensorMap& tmV, const CUtensorMap& tmK,
                              const CUtensorMap& tmW, const CUtensorMap& tmWk,
-                             const CUtensorMap& tmKc, cudaStream_t st, bool pdl) {
+                             const CUtensorMap& tmKc, bool bump, cudaStream_t st, bool pdl) {
   const int N = a.r_v + a.r_k;
   const int acc = N <= 32 ? 32 : (N <= 64 ? 64 : (N <= 128 ? 128 : 256));
   const int tmem_cols = 2 * acc;  // two accumulator buffers
@@ -656,8 +681,10 @@ cudaError_t launch_append_tc(const AppendArgs& a, const CUtensorMap& tmV, const 
   const int rows = a.B * a.n_new;
   const int n_mt = (rows + kTcBM - 1) / kTcBM;
   const int grid = std::min(n_mt * a.Hkv, num_sms());
+  static std::atomic<unsigned> next_slot{0};
+  const int bump_slot = bump ? (int)(next_slot.fetch_add(1) % kTcArriveSlots) : -1;
   return launch_k(append_tc_kernel, dim3(grid), dim3(kTcThreads), smem, st, pdl, tmV, tmK, tmW,
-                  tmWk, tmKc, a, N, tmem_cols, slots, n_mt);
+                  tmWk, tmKc, a, N, tmem_cols, slots, n_mt, bump_slot);
 }
 
 }  // namespace basiskv
