@@ -204,7 +204,10 @@ BASISKV_API int basiskv_fold_append(const basiskv_dims* dims, const basiskv_bf16
  * W_app^T with W_app as built by basiskv_fold_append (W_app may be NULL:
  * the call then folds it into the workspace first); the residual then uses
  * the bf16-rounded fold instead of the unrounded z.  Smaller appends run
- * the two-step CUDA-core form and ignore W_app. */
+ * the two-step CUDA-core form and ignore W_app.  The tensor-core path is
+ * one launch that also advances seq_lens (its last CTA to read them does);
+ * up to 64 such calls may be in flight at once on different streams (each
+ * takes one of 64 device arrival counters in turn; more would share one). */
 BASISKV_API int basiskv_append(const basiskv_dims* dims, const basiskv_bf16* k_new,
                    const basiskv_bf16* v_new, int n_new, int32_t* seq_lens,
                    const int32_t* block_table, const basiskv_bf16* A_V,
