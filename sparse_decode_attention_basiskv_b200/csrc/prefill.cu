@@ -9,9 +9,10 @@
 // (fp32 products, stored bf16) and append_tc_kernel runs the product:
 // 128-token M tiles, N = r_v + r_k, K = 2d, operands staged by TMA in
 // 128-byte-swizzled K-major tiles, a single thread issuing tcgen05.mma
-// (kind::f16, bf16 inputs, fp32 accumulator in tensor memory), and four
+// (kind::f16, bf16 inputs, fp32 accumulator in tensor memory), four
 // epilogue warps that read the accumulator with tcgen05.ld and write the
-// z / e rows, and the exact Key, into the paged caches.  The folded factor
+// z / e rows into the paged caches, and four warps that copy the exact Key
+// there; the same launch advances the sequence lengths.  The folded factor
 // is rounded to bf16 once; the decode-time append (append.cu) keeps the
 // two-step form with an unrounded z.
 #include <algorithm>
@@ -300,8 +301,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
   pdl_wait();
-  // The next launch (the length update) may be scheduled now: it waits for
-  // this grid to complete before it reads or writes anything.
+  // The next launch may be scheduled now: it waits for this grid to
+  // complete before it reads or writes anything.
   pdl_launch_dependents();
   // the epilogue and Key warps read the lengths from shared memory
   int* lens = reinterpret_cast<int*>(smem + L.lens);
