@@ -135,8 +135,10 @@ typedef struct basiskv_dims {
    *     (one block-table entry per page_size tokens), while the router
    *     scores every route_page tokens, and top_k, sink_pages,
    *     recent_pages, the selection and page_scores count routing pages.
-   *     Needs the bf16 caches, a router with a plain-load instance for it
-   *     (listed with basiskv_route), and, for basiskv_decode /
+   *     Needs a router with a routing-page instance: the B16R16 and
+   *     full-width routers at G 4, r_v 64 or 96, page 16 (route_page 4;
+   *     also 8 for B16R16 at r_v 64) and at G 8, r_v 96, page 32
+   *     (route_page 4), over bf16 or E4M3 caches; and, for basiskv_decode /
    *     basiskv_decode_latents, a batch whose (sequence, KV head) groups
    *     fit one wave of the fused selection + attention launch
    *     (basiskv_workspace_size returns 0 otherwise); basiskv_attend does
@@ -230,8 +232,9 @@ BASISKV_API int basiskv_append(const basiskv_dims* dims, const basiskv_bf16* k_n
  *   q            bf16 [B][Hq][d]
  *   seq_lens     int32 [B]; max_seq_len: host bound >= every seq_lens[b]
  *                (used to size the grid; <= max_pages_per_seq*S)
- *   page_scores  fp32 [B][Hkv][max_pages_per_seq] or NULL; entries p >= P_b
- *                are not written
+ *   page_scores  fp32 [B][Hkv][max_pages_per_seq * page_size / route_page]
+ *                (one per routing page) or NULL; entries p >= P_b are not
+ *                written
  *   sel          int32 [B][Hkv][top_k], or NULL to compute the page scores
  *                only (page_scores must then be given)
  * Both outputs NULL is BASISKV_ERR_INVALID_ARG. */

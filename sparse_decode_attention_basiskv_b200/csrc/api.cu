@@ -169,9 +169,11 @@ int check_dims(const basiskv_dims* d) {
   // routing page
   if (d->route_page != 0 && d->route_page != d->page_size) {
     if (d->route_page != 4 && d->route_page != 8) return BASISKV_ERR_INVALID_ARG;
-    if (d->route_page > d->page_size || d->cache_fp8 ||
-        !route_subpage_supported(G, d->r_v, d->r_k, route_rv(d), route_rk(d), d->page_size,
-                                 d->route_page))
+    if (d->route_page > d->page_size ||
+        !(d->cache_fp8 ? route_fp8_subpage_supported(G, d->r_v, d->r_k, route_rv(d),
+                                                     route_rk(d), d->page_size, d->route_page)
+                       : route_subpage_supported(G, d->r_v, d->r_k, route_rv(d), route_rk(d),
+                                                 d->page_size, d->route_page)))
       return BASISKV_ERR_UNSUPPORTED_SHAPE;
   }
   // cache element type

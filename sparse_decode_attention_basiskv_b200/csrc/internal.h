@@ -112,6 +112,7 @@ bool route_subpage_supported(int G, int r_v, int r_k, int rb, int rq, int S, int
 bool route_narrow_supported(int G, int r_v, int r_k, int rb, int rq, int S);
 // Whether it has an instance over E4M3 caches for this router.
 bool route_fp8_supported(int G, int r_v, int r_k, int rb, int rq, int S);
+bool route_fp8_subpage_supported(int G, int r_v, int r_k, int rb, int rq, int S, int rp);
 cudaError_t launch_route_scores_fp8(const RouteArgs& a, cudaStream_t st, bool pdl);
 cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
                                 const CUtensorMap& tmE, int wz, int we, cudaStream_t st,

@@ -583,7 +583,8 @@ cudaError_t launch_route_scores(const RouteArgs& a, const CUtensorMap& tmZ,
                                 const CUtensorMap& tmE, int wz, int we, cudaStream_t st,
                                 bool pdl) {
   if (a.rp && a.rp != a.S) {  // routing pages smaller than the cache page
-    if (a.fp8 || !(a.Z && a.E)) return cudaErrorNotSupported;
+    if (a.fp8) return launch_route_scores_fp8(a, st, pdl);
+    if (!(a.Z && a.E)) return cudaErrorNotSupported;
 #define BKV_RMP(GG, V, K, RB_, RQ_, SS, RP_)                                              \
   if (a.G == GG && a.r_v == V && a.r_k == K && a.rb == RB_ && a.rq == RQ_ && a.S == SS && \
       a.rp == RP_)                                                                       \

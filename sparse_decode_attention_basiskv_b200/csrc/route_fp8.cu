@@ -60,10 +60,15 @@ constexpr int r8_ctas_per_sm() {
              : (r8_live_regs<RB, RQ, S, G>() <= 40 ? 3 : 2);
 }
 
-template <int G, int RV, int RK, int RB, int RQ, int S, int PW>
+// RP: the routing page (RP = S: one score per cache page; RP = 4 or 8: a
+// score for every RP tokens of a cache page, the scores row of a group
+// holding max_pages * S / RP entries).
+template <int G, int RV, int RK, int RB, int RQ, int S, int PW, int RP = S>
 __global__ void __launch_bounds__(kR8Threads, (r8_ctas_per_sm<G, RB, RQ, S>()))
     route_f8_kernel(RouteArgs a) {
   static_assert((G == 4 || G == 8) && S % 16 == 0, "E4M3 scoring shapes");
+  static_assert(RP == S || RP == 4 || RP == 8, "routing pages of 4 or 8 tokens, or the page");
+  constexpr int NR = S / RP;  // routing pages per cache page
   extern __shared__ uint2 r8_frags[];
   constexpr int NZF = RB / 32, NZH = (RB % 32) / 16, NEF = RQ / 32, NEH = (RQ % 32) / 16;
   constexpr int NCZ = NZF + NZH, NC = NCZ + NEF + NEH, NT = S / 8, NM = S / 16, NJ = G / 4;
@@ -173,7 +178,9 @@ __global__ void __launch_bounds__(kR8Threads, (r8_ctas_per_sm<G, RB, RQ, S>()))
       }
     }
   };
-  // This lane's maximum over page k's live tokens and the group's heads.
+  // This lane's maximum over page k's live tokens and the group's heads;
+  // tbest[m][h] keeps it per token (16 m + r + 8 h) for routing pages.
+  float tbest[NM][2];
   auto page_best = [&](const Batch& bt, uint2 (&x)[PW][NT][NC], int k) -> float {
     float acc[NM][NJ][4];
 #pragma unroll
@@ -203,19 +210,52 @@ __global__ void __launch_bounds__(kR8Threads, (r8_ctas_per_sm<G, RB, RQ, S>()))
 #pragma unroll
     for (int mt = 0; mt < NM; ++mt) {
       const int tok = 16 * mt + lr;  // within the page
+      float t0 = -INFINITY, t1 = -INFINITY;
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
-        if (tok < bt.nv[k]) best = fmaxf(best, acc[mt][j][0] + acc[mt][j][1]);
-        if (tok + 8 < bt.nv[k]) best = fmaxf(best, acc[mt][j][2] + acc[mt][j][3]);
+        if (tok < bt.nv[k]) t0 = fmaxf(t0, acc[mt][j][0] + acc[mt][j][1]);
+        if (tok + 8 < bt.nv[k]) t1 = fmaxf(t1, acc[mt][j][2] + acc[mt][j][3]);
       }
+      tbest[mt][0] = t0;
+      tbest[mt][1] = t1;
+      best = fmaxf(best, fmaxf(t0, t1));
     }
     return best * qscale_inv;
+  };
+  // The scores of page k's routing pages (RP < S): token 16 m + r + 8 h
+  // lies in routing page (16 m + 8 h + r) / RP, held by the lanes that
+  // share r / 4 (RP = 4: lane bit 4) or by the whole warp (RP = 8); one
+  // lane per routing page writes it.
+  auto routing_scores = [&](const Batch& bt, int k) {
+#pragma unroll
+    for (int mt = 0; mt < NM; ++mt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float v = tbest[mt][h];
+#pragma unroll
+        for (int o = 1; o < (RP == 8 ? 32 : 16); o <<= 1)
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        const int sub = RP == 8 ? 2 * mt + h : 4 * mt + 2 * h + (lane >> 4);
+        if (RP == 8 ? lane == 0 : (lane & 15) == 0)
+          a.scores[((size_t)bt.bg[k] * a.max_pages + bt.lp[k]) * NR + sub] = v * qscale_inv;
+      }
   };
   auto score = [&](const Batch& bt, uint2 (&x)[PW][NT][NC]) {
     bool one_group = true;
 #pragma unroll
     for (int k = 1; k < PW; ++k) one_group = one_group && (bt.nv[k] == 0 || bt.bg[k] == bt.bg[0]);
-    if (one_group) {  // the common case: the batch's pages are scored side by side
+    if (NR > 1) {  // routing pages smaller than the cache page: one page at a time
+#pragma unroll
+      for (int k = 0; k < PW; ++k) {
+        if (bt.nv[k] == 0) continue;
+        if (bt.bg[k] != frag_bg) {
+          load_frags(bt.bg[k]);
+          frag_bg = bt.bg[k];
+        }
+        (void)page_best(bt, x, k);
+        routing_scores(bt, k);
+      }
+    } else if (one_group) {  // the common case: the batch's pages are scored side by side
       if (bt.bg[0] != frag_bg) {
         load_frags(bt.bg[0]);
         frag_bg = bt.bg[0];
@@ -259,7 +299,7 @@ __global__ void __launch_bounds__(kR8Threads, (r8_ctas_per_sm<G, RB, RQ, S>()))
   }
 }
 
-template <int G, int RV, int RK, int RB, int RQ, int S>
+template <int G, int RV, int RK, int RB, int RQ, int S, int RP = S>
 cudaError_t launch_route_f8(const RouteArgs& a, cudaStream_t st, bool pdl) {
   constexpr int PW = r8_pages_per_batch<RB, RQ, S>();
   const int P_max = (a.max_seq_len + S - 1) / S;
@@ -269,7 +309,7 @@ cudaError_t launch_route_f8(const RouteArgs& a, cudaStream_t st, bool pdl) {
   if (grid > need) grid = need;
   if (grid < 1) grid = 1;
   const size_t smem = (size_t)kR8Warps * ((RB + 31) / 32 + (RQ + 31) / 32) * 2 * (G / 4) * 32 * 8;
-  return launch_k(route_f8_kernel<G, RV, RK, RB, RQ, S, PW>, dim3((unsigned)grid),
+  return launch_k(route_f8_kernel<G, RV, RK, RB, RQ, S, PW, RP>, dim3((unsigned)grid),
                   dim3(kR8Threads), smem, st, pdl, a);
 }
 
@@ -298,8 +338,32 @@ bool route_fp8_supported(int G, int r_v, int r_k, int rb, int rq, int S) {
   return false;
 }
 
+// E4M3 instances with routing pages smaller than the cache page: the
+// routers of the bf16 list that have an E4M3 instance.
+#define BKV_RM8_SUBPAGE(X)                                                            \
+  X(4, 64, 32, 16, 16, 16, 4) X(4, 64, 32, 16, 16, 16, 8) X(4, 96, 32, 16, 16, 16, 4) \
+  X(4, 64, 32, 64, 32, 16, 4) X(4, 96, 32, 96, 32, 16, 4) X(8, 96, 32, 16, 16, 32, 4) \
+  X(8, 96, 32, 96, 32, 32, 4)
+
+bool route_fp8_subpage_supported(int G, int r_v, int r_k, int rb, int rq, int S, int rp) {
+#define BKV_RM8P(GG, V, K, RB_, RQ_, SS, RP_) \
+  if (G == GG && r_v == V && r_k == K && rb == RB_ && rq == RQ_ && S == SS && rp == RP_) return true;
+  BKV_RM8_SUBPAGE(BKV_RM8P)
+#undef BKV_RM8P
+  return false;
+}
+
 cudaError_t launch_route_scores_fp8(const RouteArgs& a, cudaStream_t st, bool pdl) {
   if (!(a.Z && a.E)) return cudaErrorNotSupported;
+  if (a.rp && a.rp != a.S) {  // routing pages smaller than the cache page
+#define BKV_RM8P(GG, V, K, RB_, RQ_, SS, RP_)                                               \
+  if (a.G == GG && a.r_v == V && a.r_k == K && a.rb == RB_ && a.rq == RQ_ && a.S == SS && \
+      a.rp == RP_)                                                                          \
+    return launch_route_f8<GG, V, K, RB_, RQ_, SS, RP_>(a, st, pdl);
+    BKV_RM8_SUBPAGE(BKV_RM8P)
+#undef BKV_RM8P
+    return cudaErrorNotSupported;
+  }
 #define BKV_RM8(GG, V, K, RB_, RQ_, SS)                                                   \
   if (a.G == GG && a.r_v == V && a.r_k == K && a.rb == RB_ && a.rq == RQ_ && a.S == SS) \
     return launch_route_f8<GG, V, K, RB_, RQ_, SS>(a, st, pdl);

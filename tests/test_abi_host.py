@@ -251,9 +251,10 @@ def test_noalloc_reports_the_validation_status(lib):
 
 def test_route_page_validation(lib):
     """Routing pages of 4 or 8 tokens (Table 10's Page4) over cache pages of
-    16 or 32: accepted for routers with such an instance and bf16 caches;
-    other values, E4M3 caches and routers without an instance are refused;
-    the standalone attention takes cache pages only."""
+    16 or 32: accepted for routers with such an instance, bf16 or E4M3
+    (Table 13's B16R16 Page4 over FP8 caches); other values and routers
+    without an instance are refused; the standalone attention takes cache
+    pages only."""
     nar = dict(Hq=8, Hkv=2, r_v=64, r_k=32, route_r_v=16, route_r_k=16, sink_pages=-1,
                recent_pages=4)
     ok = _dims(**nar, route_page=4)
@@ -267,7 +268,9 @@ def test_route_page_validation(lib):
         d = _dims(**nar, route_page=bad)
         assert lib.basiskv_route(ctypes.byref(d), FAKE, FAKE, 256, FAKE, FAKE, FAKE, FAKE, FAKE,
                                  64, None, FAKE, FAKE, 1 << 20, None) == status
-    for d in (_dims(**nar, route_page=4, cache_fp8=1),  # E4M3 caches
+    assert lib.basiskv_workspace_size(ctypes.byref(_dims(**nar, route_page=4, cache_fp8=1)),
+                                      64, 1024) > 0
+    for d in (_dims(**dict(nar, r_v=96), route_page=8, cache_fp8=1),  # no E4M3 instance
               _dims(route_page=4, r_v=32, r_k=16),      # no routing-page instance
               _dims(**nar, route_page=8, page_size=8)):  # not smaller than the page
         assert lib.basiskv_workspace_size(ctypes.byref(d), 64, 1024) == 0
