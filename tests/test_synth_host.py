@@ -39,3 +39,14 @@ def test_paged_keys_view_reads_logical_keys():
     q_log, used_log = synth.make_query(wl, pb.cache["K"], wl.T, step=2)
     q_pag, used_pag = synth.make_query(wl, view, wl.T, step=2)
     assert torch.equal(q_log, q_pag) and torch.equal(used_log, used_pag)
+
+
+def test_tokens_are_dense():
+    """The new tokens are handed to the library as raw pointers: both k and
+    v come back dense and row-major, whatever layout the einsum that builds
+    k picked."""
+    wl = synth.with_sizes(synth.TINY, B=2)
+    factors = synth.make_factors(wl)
+    k, v = synth.make_tokens(wl, factors, 5)
+    assert k.shape == v.shape == (2, 5, wl.Hkv, wl.d)
+    assert k.is_contiguous() and v.is_contiguous()
